@@ -1,0 +1,8 @@
+"""EntroPack fused GPU weight reconstruction for B200 (sm_100a).
+
+The library is ``libentropack.so`` (C ABI, ``include/entropack.h``): a CPU packer
+``ep_encode_tensor`` and the stream-ordered GPU decoder ``ep_decode_tensor``.
+This package is a thin ctypes binding over it; nothing here computes the codec.
+Importing the package does not load the library; the first call does, and it
+raises if the library has not been built.
+"""
