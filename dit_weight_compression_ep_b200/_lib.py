@@ -1,0 +1,212 @@
+"""ctypes binding of libentropack.so (the C ABI of include/entropack.h).
+
+Argument marshalling only: every step of the codec runs inside the library (the
+packer on the host, the decoder in its sm_100a kernel).  PyTorch provides device
+memory and streams.  There is no fallback: if the library has not been built the
+first call raises.
+"""
+from __future__ import annotations
+
+import ctypes as C
+import os
+from dataclasses import dataclass
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+SO_PATH = os.path.join(_HERE, "libentropack.so")
+
+# ep_dtype
+BF16, FP16, FP8_E4M3, INT8, FP32, LATTICE_I32 = 0, 1, 2, 3, 4, 5
+DTYPE_NAMES = {"bf16": BF16, "fp16": FP16, "e4m3": FP8_E4M3, "fp8_e4m3": FP8_E4M3, "int8": INT8, "fp32": FP32,
+               "lattice": LATTICE_I32}
+OUT_BYTES = {BF16: 2, FP16: 2, FP8_E4M3: 1, INT8: 1, FP32: 4, LATTICE_I32: 4}
+
+# ep_status
+STATUS = {0: "EP_OK", 1: "EP_EINVAL", 2: "EP_EUNSUPPORTED", 3: "EP_EALPHABET", 4: "EP_ECUDA", 5: "EP_ECORRUPT",
+          6: "EP_ENOMEM"}
+STATUS_CODES = {v: k for k, v in STATUS.items()}
+
+
+class EntroPackError(RuntimeError):
+    def __init__(self, code: int, what: str):
+        super().__init__(f"{what}: {STATUS.get(code, code)}")
+        self.code = code
+
+
+class _Opts(C.Structure):
+    _fields_ = [
+        ("prob_bits", C.c_int),
+        ("tile_vectors", C.c_int),
+        ("sample_vectors", C.c_int64),
+        ("search_steps", C.c_int),
+        ("seed", C.c_uint64),
+        ("has_container_scales", C.c_int),
+        ("num_threads", C.c_int),
+    ]
+
+
+class _Blob(C.Structure):
+    _fields_ = [
+        ("rows", C.c_int64),
+        ("cols", C.c_int64),
+        ("b", C.c_int),
+        ("V", C.c_int),
+        ("J", C.c_int),
+        ("ntiles", C.c_int),
+        ("payload", C.POINTER(C.c_uint16)),
+        ("payload_words", C.c_size_t),
+        ("payload_alloc_words", C.c_size_t),
+        ("tile_index", C.POINTER(C.c_uint32)),
+        ("freq_tables", C.POINTER(C.c_uint8)),
+        ("freq_bytes", C.c_size_t),
+        ("row_scales", C.POINTER(C.c_float)),
+        ("s", C.c_double),
+        ("stored_bpp", C.c_double),
+        ("stored_bytes", C.c_int64),
+    ]
+
+
+_lib = None
+
+
+def lib() -> C.CDLL:
+    """Load libentropack.so; raise if it is missing (no fallback path exists)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(SO_PATH):
+            raise RuntimeError(f"{SO_PATH} is not built; run `python -m dit_weight_compression_ep_b200.build`")
+        L = C.CDLL(SO_PATH)
+        P = C.c_void_p
+        L.ep_encode_tensor.argtypes = [P, C.c_int64, C.c_int64, C.c_double, C.POINTER(_Opts),
+                                       C.POINTER(C.POINTER(_Blob))]
+        L.ep_encode_tensor.restype = C.c_int
+        L.ep_free_blob.argtypes = [C.POINTER(_Blob)]
+        L.ep_free_blob.restype = None
+        L.ep_decode_tensor.argtypes = [P, P, P, P, P, C.c_int64, C.c_int64, C.c_int, P]
+        L.ep_decode_tensor.restype = C.c_int
+        L.ep_decode_status.argtypes = [P]
+        L.ep_decode_status.restype = C.c_int
+        L.ep_status_string.argtypes = [C.c_int]
+        L.ep_status_string.restype = C.c_char_p
+        _lib = L
+    return _lib
+
+
+EXPORTED = ("ep_encode_tensor", "ep_free_blob", "ep_decode_tensor", "ep_decode_status", "ep_status_string")
+
+
+@dataclass
+class Blob:
+    """Host copy of a compressed tensor (the packer's output)."""
+
+    rows: int
+    cols: int
+    b: int
+    V: int
+    ntiles: int
+    payload: np.ndarray       # uint16, padded with zero words to a multiple of 8
+    payload_words: int        # stored words (the final offset)
+    tile_index: np.ndarray    # uint32 [33*T + 1]
+    freq_tables: np.ndarray   # uint8
+    row_scales: np.ndarray    # float32 [rows]
+    s: float = 0.0
+    stored_bpp: float = 0.0
+    stored_bytes: int = 0
+
+    @property
+    def numel(self) -> int:
+        return self.rows * self.cols
+
+    def stored_device_bytes(self) -> int:
+        """Bytes the decoder reads: payload + tile index + tables + row scales."""
+        return 2 * self.payload_words + 4 * self.tile_index.size + self.freq_tables.size + 4 * self.rows
+
+    @staticmethod
+    def from_arrays(payload, tile_index, freq_tables, row_scales, rows: int, cols: int) -> "Blob":
+        """Wrap stored arrays produced elsewhere (e.g. read from a file)."""
+        payload = np.asarray(payload, np.uint16).reshape(-1)
+        words = payload.size
+        pad = (-words) % 8
+        padded = np.concatenate([payload, np.zeros(pad, np.uint16)]) if pad else payload.copy()
+        ft = np.ascontiguousarray(freq_tables, np.uint8)
+        h = ft[:24].view(np.uint32)
+        return Blob(rows, cols, int(h[2]), int(h[3]), int(h[5]), padded, words,
+                    np.ascontiguousarray(tile_index, np.uint32), ft, np.ascontiguousarray(row_scales, np.float32))
+
+
+def encode_tensor(W: np.ndarray, target_bpp: float, *, prob_bits: int = 0, tile_vectors: int = 0,
+                  sample_vectors: int = 0, search_steps: int = 0, seed: int = 0,
+                  has_container_scales: bool = False, num_threads: int = 0) -> Blob:
+    """Compress a host float32 matrix with the library's CPU packer (ep_encode_tensor)."""
+    W = np.ascontiguousarray(W, np.float32)
+    if W.ndim != 2:
+        raise ValueError("W must be 2-D")
+    o = _Opts(prob_bits, tile_vectors, sample_vectors, search_steps, seed, int(has_container_scales), num_threads)
+    out = C.POINTER(_Blob)()
+    rc = lib().ep_encode_tensor(W.ctypes.data, W.shape[0], W.shape[1], float(target_bpp), C.byref(o), C.byref(out))
+    if rc:
+        raise EntroPackError(rc, "ep_encode_tensor")
+    try:
+        b = out.contents
+        T = b.ntiles
+        payload = np.ctypeslib.as_array(b.payload, shape=(b.payload_alloc_words,)).copy() if b.payload_alloc_words \
+            else np.zeros(0, np.uint16)
+        tix = np.ctypeslib.as_array(b.tile_index, shape=(33 * T + 1,)).copy()
+        ft = np.ctypeslib.as_array(b.freq_tables, shape=(b.freq_bytes,)).copy()
+        rs = np.ctypeslib.as_array(b.row_scales, shape=(b.rows,)).copy()
+        return Blob(b.rows, b.cols, b.b, b.V, T, payload, int(b.payload_words), tix, ft, rs, b.s, b.stored_bpp,
+                    int(b.stored_bytes))
+    finally:
+        lib().ep_free_blob(out)
+
+
+class DeviceBlob:
+    """A compressed tensor resident in GPU memory (torch tensors own the buffers)."""
+
+    def __init__(self, blob: Blob, device="cuda"):
+        import torch
+
+        self.rows, self.cols, self.b, self.V, self.ntiles = blob.rows, blob.cols, blob.b, blob.V, blob.ntiles
+        pay = blob.payload if blob.payload.size else np.zeros(8, np.uint16)
+        self.payload = torch.from_numpy(pay.view(np.int16)).to(device)
+        self.tile_index = torch.from_numpy(blob.tile_index.view(np.int32)).to(device)
+        self.freq_tables = torch.from_numpy(blob.freq_tables).to(device)
+        self.row_scales = torch.from_numpy(blob.row_scales).to(device)
+        self.read_bytes = blob.stored_device_bytes()
+
+
+def _torch_dtype(dt: int):
+    import torch
+
+    return {BF16: torch.bfloat16, FP16: torch.float16, FP8_E4M3: torch.float8_e4m3fn, INT8: torch.int8,
+            FP32: torch.float32, LATTICE_I32: torch.int32}[dt]
+
+
+def decode_tensor(db: DeviceBlob, out_dtype: int = BF16, out=None, stream=None):
+    """Launch ep_decode_tensor on `stream` (default: torch's current stream); returns `out`."""
+    import torch
+
+    if out is None:
+        out = torch.empty((db.rows, db.cols), dtype=_torch_dtype(out_dtype), device=db.payload.device)
+    st = stream if stream is not None else torch.cuda.current_stream(db.payload.device)
+    rc = lib().ep_decode_tensor(C.c_void_p(st.cuda_stream), db.payload.data_ptr(), db.tile_index.data_ptr(),
+                                db.freq_tables.data_ptr(), db.row_scales.data_ptr(), db.rows, db.cols,
+                                int(out_dtype), out.data_ptr())
+    if rc:
+        raise EntroPackError(rc, "ep_decode_tensor")
+    return out
+
+
+def decode_status(stream=None) -> int:
+    """Synchronise the stream and read (and clear) the device status word; returns the ep_status code."""
+    import torch
+
+    st = stream if stream is not None else torch.cuda.current_stream()
+    return int(lib().ep_decode_status(C.c_void_p(st.cuda_stream)))
+
+
+def check_status(stream=None) -> None:
+    rc = decode_status(stream)
+    if rc:
+        raise EntroPackError(rc, "decode")

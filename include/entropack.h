@@ -1,0 +1,150 @@
+/*
+ * entropack.h -- C ABI of the EntroPack codec for B200 (sm_100a).
+ *
+ * EntroPack ("EntroPack: Fast and Accurate Entropy-Coded Weight Compression at
+ * Arbitrary Bitrates") stores a weight matrix as independently decodable rANS
+ * tiles of coset-conditioned E8-lattice fields, one FP32 reconstruction scale
+ * per row, and seventeen frequency tables (§3.6 "Stored representation").
+ * This library offers:
+ *   ep_encode_tensor  -- the CPU packer (§3.1 pipeline, §3.4 scale search,
+ *                        §3.5 refit, §3.6 tiles; App. C.1, C.3), threaded;
+ *   ep_decode_tensor  -- the fused GPU reconstruction (Fig. 2b; §3.6 "one tile
+ *                        to a GPU warp and one state to each lane"; App. C.3),
+ *                        stream-ordered, one kernel launch per call.
+ *
+ * Stored representation (all little-endian; the packer writes it, the decoder
+ * reads it):
+ *   payload      uint16 words of all tiles, concatenated.
+ *   tile_index   uint32[33*T + 1]: for tile t, [33t] = payload offset of the
+ *                tile (in 16-bit words), [33t+1+j] = terminal rANS state of
+ *                lane j (j < 32); [33T] = final boundary offset = payload size.
+ *                (App. C.3: J = 32 states and one 32-bit offset per tile.)
+ *   freq_tables  48-byte header {u32 magic 0x314B5045 "EPK1", u32 version 1,
+ *                u32 b, u32 V, u32 J = 32, u32 T, i64 rows, i64 cols,
+ *                u32 ntables = 17, u32 flags = 0}, then 17 x {i32 min, u32 A},
+ *                zero padding to a multiple of 16 bytes, then the uint16
+ *                frequencies of every table in table order (A per table).
+ *                Table 0 codes the coset bit c; table 1 + 2(k-1) + c codes field
+ *                k (z1..z7, then m) of a vector in coset c (App. A.3).
+ *   row_scales   float32[rows]: reconstruction scale of each row.
+ * Vector g (8 consecutive weights of a row, g = row*cols/8 + col/8) lies in tile
+ * g / V, on lane (g mod V) mod 32, round (g mod V) / 32 (the lane interleave).
+ */
+#ifndef ENTROPACK_H
+#define ENTROPACK_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Output element types of the decoder. */
+typedef enum {
+    EP_BF16 = 0,        /* bfloat16, round to nearest even */
+    EP_FP16 = 1,        /* IEEE binary16, round to nearest even, overflow to inf */
+    EP_FP8_E4M3 = 2,    /* OCP FP8 E4M3 ("fn"), round to nearest even, saturating to +-448 */
+    EP_INT8 = 3,        /* nearest-even integer, clamped to [-127, 127] */
+    EP_FP32 = 4,        /* the FP32 product itself */
+    EP_LATTICE_I32 = 5  /* int32 2y (twice the lattice coordinates), for verification */
+} ep_dtype;
+
+typedef enum {
+    EP_OK = 0,
+    EP_EINVAL = 1,        /* a null pointer, a bad size, a misaligned buffer */
+    EP_EUNSUPPORTED = 2,  /* cols % 8 != 0, an unknown dtype, a format variant the GPU does not decode */
+    EP_EALPHABET = 3,     /* the packer could not fit the alphabets (should not happen) */
+    EP_ECUDA = 4,         /* a CUDA runtime error at launch */
+    EP_ECORRUPT = 5,      /* the device found an inconsistent stream or table header */
+    EP_ENOMEM = 6         /* host allocation failed in the packer */
+} ep_status;
+
+/* Packer options; zero-initialise and set what you need. */
+typedef struct {
+    int prob_bits;            /* starting precision b in [9, 15]; 0: 11 for targets <= 7 bpp, else 12 (App. C.1) */
+    int tile_vectors;         /* V; 0: max(32, floor(S/9)), S = 32768 / 16384 / 8192 / 4096 by target (Table 5) */
+    int64_t sample_vectors;   /* rate-estimation sample; 0: 2^18 vectors of complete rows (App. C.1) */
+    int search_steps;         /* geometric bisection steps; 0: 12 (App. C.1) */
+    uint64_t seed;            /* sample seed; 0: derived from the shape */
+    int has_container_scales; /* 1: count 4 bytes per row of FP8/INT8 container scales in the rate */
+    int num_threads;          /* 0: all hardware threads */
+} ep_encode_opts;
+
+/* The packer's output; host memory owned by the library, freed by ep_free_blob. */
+typedef struct {
+    int64_t rows, cols;
+    int b;                 /* probability precision, M = 2^b */
+    int V;                 /* vectors per tile */
+    int J;                 /* 32 */
+    int ntiles;            /* T */
+    uint16_t* payload;     /* payload_words words, followed by zero words up to a multiple of 8 */
+    size_t payload_words;  /* the stored payload (= tile_index[33T]) */
+    size_t payload_alloc_words; /* payload_words rounded up to a multiple of 8 */
+    uint32_t* tile_index;  /* 33*T + 1 words */
+    uint8_t* freq_tables;  /* freq_bytes bytes */
+    size_t freq_bytes;
+    float* row_scales;     /* rows floats */
+    double s;              /* selected quantisation scale */
+    double stored_bpp;     /* 8 * stored_bytes / (rows*cols)  ([paper] §4.1 "Metrics") */
+    int64_t stored_bytes;  /* payload + tile metadata + tables + row scales (+ container scales) */
+} ep_blob;
+
+/*
+ * ep_encode_tensor -- compress W (host, row-major float32 [rows, cols], the
+ * container's values) to about target_bpp stored bits per weight.
+ * Follows §3.1: row normalisation, sampled-row scale search (§3.4, App. C.1),
+ * E8 quantisation, row-scale refit (§3.5), seventeen tables and tiled
+ * interleaved rANS (§3.6, App. C.3).  Runs on the host with num_threads threads.
+ * opts may be NULL.  On EP_OK *out holds a new blob (free with ep_free_blob).
+ * Errors: EP_EINVAL (null W/out, rows or cols <= 0, target_bpp <= 0, b out of
+ * [9, 15]), EP_EUNSUPPORTED (cols % 8 != 0), EP_EALPHABET, EP_ENOMEM.
+ */
+ep_status ep_encode_tensor(const float* W, int64_t rows, int64_t cols, double target_bpp,
+                           const ep_encode_opts* opts, ep_blob** out);
+
+/* Free a blob returned by ep_encode_tensor (NULL is allowed). */
+void ep_free_blob(ep_blob* blob);
+
+/*
+ * ep_decode_tensor -- reconstruct the dense [rows, cols] matrix on the GPU
+ * (Fig. 2b: symbol decode, lattice reconstruction, row rescale, dtype
+ * conversion fused in one pass; App. C.3 tile layout).
+ *   stream       cudaStream_t to launch on (NULL: the legacy default stream).
+ *   tiles        device, the payload; 16-byte aligned; the buffer must be
+ *                readable up to the final offset rounded up to a multiple of 8
+ *                words (the packer's payload_alloc_words).
+ *   tile_index   device, uint32[33*T + 1], 4-byte aligned.
+ *   freq_tables  device, the table header and frequencies, 16-byte aligned.
+ *   row_scales   device, float32[rows].
+ *   rows, cols   the matrix shape; must match the header.
+ *   out_dtype    one of ep_dtype.
+ *   out          device, rows*cols elements of out_dtype, row-major, 16-byte aligned.
+ * All buffers belong to the caller; the library allocates no device memory.
+ * The call is asynchronous: it validates the arguments on the host, launches
+ * one kernel on the stream and returns.  Argument errors return at once
+ * (EP_EINVAL, EP_EUNSUPPORTED), launch errors as EP_ECUDA.  The stream itself
+ * is checked on the device without trapping: a corrupt payload, state, offset
+ * or table raises a device-side status word that ep_decode_status reads.
+ * Outputs of a corrupt tile are unspecified; no access leaves the buffers
+ * described above.
+ */
+ep_status ep_decode_tensor(void* stream, const uint16_t* tiles, const uint32_t* tile_index,
+                           const uint8_t* freq_tables, const float* row_scales, int64_t rows,
+                           int64_t cols, ep_dtype out_dtype, void* out);
+
+/*
+ * ep_decode_status -- synchronise `stream`, read and clear the status word of
+ * the current device: EP_OK, EP_ECORRUPT (an inconsistent stream or header),
+ * or EP_EUNSUPPORTED (a header variant the GPU decoder does not handle).
+ * The word is shared by every decode on the device since the last read.
+ */
+ep_status ep_decode_status(void* stream);
+
+/* A static description of a status code. */
+const char* ep_status_string(ep_status s);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* ENTROPACK_H */

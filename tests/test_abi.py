@@ -1,0 +1,80 @@
+"""The C ABI library loads on a host without a GPU, exports every entry point
+include/*.h declares, and rejects bad arguments on the host before any CUDA call."""
+import ctypes as C
+import glob
+import os
+import re
+
+import numpy as np
+import pytest
+
+import dit_weight_compression_ep_b200 as ep
+from dit_weight_compression_ep_b200 import build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build.build()
+    return ep.lib()
+
+
+def _declared():
+    names = set()
+    for h in glob.glob(os.path.join(ROOT, "include", "*.h")):
+        src = open(h).read()
+        src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+        src = re.sub(r"//[^\n]*", "", src)
+        for m in re.finditer(r"\b(ep_[a-z0-9_]+)\s*\(", src):
+            names.add(m.group(1))
+    return names
+
+
+def test_exports_every_declared_symbol(lib):
+    names = _declared()
+    assert {"ep_encode_tensor", "ep_free_blob", "ep_decode_tensor", "ep_decode_status", "ep_status_string"} <= names
+    for n in sorted(names):
+        assert hasattr(lib, n), n
+
+
+def test_status_strings(lib):
+    for code in range(7):
+        assert lib.ep_status_string(code)
+
+
+def test_decode_rejects_bad_arguments_on_host(lib):
+    good = C.c_void_p(0x10000)
+    args = [None, good, good, good, good, 64, 64, ep.BF16, good]
+    EINVAL, EUNSUP = ep._lib.STATUS_CODES["EP_EINVAL"], ep._lib.STATUS_CODES["EP_EUNSUPPORTED"]
+    for i in (1, 2, 3, 4, 8):  # null buffers
+        a = list(args)
+        a[i] = None
+        assert lib.ep_decode_tensor(*a) == EINVAL
+    a = list(args)
+    a[6] = 60                   # cols % 8 != 0
+    assert lib.ep_decode_tensor(*a) == EUNSUP
+    a = list(args)
+    a[7] = 9                    # unknown dtype
+    assert lib.ep_decode_tensor(*a) == EUNSUP
+    a = list(args)
+    a[5] = 0                    # rows <= 0
+    assert lib.ep_decode_tensor(*a) == EINVAL
+    a = list(args)
+    a[1] = C.c_void_p(0x10008)  # payload not 16-byte aligned
+    assert lib.ep_decode_tensor(*a) == EINVAL
+    a = list(args)
+    a[8] = C.c_void_p(0x10004)  # output not 16-byte aligned
+    assert lib.ep_decode_tensor(*a) == EINVAL
+
+
+def test_encode_rejects_bad_arguments(lib):
+    W = np.zeros((4, 16), np.float32)
+    with pytest.raises(ep.EntroPackError):
+        ep.encode_tensor(np.zeros((4, 12), np.float32), 4.0)     # cols % 8
+    with pytest.raises(ep.EntroPackError):
+        ep.encode_tensor(W, 0.0)
+    with pytest.raises(ep.EntroPackError):
+        ep.encode_tensor(W, 4.0, prob_bits=16)
+    with pytest.raises(ep.EntroPackError):
+        ep.encode_tensor(W, 4.0, prob_bits=8)

@@ -1,0 +1,257 @@
+"""GPU parity: ep_decode_tensor (through the C ABI) against the CPU oracle.
+
+Inputs are seeded synthetic tensors; streams come from the oracle's encoder for
+the small cases and from the library's packer (byte-identical to the oracle's
+encoder, see test_packer.py) for the full-size workloads.  Expected values come
+only from the oracle's decoder.  The comparison is bit-exact for every output
+type (the spec allows 1 ulp for floating outputs; the single-rounding FFMA design
+reaches exact equality).
+"""
+import numpy as np
+import pytest
+
+import oracle
+import dit_weight_compression_ep_b200 as ep
+from dit_weight_compression_ep_b200 import synth
+from gpu_util import as_lib_blob, assert_parity, oracle_decode, to_raw
+
+pytestmark = pytest.mark.gpu
+
+ALL_DT = [ep.BF16, ep.FP16, ep.FP8_E4M3, ep.INT8, ep.FP32, ep.LATTICE_I32]
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _cuda():
+    import torch
+
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    from dit_weight_compression_ep_b200 import build
+
+    build.build()
+    ep.lib()
+    ep.decode_status()  # clear the status word
+
+
+def _gpu(blob, dt, stream=None):
+    db = ep.DeviceBlob(blob)
+    out = ep.decode_tensor(db, dt, stream=stream)
+    rc = ep.decode_status(stream)
+    assert rc == 0, f"device status {rc}"
+    return to_raw(out)
+
+
+def _check(blob, dts=ALL_DT, what=""):
+    for dt in dts:
+        assert_parity(_gpu(blob, dt), oracle_decode(blob, dt), dt, f"{what} dt={dt}")
+
+
+# ---------------------------------------------------------------- small cases
+
+def test_small_fp32_all_dtypes():
+    W = synth.generate(synth.small_fp32())
+    ob = oracle.encode(W, 4.0, prob_bits=12, tile_vectors=512)
+    assert ob.ntiles == 32 and ob.b == 12
+    _check(as_lib_blob(ob), what="256x512 fp32")
+
+
+@pytest.mark.parametrize("b", [9, 10, 11, 12, 13, 15])
+@pytest.mark.parametrize("V", [32, 33, 100, 455])
+def test_precisions_and_tile_sizes(b, V):
+    rng = np.random.default_rng(100 * b + V)
+    W = (rng.standard_normal((96, 1024)) * 0.02 * np.exp(rng.normal(0, 0.4, (96, 1)))).astype(np.float32)
+    ob = oracle.encode(W, 4.0 if b <= 11 else 7.5, prob_bits=b, tile_vectors=V)
+    assert ob.b == b
+    _check(as_lib_blob(ob), [ep.BF16, ep.INT8, ep.LATTICE_I32], f"b={b} V={V}")
+
+
+@pytest.mark.parametrize("rows,cols,V", [(1, 8, 32), (1, 256, 1), (3, 64, 32), (5, 24, 7), (17, 8, 50),
+                                         (40, 2048, 1820), (7, 4096, 3640)])
+def test_shapes(rows, cols, V):
+    rng = np.random.default_rng(rows * cols + V)
+    W = (rng.standard_t(5, (rows, cols)) * 0.02).astype(np.float32)
+    ob = oracle.encode(W, 5.0, tile_vectors=V)
+    _check(as_lib_blob(ob), [ep.BF16, ep.FP32, ep.LATTICE_I32], f"{rows}x{cols} V={V}")
+
+
+def test_one_coset_and_wide_alphabet():
+    # every vector in D8 (the c = 1 tables are empty) and a coordinate alphabet of exactly 2^b
+    b = 9
+    M = 1 << b
+    nvec = 6 * M
+    z = np.zeros((nvec, 8))
+    z[:, 0] = np.tile(np.arange(M), 6) - M // 2
+    z[:, 1:7] = np.random.default_rng(1).integers(-3, 4, (nvec, 6))
+    z[:, 7] = z[:, :7].sum(axis=1) % 2
+    f = oracle.fields_of(z, np.zeros(nvec, np.int32))
+    rows, cols = 12, 8 * nvec // 12
+    rs = np.linspace(0.01, 0.1, rows).astype(np.float32)
+    ob = oracle.encode_fields(f, rows, cols, rs, b, 200)
+    _check(as_lib_blob(ob), ALL_DT, "one coset, A = 2^b")
+
+
+def test_zero_rows_and_signed_zeros():
+    rng = np.random.default_rng(3)
+    W = (rng.standard_normal((64, 512)) * 0.05).astype(np.float32)
+    W[3] = 0
+    W[10] = -W[10]
+    ob = oracle.encode(W, 3.0, tile_vectors=64)
+    _check(as_lib_blob(ob), ALL_DT, "zero rows")
+
+
+def test_tiny_and_negative_scales():
+    # rows whose reconstruction scale is subnormal, zero or negative take the exact slow path
+    rng = np.random.default_rng(4)
+    W = (rng.standard_normal((32, 256)) * 0.05).astype(np.float32)
+    ob = oracle.encode(W, 4.0, tile_vectors=64)
+    rs = ob.row_scales.copy()
+    rs[0] = np.float32(1e-39)
+    rs[1] = np.float32(-3e-38)
+    rs[2] = np.float32(0.0)
+    rs[3] = np.float32(-0.5)
+    rs[4] = np.float32(2.0 ** -125)
+    blob = ep.Blob.from_arrays(ob.payload, ob.tile_index, ob.freq_tables, rs, ob.rows, ob.cols)
+    _check(blob, ALL_DT, "tiny scales")
+
+
+def test_repeat_on_side_stream():
+    import torch
+
+    W = synth.generate(synth.small_fp32(seed=11))
+    blob = ep.encode_tensor(W, 4.0)
+    s = torch.cuda.Stream()
+    with torch.cuda.stream(s):
+        a = _gpu(blob, ep.BF16, stream=s)
+        b = _gpu(blob, ep.BF16, stream=s)
+    np.testing.assert_array_equal(a, b)
+    assert_parity(a, oracle_decode(blob, ep.BF16), ep.BF16, "side stream")
+
+
+# ------------------------------------------------------------ corrupt streams
+
+def _status_of(blob):
+    db = ep.DeviceBlob(blob)
+    ep.decode_tensor(db, ep.BF16)
+    return ep.decode_status()
+
+
+def test_corruption_sets_status_without_fault():
+    rng = np.random.default_rng(9)
+    W = (rng.standard_normal((128, 1024)) * 0.02).astype(np.float32)
+    good = ep.encode_tensor(W, 4.0, tile_vectors=200)
+    assert _status_of(good) == 0
+
+    def variant(**kw):
+        d = dict(payload=good.payload.copy(), tile_index=good.tile_index.copy(),
+                 freq_tables=good.freq_tables.copy(), row_scales=good.row_scales.copy())
+        d.update(kw)
+        b = ep.Blob(good.rows, good.cols, good.b, good.V, good.ntiles, d["payload"], good.payload_words,
+                    d["tile_index"], d["freq_tables"], d["row_scales"])
+        return b
+
+    p = good.payload.copy()
+    p[good.payload_words // 2] ^= 0x1234
+    assert _status_of(variant(payload=p)) == ep._lib.STATUS_CODES["EP_ECORRUPT"]
+    t = good.tile_index.copy()
+    t[1 + 33 * 3] = 7                       # a state below 2^15
+    assert _status_of(variant(tile_index=t)) == ep._lib.STATUS_CODES["EP_ECORRUPT"]
+    t = good.tile_index.copy()
+    t[33 * 2] = t[33 * 3] + 5               # offsets out of order
+    assert _status_of(variant(tile_index=t)) == ep._lib.STATUS_CODES["EP_ECORRUPT"]
+    t = good.tile_index.copy()
+    t[33 * 4] = 0                           # a truncated tile
+    assert _status_of(variant(tile_index=t)) == ep._lib.STATUS_CODES["EP_ECORRUPT"]
+    ft = good.freq_tables.copy()
+    ft[0] ^= 0xFF                           # bad magic
+    assert _status_of(variant(freq_tables=ft)) == ep._lib.STATUS_CODES["EP_ECORRUPT"]
+    ft = good.freq_tables.copy()
+    ft[8:12] = np.array([16], np.uint32).view(np.uint8)   # b > 15
+    assert _status_of(variant(freq_tables=ft)) == ep._lib.STATUS_CODES["EP_ECORRUPT"]
+    ft = good.freq_tables.copy()
+    ft[-2:] = np.array([ft[-2:].view(np.uint16)[0] + 1], np.uint16).view(np.uint8)  # sum != 2^b
+    assert _status_of(variant(freq_tables=ft)) == ep._lib.STATUS_CODES["EP_ECORRUPT"]
+    ft = good.freq_tables.copy()
+    ft[44:48] = np.array([1], np.uint32).view(np.uint8)   # an ablation variant the GPU does not decode
+    assert _status_of(variant(freq_tables=ft)) == ep._lib.STATUS_CODES["EP_EUNSUPPORTED"]
+    # the device stays usable: a good stream still decodes exactly
+    assert _status_of(good) == 0
+    assert_parity(_gpu(good, ep.BF16), oracle_decode(good, ep.BF16), ep.BF16, "after corruption")
+
+
+# ---------------------------------------------------- full-size workloads
+
+def _full_check(blob, dts, what, sample_tiles=None):
+    """Full oracle decode, or (sample_tiles) a seeded sample of tiles + first/last."""
+    db = ep.DeviceBlob(blob)
+    for dt in dts:
+        out = ep.decode_tensor(db, dt)
+        assert ep.decode_status() == 0
+        got = to_raw(out).reshape(-1)
+        if sample_tiles is None:
+            assert_parity(got, oracle_decode(blob, dt), dt, what)
+        else:
+            rng = np.random.default_rng(12345)
+            tiles = sorted(set([0, blob.ntiles - 1] + list(rng.choice(blob.ntiles, sample_tiles, replace=False))))
+            per = 8 * blob.V
+            for t in tiles:
+                lo = t * per
+                hi = min(lo + per, blob.rows * blob.cols)
+                assert_parity(got[lo:hi], oracle_decode(blob, dt, t, t + 1), dt, f"{what} tile {t}")
+        del out
+
+
+def test_headline_3840x10240_bf16_4bpp():
+    W = synth.generate(synth.headline())
+    blob = ep.encode_tensor(W, 4.0)
+    assert blob.b == 11 and blob.V == 1820 and blob.ntiles == 2701
+    _full_check(blob, [ep.BF16, ep.FP16], "headline")
+    # property at full size: every decoded point lies in E8
+    import torch
+
+    y2 = ep.decode_tensor(ep.DeviceBlob(blob), ep.LATTICE_I32).view(-1, 8).to(torch.int64)
+    par = y2 & 1
+    assert bool((par == par[:, :1]).all()) and bool(((y2.sum(dim=1) // 2) % 2 == 0).all())
+
+
+def test_dit_attention_projection_5bpp():
+    W = synth.generate(synth.dit_attn_proj())
+    blob = ep.encode_tensor(W, 5.0)
+    _full_check(blob, [ep.BF16, ep.FP16], "attn proj")
+
+
+def test_fp8_and_int8_containers_5bpp():
+    src = synth.generate(synth.lowp_source())
+    for kind in ("e4m3", "int8"):
+        vals, scales = synth.to_e4m3_container(src) if kind == "e4m3" else synth.to_int8_container(src)
+        blob = ep.encode_tensor(vals, 5.0, has_container_scales=True)
+        assert abs(blob.stored_bpp / 5.0 - 1) < 0.03
+        dt = ep.FP8_E4M3 if kind == "e4m3" else ep.INT8
+        _full_check(blob, [dt], kind)
+
+
+@pytest.mark.parametrize("wide", [True, False])
+def test_llm_prefill_sweep_sampled(wide):
+    W = synth.generate(synth.llm_prefill(wide))
+    prev = None
+    for bpp in (2, 3, 4, 5, 6, 7, 8):
+        blob = ep.encode_tensor(W, float(bpp))
+        assert abs(blob.stored_bpp / bpp - 1) < 0.03
+        _full_check(blob, [ep.BF16], f"llm {wide} {bpp}", sample_tiles=24)
+        import torch
+
+        out = ep.decode_tensor(ep.DeviceBlob(blob), ep.FP32)
+        Wt = torch.from_numpy(W).cuda()
+        rel = float(torch.linalg.vector_norm(out - Wt) / torch.linalg.vector_norm(Wt))
+        if prev is not None:
+            assert rel < prev
+        prev = rel
+        del out, Wt
+
+
+def test_dit_stack_layers_sampled():
+    alloc = synth.dit_stack_bpp()
+    for kind in synth.DIT_KINDS:
+        blk = 7
+        W = synth.generate(synth.dit_stack_layer(blk, kind))
+        blob = ep.encode_tensor(W, alloc[(blk, kind)])
+        _full_check(blob, [ep.BF16], f"dit {kind}", sample_tiles=16)
