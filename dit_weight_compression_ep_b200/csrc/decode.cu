@@ -295,13 +295,13 @@ struct CoarseLut {
             const int t = 1 + 2 * (K - 1) + (int)((cb - lut_s) >> (nb_shift + 3));
             const int mn = s_min[t];
             const uint32_t A = s_A[t], off = s_off[t];
-            const uint32_t lim = 1u << sh;
-            uint32_t it = 0;
+            // the walk may cross zero-frequency symbols (unobserved values inside
+            // the alphabet), so it is bounded by the alphabet, not by the bucket width
             while (slot >= c0 + f) {
                 c0 += f;
                 ++z;
                 const uint32_t s = (uint32_t)(z - mn);
-                if (s >= A || ++it > lim) {
+                if (s >= A) {
                     bad = true;
                     f = 1u;
                     c0 = slot;
