@@ -1,0 +1,393 @@
+"""Benchmark of the fused EntroPack decode on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+One step = one ep_decode_tensor call: the whole hot path (tile setup, table
+staging, payload staging, rANS decode, lattice reconstruction, row rescale,
+conversion and store) over the 3840x10240 bf16 Student-t(6)*0.02 weight matrix
+(the DiT FFN down-projection shape) compressed at 4 bpp, decoded to bf16.
+Inputs are resident in HBM; steps rotate over 4 copies of (stream, output) so
+the working set (4 x ~98 MB) exceeds the 126 MB L2.  Multi-GPU: every rank
+decodes its own copy (independent tensors, no collective on the data path);
+the value is the weights of all ranks over the slowest rank's time.
+
+Prints one JSON line on rank 0.  --impl reference times the CPU oracle instead
+(the plain C decoder, threads over tile ranges) on a bounded sample of the same
+stream.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+from types import SimpleNamespace
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "decoded G weights/s and achieved HBM GB/s vs B200 peak (BF16 out, 4 bpp)"
+UNIT = "G weights/s"
+ROWS, COLS, TARGET = 3840, 10240, 4.0
+WORKLOAD = "3840x10240 bf16 Student-t(6)*0.02 weight (DiT FFN down projection), 4 bpp, decode to bf16"
+# the pages' 0.23 ms for a 39.3 M-weight layer, BF16 out, 4 bpp, on one H20 (context only)
+PAGES_GWPS = 39321600 / 0.23e-3 / 1e9
+ROTATE = 4
+L2_BYTES = 126 * 1024 * 1024
+
+
+def _peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    except Exception:
+        return 6650.0, "fallback"
+
+
+def _kernel_sha():
+    h = hashlib.sha256()
+    for p in ("dit_weight_compression_ep_b200/csrc/decode.cu", "dit_weight_compression_ep_b200/csrc/ep_format.h"):
+        with open(os.path.join(ROOT, p), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def _traffic_per_launch():
+    """DRAM bytes per launch from the committed ncu summary, if it was taken on this kernel source."""
+    try:
+        with open(os.path.join(ROOT, "profiles", "decode_headline_traffic.json")) as f:
+            d = json.load(f)
+        if d.get("kernel_sha") == _kernel_sha():
+            return float(d["dram_bytes_per_launch"])
+    except Exception:
+        pass
+    return None
+
+
+class Clocks:
+    """nvidia-smi samples (SM clock, throttle reasons) taken while the benchmark runs."""
+
+    Q = ("timestamp,index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.rows = []
+        self.proc = None
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", f"--query-gpu={self.Q}", "--format=csv,noheader,nounits",
+                                          "-lms", "50", "-i", str(index)], stdout=subprocess.PIPE,
+                                         stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+        except Exception:
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.rows.append((time.time(), [c.strip() for c in line.split(",")]))
+
+    def stop(self):
+        if self.proc:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+
+    def summary(self, t0: float, t1: float):
+        if not self.rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        inside = [r for t, r in self.rows if t0 <= t <= t1]
+        window = "timed region"
+        if len(inside) < 3:
+            inside = [r for _, r in self.rows]
+            window = "whole run (timed region shorter than the sampling period)"
+        sm = [float(r[2]) for r in inside if r[2].replace(".", "").isdigit()]
+        mx = [float(r[3]) for r in inside if r[3].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in inside for i in range(4) if len(r) > 6 + i and r[6 + i] == "Active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": reasons, "samples": len(inside), "window": window}
+
+
+def _make_weights():
+    from dit_weight_compression_ep_b200 import synth
+
+    return synth.generate(synth.headline())
+
+
+def run_ours(args, rank: int, world: int, local_rank: int):
+    import torch
+    import torch.distributed as dist
+
+    import dit_weight_compression_ep_b200 as ep
+    from dit_weight_compression_ep_b200 import build
+
+    build.build()
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    W = _make_weights()
+    t_enc = time.time()
+    blob = ep.encode_tensor(W, TARGET)
+    t_enc = time.time() - t_enc
+    numel = blob.rows * blob.cols
+    read_bytes = blob.stored_device_bytes()
+    write_bytes = numel * 2
+    sets = [(ep.DeviceBlob(blob, dev), torch.empty((blob.rows, blob.cols), dtype=torch.bfloat16, device=dev))
+            for _ in range(ROTATE)]
+    stream = torch.cuda.current_stream(dev)
+
+    def step(i):
+        db, out = sets[i % ROTATE]
+        ep.decode_tensor(db, ep.BF16, out=out, stream=stream)
+
+    for i in range(args.warmup):
+        step(i)
+    torch.cuda.synchronize(dev)
+    if ep.decode_status(stream) != 0:
+        raise RuntimeError("decode reported a corrupt stream")
+
+    clocks = Clocks(local_rank) if rank == 0 else None
+    time.sleep(0.3 if clocks else 0.0)
+    # per-launch events give the kernel duration for the roofline; the bracket gives the step time
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    t0w = time.time()
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    start.record(stream)
+    for i in range(args.steps):
+        ev[i][0].record(stream)
+        step(i)
+        ev[i][1].record(stream)
+    end.record(stream)
+    torch.cuda.synchronize(dev)
+    if world > 1:
+        dist.barrier()
+    t1w = time.time()
+    ms_total = start.elapsed_time(end)
+    launch_ms = [a.elapsed_time(b) for a, b in ev]
+    status = ep.decode_status(stream)
+    if status != 0:
+        raise RuntimeError(f"decode status {status}")
+    t = torch.tensor([ms_total, sum(launch_ms) / len(launch_ms)], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    ms_total, avg_launch_ms = float(t[0]), float(t[1])
+    if clocks:
+        time.sleep(0.2)
+        clocks.stop()
+
+    # ---- end to end through the public API: pinned host stream in, pinned host weights out
+    e2e_steps = max(3, min(args.steps, 20))
+    h_pay = torch.from_numpy(blob.payload.view(np.int16)).pin_memory()
+    h_tix = torch.from_numpy(blob.tile_index.view(np.int32)).pin_memory()
+    h_ft = torch.from_numpy(blob.freq_tables).pin_memory()
+    h_rs = torch.from_numpy(blob.row_scales).pin_memory()
+    h_out = torch.empty((blob.rows, blob.cols), dtype=torch.bfloat16).pin_memory()
+    db = sets[0][0]
+    out = sets[0][1]
+    h2d = h_pay.numel() * 2 + h_tix.numel() * 4 + h_ft.numel() + h_rs.numel() * 4
+    d2h = h_out.numel() * 2
+
+    def e2e_step():
+        db.payload.copy_(h_pay, non_blocking=True)
+        db.tile_index.copy_(h_tix, non_blocking=True)
+        db.freq_tables.copy_(h_ft, non_blocking=True)
+        db.row_scales.copy_(h_rs, non_blocking=True)
+        ep.decode_tensor(db, ep.BF16, out=out, stream=stream)
+        h_out.copy_(out, non_blocking=True)
+
+    for _ in range(3):
+        e2e_step()
+    torch.cuda.synchronize(dev)
+    if world > 1:
+        dist.barrier()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for _ in range(e2e_steps):
+        e2e_step()
+    b.record(stream)
+    torch.cuda.synchronize(dev)
+    e2e_ms = a.elapsed_time(b) / e2e_steps
+    te = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(te, op=dist.ReduceOp.MAX)
+    e2e_ms = float(te[0])
+    if ep.decode_status(stream) != 0:
+        raise RuntimeError("e2e decode reported a corrupt stream")
+
+    # ---- context: a torch bf16 matmul of the same layer with 4096 tokens
+    X = torch.randn(4096, blob.cols, dtype=torch.bfloat16, device=dev)
+    Wd = sets[0][1]
+    for _ in range(3):
+        torch.matmul(X, Wd.t())
+    torch.cuda.synchronize(dev)
+    ma, mb = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    ma.record(stream)
+    for _ in range(10):
+        torch.matmul(X, Wd.t())
+    mb.record(stream)
+    torch.cuda.synchronize(dev)
+    mm_ms = ma.elapsed_time(mb) / 10
+
+    if rank != 0:
+        return None
+    ms_per_step = ms_total / args.steps
+    value = world * numel / (ms_per_step * 1e-3) / 1e9
+    peak, peak_kind = _peaks()
+    alg_bytes = read_bytes + write_bytes
+    achieved = alg_bytes / (avg_launch_ms * 1e-3) / 1e9
+    traffic = _traffic_per_launch()
+    cpu = cpu_baseline(blob, seconds=args.cpu_seconds) if world == 1 else None
+    return {
+        "metric": METRIC, "value": round(value, 2), "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(ms_per_step, 5), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": round(value / (world * PAGES_GWPS), 3), "dtype": "u32+f32", "data": "synthetic",
+        "config": {"workload": WORKLOAD, "rows": blob.rows, "cols": blob.cols, "target_bpp": TARGET,
+                   "stored_bpp": round(blob.stored_bpp, 4), "b": blob.b, "tile_vectors": blob.V,
+                   "tiles": blob.ntiles, "out": "bf16",
+                   "l2": f"inputs larger than L2: steps rotate over {ROTATE} stream/output copies "
+                         f"({ROTATE * alg_bytes / 1e6:.0f} MB > {L2_BYTES / 1e6:.0f} MB L2)",
+                   "vs_baseline_ref": "pages' 0.23 ms per 39.3 M-weight layer on one H20 (Table 6), context only",
+                   "encode_s": round(t_enc, 3)},
+        "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
+                     "frac": round(achieved / peak, 4), "traffic": traffic,
+                     "algorithmic_bytes_per_launch": alg_bytes, "read_bytes": read_bytes, "write_bytes": write_bytes,
+                     "avg_launch_us": round(avg_launch_ms * 1e3, 3), "peak_kind": peak_kind},
+        "cpu_baseline": cpu,
+        "e2e": {"value": round(world * numel / (e2e_ms * 1e-3) / 1e9, 3), "unit": UNIT, "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h, "steps": e2e_steps},
+        "gpu_launches": args.steps,
+        "clocks": clocks.summary(t0w, t1w) if clocks else None,
+        "context": {"torch_bf16_matmul_4096_tokens_us": round(mm_ms * 1e3, 2),
+                    "decode_over_matmul": round(avg_launch_ms / mm_ms, 4),
+                    "pages_decode_over_matmul_h20": 0.094},
+    }
+
+
+def _oracle_threads(blob, t_ranges, nthreads, dtype):
+    """Decode tile ranges with the oracle on nthreads host threads (the C call releases the GIL)."""
+    import oracle
+    from concurrent.futures import ThreadPoolExecutor
+
+    pay = blob.payload[:blob.payload_words]
+
+    def work(rng):
+        t0, t1 = rng
+        oracle.decode(pay, blob.tile_index, blob.freq_tables, blob.row_scales, blob.rows, blob.cols, dtype, t0, t1)
+        return min(t1 * blob.V, blob.rows * blob.cols // 8) - t0 * blob.V
+
+    with ThreadPoolExecutor(nthreads) as ex:
+        return sum(ex.map(work, t_ranges)) * 8
+
+
+def cpu_baseline(blob, seconds: float = 10.0):
+    """The oracle decoder, as it stands, on all host cores over a bounded sample of the stream."""
+    import oracle
+
+    oracle.build()
+    cores = os.cpu_count() or 1
+    per = max(1, blob.ntiles // (4 * cores))
+    ranges = [(t, min(t + per, blob.ntiles)) for t in range(0, blob.ntiles, per)]
+    weights = 0
+    t0 = time.time()
+    passes = 0
+    while True:
+        weights += _oracle_threads(blob, ranges[: 2 * cores], cores, oracle.BF16)
+        passes += 1
+        if time.time() - t0 >= seconds:
+            break
+    dt = time.time() - t0
+    return {"value": round(weights / dt / 1e9, 5), "unit": UNIT, "cores": cores, "kind": "oracle",
+            "sample": f"{passes} pass(es) over tiles 0..{ranges[min(2 * cores, len(ranges)) - 1][1]} of the "
+                      f"{blob.ntiles}-tile stream ({weights / passes / 1e6:.1f} M weights per pass), "
+                      f"{cores} threads, {dt:.1f} s"}
+
+
+def run_reference(args):
+    """The oracle as the reference arm: CPU decode, each step a bounded tile sample."""
+    import oracle
+
+    oracle.build()
+    W = _make_weights()
+    ob = oracle.encode(W, TARGET)
+    blob = SimpleNamespace(payload=ob.payload, payload_words=ob.payload.size, tile_index=ob.tile_index,
+                           freq_tables=ob.freq_tables, row_scales=ob.row_scales, rows=ob.rows, cols=ob.cols,
+                           V=ob.V, ntiles=ob.ntiles)
+    cores = os.cpu_count() or 1
+    per = max(1, blob.ntiles // (4 * cores))
+    ranges = [(t, min(t + per, blob.ntiles)) for t in range(0, blob.ntiles, per)][: 2 * cores]
+    for _ in range(args.warmup):
+        _oracle_threads(blob, ranges, cores, oracle.BF16)
+    t0 = time.time()
+    weights = 0
+    for _ in range(args.steps):
+        weights += _oracle_threads(blob, ranges, cores, oracle.BF16)
+    dt = time.time() - t0
+    value = weights / dt / 1e9
+    sample = (f"tiles 0..{ranges[-1][1]} of the {blob.ntiles}-tile stream per step "
+              f"({weights / args.steps / 1e6:.1f} M weights), {cores} threads")
+    return {"metric": METRIC, "value": round(value, 5), "unit": UNIT, "n_gpus": args.gpus, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": round(dt / args.steps * 1e3, 3), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": round(value / PAGES_GWPS, 6), "dtype": "u32+f32", "data": "synthetic",
+            "config": {"workload": WORKLOAD, "rows": ROWS, "cols": COLS, "target_bpp": TARGET, "out": "bf16"},
+            "impl": "reference",
+            "cpu_baseline": {"value": round(value, 5), "unit": UNIT, "cores": cores, "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": round(value, 5), "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be at least 3")
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.impl == "reference":
+        if rank != 0:
+            return
+        res = run_reference(args)
+        print(json.dumps(res), flush=True)
+        return
+
+    if world > 1:
+        import datetime
+
+        import torch
+        import torch.distributed as dist
+
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=torch.device("cuda", local_rank))
+    try:
+        res = run_ours(args, rank, world, local_rank)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+
+            dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(res), flush=True)
+
+
+if __name__ == "__main__":
+    main()

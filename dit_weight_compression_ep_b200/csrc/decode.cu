@@ -1,36 +1,43 @@
 // decode.cu -- fused EntroPack weight reconstruction for B200 (sm_100a).
 //
-// One launch decodes a whole tensor (EntroPack paper, Fig. 2b: symbol decode,
-// lattice reconstruction, row rescaling and dtype conversion fused on the GPU;
-// §3.6 "one tile to a GPU warp and one state to each lane"; App. C.3).
+// EntroPack paper, Fig. 2b: symbol decoding, lattice reconstruction, row
+// rescaling and dtype conversion fused on the GPU; §3.6 "one tile to a GPU warp
+// and one state to each lane"; App. C.3 tile layout, state normalisation and the
+// decoder lookup tables ("in shared memory or packed global memory").
 //
-// Grid: one persistent CTA of 32 warps per SM.  Tile t goes to CTA t mod G; the
-// CTA's i-th tile goes to warp i mod 32, so every SM gets within one tile of the
-// same work.  Per CTA:
-//   a2  the 16 coordinate tables become decode LUTs in shared memory:
-//       PACKED (b <= 11, |z| small): one 32-bit entry per slot,
-//         [bias = slot - cum : b][f - 1 : b][z : 32 - 2b, signed], one LDS per symbol;
-//       COARSE (any b): one 64-bit entry per bucket of 2^(b-k) slots,
-//         {cum | f << 16, z}, plus a short forward walk over global frequencies.
-//       The coset table (2 symbols) needs no LUT: a compare picks c.
+// One call = one cooperative launch of decode_kernel on the caller's stream:
+// one persistent CTA of 24 warps per SM (all co-resident).  Its prologue reads
+// the header and starts staging every warp's first tile; then every CTA builds
+// 1/G of the decode-LUT image in a stream-ordered global workspace (binary
+// search of every slot in its table's cumulative frequencies):
+//   PACKED (b <= 11 and |z| small): 32-bit entry per slot, either
+//     [bias = slot - cum : b][f : b+1][z : 31 - 2b, signed] or
+//     [bias : b][f - 1 : b][z : 32 - 2b, signed] when z needs the extra bit;
+//   COARSE (otherwise): 64-bit entry per bucket of 2^(b-k) slots (k <= 10)
+//     {cum | f << 16, z} of the symbol owning the bucket's first slot;
+// arrives on a grid-wide counter, waits (bounded) for every CTA, and copies
+// the whole image into shared memory with cp.async.bulk.  Tile t goes to CTA
+// t mod G and, within the CTA, to warp (t / G) mod 24.
 // Per warp and tile:
-//   a1  32 terminal states (one per lane) and the payload offsets;
-//   a3  payload words staged by cp.async.bulk (TMA 1-D) into a double-buffered
-//       ring of 2 x 512 words; each chunk landing in the first half is also
-//       copied to a 288-word mirror after the ring, so one round (at most 288
-//       words) never needs to wrap an index;
-//   a4  per round r: every lane decodes the 9 fields of vector 32r + lane
-//       (c, z1..z7, m); the lanes that renormalise read consecutive words in
-//       ascending lane order (ballot + popc);
-//   a5  z8 = 2m + parity(z1..z7); y = z + c/2;
-//   a6  w = fl32(sigma_row * y) as one FFMA: fma(sigma, z, c ? sigma/2 : -0),
-//       exact to a single rounding because sigma/2 is exact;
-//   a7  conversion (cvt.rn bf16x2 / f16x2, satfinite e4m3x2, rni + clamp for
-//       int8) and one 16-byte (8-byte for 8-bit outputs) store per lane, so a
-//       warp writes 512 (256) contiguous bytes per round.
+//   a1  32 terminal states (one per lane), the tile's payload offsets;
+//   a3  payload words staged by cp.async.bulk into a double-buffered ring of
+//       2 x 512 words; a chunk landing in the first half is also copied to a
+//       288-word mirror after the ring so that one round (at most 288 words)
+//       reads without wrapping;
+//   a4  per round r each lane decodes the 9 fields (c, z1..z7, m) of vector
+//       32r + lane; the coset bit needs no LUT (two symbols, one compare); the
+//       lanes that renormalise read consecutive words in ascending lane order
+//       (ballot + popc);
+//   a5  z8 = 2m + parity(z1..z7), y = z + c/2;
+//   a6  w = fl32(sigma_row * y): y = z + c/2 is formed exactly in FP32 (from the
+//       bits of 1.5*2^22 + (2z + c)/2) and multiplied once by sigma, so every
+//       weight gets a single rounding, whatever sigma;
+//   a7  cvt.rn bf16x2 / f16x2, cvt.rn.satfinite e4m3x2, or rni + clamp for
+//       INT8, and one 16-byte (8-byte) store per lane, so a warp writes 512
+//       (256) contiguous bytes per round.
 // Stream errors never fault or trap: every shared-memory index is masked or
-// bounded, every global read stays inside the buffers the header describes, and
-// inconsistencies raise bits in a device status word read by ep_decode_status.
+// bounded, every global read stays inside the buffers the header describes,
+// every wait is bounded, and inconsistencies raise bits in a device status word.
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 #include <cuda_fp8.h>
@@ -38,6 +45,7 @@
 #include <stdint.h>
 
 #include <mutex>
+#include <type_traits>
 
 #include "entropack.h"
 #include "ep_format.h"
@@ -45,23 +53,33 @@
 namespace ep {
 namespace {
 
-constexpr int kWarps = 32;
+constexpr int kWarps = 24;
 constexpr int kThreads = 32 * kWarps;
-constexpr int kChunkWords = 512;                 // words per staged chunk
+constexpr int kChunkWords = 512;               // words per staged chunk
 constexpr int kChunkShift = 9;
-constexpr int kRingWords = 2 * kChunkWords;      // double buffer
-constexpr int kRoundWords = kFields * kLanes;    // 288: most words one round can consume
-constexpr int kRingAllocBytes = 2688;            // (1024 + 288) words, rounded up to 128 bytes
-constexpr int kCoarseBits = 10;                  // COARSE: 2^10 buckets per table
+constexpr int kRingWords = 2 * kChunkWords;    // double buffer
+constexpr int kRoundWords = kFields * kLanes;  // 288: most words one round can consume
+constexpr int kRingAllocBytes = 2688;          // (1024 + 288) words, rounded up to 128 bytes
+constexpr int kCoarseBits = 10;                // COARSE: at most 2^10 buckets per table
 
-// shared-memory layout (bytes)
+// decode_kernel shared-memory layout (bytes)
 constexpr int kLutBytes = 128 * 1024;
 constexpr int kOffLut = 0;
 constexpr int kOffRing = kOffLut + kLutBytes;
-constexpr int kOffBar = kOffRing + kWarps * kRingAllocBytes;
-constexpr int kOffDesc = kOffBar + kWarps * 16;
-constexpr int kOffFlag = kOffDesc + 3 * 32 * 4;
-constexpr int kSmemBytes = kOffFlag + 16;
+constexpr int kOffBar = kOffRing + kWarps * kRingAllocBytes;  // 2 per warp + 1 for the LUT
+constexpr int kOffDesc = kOffBar + kWarps * 16 + 16;
+constexpr int kSmemBytes = kOffDesc + 3 * 32 * 4;
+
+// LUT workspace (global, one per device, zeroed once): the image, then the
+// state of a self-resetting grid barrier: arrival counter (wraps to 0 on the
+// last arrival), bad-table count of the current generation, generation, and
+// the bad-table result of the last two generations
+constexpr int kWsCountOffset = kLutBytes;
+constexpr int kWsBadCountOffset = kLutBytes + 4;
+constexpr int kWsGenOffset = kLutBytes + 8;
+constexpr int kWsResultOffset = kLutBytes + 16;  // 2 words
+constexpr int kWsBytes = kLutBytes + 32;
+constexpr uint32_t kGridSpins = 1u << 22;  // bound on the grid-barrier polls
 
 // status bits
 constexpr unsigned kStCorrupt = 1u;      // payload / state / offset inconsistent
@@ -70,24 +88,17 @@ constexpr unsigned kStUnsupported = 4u;  // a format variant this decoder does n
 constexpr unsigned kStTimeout = 8u;      // a bulk copy did not complete in time
 
 constexpr unsigned kFull = 0xFFFFFFFFu;
-constexpr uint32_t kWaitSpins = 1u << 20;  // bound on mbarrier polls (each poll may suspend)
+constexpr uint32_t kWaitSpins = 1u << 20;  // bound on mbarrier polls
+
+// PACKED modes: b (entries hold f - 1) or 16 + b (entries hold f; one add fewer
+// per symbol, needs one more bit); COARSE otherwise.
+enum : int { kModeCoarse = 1, kModeF = 16 };
 
 }  // namespace
 
 __device__ unsigned int g_decode_status;
 
 namespace {
-
-enum : int { kModePacked9 = 9, kModePacked10 = 10, kModePacked11 = 11, kModeCoarse = 1 };
-
-struct Params {
-    const uint16_t* tiles;
-    const uint32_t* tix;
-    const uint8_t* ft;
-    const float* scales;
-    void* out;
-    int64_t rows, cols;
-};
 
 // ---------------------------------------------------------------- PTX helpers
 
@@ -99,9 +110,6 @@ __device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
 }
 __device__ __forceinline__ void fence_barrier_init() {
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-}
-__device__ __forceinline__ void fence_proxy_async_smem() {
-    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 __device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t bar, uint32_t bytes) {
     asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes) : "memory");
@@ -123,19 +131,17 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
         : "memory");
     return ok != 0;
 }
-__device__ __forceinline__ uint32_t lds_u32(uint32_t a) {
+// Bounded wait; returns false when the bound ran out.
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity) {
+    for (uint32_t spins = 0; spins < kWaitSpins; ++spins)
+        if (mbar_try_wait(bar, parity)) return true;
+    return false;
+}
+__device__ __forceinline__ void fence_proxy_async_shared() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
+__device__ __forceinline__ void fence_proxy_async_global() { asm volatile("fence.proxy.async.global;" ::: "memory"); }
+__device__ __forceinline__ uint32_t ld_acquire_gpu(const uint32_t* p) {
     uint32_t v;
-    asm volatile("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(a));
-    return v;
-}
-__device__ __forceinline__ uint2 lds_u64(uint32_t a) {
-    uint2 v;
-    asm volatile("ld.shared.v2.u32 {%0, %1}, [%2];" : "=r"(v.x), "=r"(v.y) : "r"(a));
-    return v;
-}
-__device__ __forceinline__ uint32_t lds_u16(uint32_t a) {
-    unsigned short v;
-    asm volatile("ld.shared.u16 %0, [%1];" : "=h"(v) : "r"(a));
+    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
     return v;
 }
 __device__ __forceinline__ uint32_t lanemask_lt() {
@@ -143,45 +149,171 @@ __device__ __forceinline__ uint32_t lanemask_lt() {
     asm("mov.u32 %0, %%lanemask_lt;" : "=r"(m));
     return m;
 }
-
 __device__ __forceinline__ void raise_status(unsigned bits) { atomicOr(&g_decode_status, bits); }
-
-// ------------------------------------------------------ per-warp payload ring
-
-struct Ring {
-    uint32_t ring_s;  // shared address of this warp's ring
-    uint32_t bar_s;   // shared address of its two mbarriers
-    uint32_t seq;     // chunks issued by this warp so far (all tiles)
-    uint32_t waited;  // chunks waited for so far
-    bool timed_out;
-};
-
-// Issue chunk `seq_no` of the current tile: words [src, src + n) into ring half
-// seq_no & 1 (and its first 288 words to the mirror when it is the first half).
-__device__ __forceinline__ void ring_issue(Ring& rg, const uint16_t* src, uint32_t n, int lane) {
-    const uint32_t half = rg.seq & 1u;
-    const uint32_t bar = rg.bar_s + 8u * half;
-    const uint32_t mirror = half == 0 ? (n < (uint32_t)kRoundWords ? n : (uint32_t)kRoundWords) : 0u;
-    if (lane == 0) {
-        mbar_arrive_expect_tx(bar, 2u * (n + mirror));
-        bulk_g2s(rg.ring_s + 2u * kChunkWords * half, src, 2u * n, bar);
-        if (mirror) bulk_g2s(rg.ring_s + 2u * kRingWords, src, 2u * mirror, bar);
-    }
-    rg.seq += 1;
+// Shared-memory loads at 32-bit shared addresses.  The "memory" clobber keeps
+// them after the barrier waits that publish the data they read.
+template <int OFF = 0>
+__device__ __forceinline__ uint32_t ld_s32(uint32_t a) {
+    uint32_t v;
+    asm("ld.shared.u32 %0, [%1+%2];" : "=r"(v) : "r"(a), "n"(OFF) : "memory");
+    return v;
+}
+template <int OFF = 0>
+__device__ __forceinline__ uint2 ld_s64(uint32_t a) {
+    uint2 v;
+    asm("ld.shared.v2.u32 {%0, %1}, [%2+%3];" : "=r"(v.x), "=r"(v.y) : "r"(a), "n"(OFF) : "memory");
+    return v;
+}
+__device__ __forceinline__ uint32_t ld_s16(uint32_t a) {
+    uint32_t v;
+    asm("ld.shared.u16 %0, [%1];" : "=r"(v) : "r"(a) : "memory");
+    return v;
 }
 
-__device__ __forceinline__ void ring_wait_one(Ring& rg) {
-    const uint32_t s = rg.waited;
-    const uint32_t bar = rg.bar_s + 8u * (s & 1u);
-    const uint32_t parity = (s >> 1) & 1u;
-    uint32_t spins = 0;
-    while (!mbar_try_wait(bar, parity)) {
-        if (++spins > kWaitSpins) {
-            rg.timed_out = true;
-            break;
+// ------------------------------------------------------------ header checks
+
+struct Geo {
+    uint32_t b, V, T, M;
+    int mode;
+    uint32_t k;            // COARSE: log2 buckets per table
+    uint32_t image_bytes;  // bytes of the LUT image
+    int64_t nvec;
+};
+
+// Parse and check the table header (every thread reads the same words, so the
+// result is uniform).  Returns 0, kStHeader or kStUnsupported.
+__device__ unsigned parse_header(const uint8_t* ft, int64_t rows, int64_t cols, Geo& g) {
+    // the 192 header bytes in twelve independent 16-byte loads (one round trip)
+    uint32_t h[48];
+#pragma unroll
+    for (int i = 0; i < 12; ++i) {
+        const uint4 v = __ldg(reinterpret_cast<const uint4*>(ft) + i);
+        h[4 * i] = v.x;
+        h[4 * i + 1] = v.y;
+        h[4 * i + 2] = v.z;
+        h[4 * i + 3] = v.w;
+    }
+    g.b = h[kHB];
+    g.V = h[kHV];
+    g.T = h[kHT];
+    g.nvec = rows * (cols / 8);
+    const int64_t hrows = (int64_t)(((uint64_t)h[2 * kHRows64 + 1] << 32) | h[2 * kHRows64]);
+    const int64_t hcols = (int64_t)(((uint64_t)h[2 * kHCols64 + 1] << 32) | h[2 * kHCols64]);
+    bool ok = h[kHMagic] == kMagic && h[kHVersion] == kVersion && h[kHJ] == (uint32_t)kLanes &&
+              g.b >= (uint32_t)kMinB && g.b <= (uint32_t)kMaxB && g.V >= 1 && hrows == rows && hcols == cols;
+    ok = ok && (int64_t)g.T == (g.nvec + g.V - 1) / g.V;
+    if (!ok) return kStHeader;
+    if (h[kHNTab] != (uint32_t)kTables || h[kHFlags] != 0u) return kStUnsupported;
+    g.M = 1u << g.b;
+    bool packed = g.b <= 11, fstored = g.b <= 11, bad = false;
+    const int bb = g.b <= 11 ? (int)g.b : 11;
+    const int64_t zlim = 1ll << (31 - 2 * bb), zlim_f = 1ll << (30 - 2 * bb);
+#pragma unroll
+    for (int t = 0; t < kTables; ++t) {
+        const int mn = static_cast<int>(h[12 + 2 * t]);
+        const uint32_t A = h[13 + 2 * t];
+        bad |= A > g.M;
+        if (t == 0) bad |= A < 1 || A > 2 || mn < 0 || mn + (int)A > 2;
+        if (t > 0 && A > 0) {
+            packed &= mn >= -zlim && (int64_t)mn + A - 1 < zlim;
+            fstored &= mn >= -zlim_f && (int64_t)mn + A - 1 < zlim_f;
         }
     }
-    rg.waited = s + 1;
+    if (bad) return kStHeader;
+    g.mode = fstored ? kModeF + (int)g.b : (packed ? (int)g.b : kModeCoarse);
+    g.k = g.b < (uint32_t)kCoarseBits ? g.b : (uint32_t)kCoarseBits;
+    g.image_bytes = packed ? 16u * g.M * 4u : 16u * (1u << g.k) * 8u;
+    return 0;
+}
+
+// ------------------------------------------------------- LUT image slice
+
+// a2, part 1.  Every CTA builds 1/G of the decode-LUT image in the global
+// workspace: 16 tables x E entries (E = 2^b slots for PACKED, 2^k buckets for
+// COARSE); its range touches at most two tables.  For each touched table the
+// CTA scans the frequencies into cumulative counts (u16; M <= 2^15) in shared
+// scratch and finds the owner of every slot by binary search.  Returns true
+// when a touched table does not sum to 2^b.
+__device__ bool build_lut_slice(const Geo& g, const uint16_t* fq, const int* s_min, const uint32_t* s_A,
+                                const uint32_t* s_off, uint8_t* ws, uint16_t* scratch) {
+    __shared__ uint32_t part_sum[kWarps];
+    const bool coarse = g.mode == kModeCoarse;
+    const bool fstored = g.mode >= kModeF;
+    const uint32_t E = coarse ? (1u << g.k) : g.M;
+    const uint32_t sh = coarse ? g.b - g.k : 0u;
+    const uint32_t all = 16u * E;
+    const uint32_t per = (all + gridDim.x - 1) / gridDim.x;
+    const uint32_t e0 = min(all, blockIdx.x * per), e1 = min(all, e0 + per);
+    const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
+    bool bad = false;
+    if (e0 >= e1) return false;
+    const int tfirst = 1 + (int)(e0 / E), tlast = 1 + (int)((e1 - 1) / E);
+    for (int t = tfirst; t <= tlast; ++t) {
+        uint16_t* cum = scratch;  // one table at a time: A + 1 <= 2^15 + 1 entries
+        const uint32_t A = s_A[t], off = s_off[t];
+        const int mn = s_min[t];
+        // frequencies into shared memory, then an in-place exclusive scan by contiguous chunks
+        for (uint32_t q = tid; q < A; q += kThreads) cum[q] = fq[off + q];
+        __syncthreads();
+        const uint32_t chunk = (A + kThreads - 1) / kThreads;
+        const uint32_t q0 = min(A, tid * chunk), q1 = min(A, q0 + chunk);
+        uint32_t local = 0;
+        for (uint32_t q = q0; q < q1; ++q) local += cum[q];
+        uint32_t incl = local;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const uint32_t v = __shfl_up_sync(kFull, incl, o);
+            if (lane >= o) incl += v;
+        }
+        if (lane == 31) part_sum[wid] = incl;
+        __syncthreads();
+        uint32_t before = 0, total = 0;
+        for (int w = 0; w < kWarps; ++w) {
+            if (w < wid) before += part_sum[w];
+            total += part_sum[w];
+        }
+        uint32_t run = before + incl - local;
+        for (uint32_t q = q0; q < q1; ++q) {
+            const uint32_t f = cum[q];
+            cum[q] = (uint16_t)(run < g.M ? run : g.M);
+            run += f;
+        }
+        if (tid == 0) cum[A] = (uint16_t)(total < g.M ? total : g.M);
+        __syncthreads();
+        const bool valid = A == 0 || total == g.M;
+        bad |= !valid;
+        // entries of this table inside [e0, e1)
+        const uint32_t lo = max(e0, (uint32_t)(t - 1) * E), hi = min(e1, (uint32_t)t * E);
+        for (uint32_t idx = lo + tid; idx < hi; idx += kThreads) {
+            const uint32_t j = idx - (uint32_t)(t - 1) * E;  // slot (PACKED) or bucket (COARSE)
+            const uint32_t slot = j << sh;
+            uint32_t s = 0, c0 = 0, f = 0;
+            if (A > 0 && valid) {
+                uint32_t l = 0, r = A;  // cum[l] <= slot < cum[r]
+                while (r - l > 1) {
+                    const uint32_t mid = (l + r) >> 1;
+                    if (cum[mid] <= slot) l = mid;
+                    else r = mid;
+                }
+                s = l;
+                c0 = cum[s];
+                f = cum[s + 1] - c0;
+            }
+            if (coarse) {
+                reinterpret_cast<uint2*>(ws)[idx] =
+                    A > 0 && valid ? make_uint2(c0 | (f << 16), (uint32_t)((int)s + mn)) : make_uint2(0u, 0u);
+            } else {
+                const uint32_t b = g.b;
+                uint32_t e = 0;
+                if (A > 0 && valid)
+                    e = fstored ? (slot - c0) | (f << b) | ((uint32_t)((int)s + mn) << (2 * b + 1))
+                                : (slot - c0) | ((f - 1) << b) | ((uint32_t)((int)s + mn) << (2 * b));
+                reinterpret_cast<uint32_t*>(ws)[idx] = e;
+            }
+        }
+        __syncthreads();  // the scratch is reused by the next table
+    }
+    return bad;
 }
 
 // ------------------------------------------------------------ output writers
@@ -255,31 +387,35 @@ struct Out<EP_FP32> {
 
 // ------------------------------------------------------------- symbol LUTs
 
-// PACKED: 16 tables x 2^B slots x 32-bit entries at lut_s; table (2(k-1) + c).
-template <int B>
+// PACKED: 16 tables x 2^B slots x 32-bit entries at shared address lut_s;
+// table (2(k-1) + c).  F: the entry holds f in B+1 bits (z in 31 - 2B bits),
+// otherwise f - 1 in B bits (z in 32 - 2B bits).
+template <int B, bool F>
 struct PackedLut {
     static constexpr uint32_t kM = 1u << B;
+    static constexpr int kB = B;
     uint32_t lut_s;
     __device__ __forceinline__ uint32_t coset_base(int c) const { return lut_s + ((uint32_t)c << (B + 2)); }
-    // Decode one coordinate symbol of field k (1..8) for the coset base cb.
     template <int K>
     __device__ __forceinline__ int decode(uint32_t& x, uint32_t cb, bool& bad) const {
-        const uint32_t slot = x & (kM - 1);
-        const uint32_t e = lds_u32(cb + (uint32_t)(2 * (K - 1)) * (kM * 4u) + slot * 4u);
-        const uint32_t bias = e & (kM - 1);
-        const uint32_t fm1 = (e >> B) & (kM - 1);
+        const uint32_t e = ld_s32<(2 * (K - 1)) * (int)kM * 4>(cb + ((x & (kM - 1)) << 2));
         const uint32_t xs = x >> B;
-        x = fm1 * xs + (xs + bias);
+        if constexpr (F) {
+            x = ((e >> B) & (2 * kM - 1)) * xs + (e & (kM - 1));
+        } else {
+            x = ((e >> B) & (kM - 1)) * xs + (xs + (e & (kM - 1)));
+        }
         (void)bad;
-        return static_cast<int>(e) >> (2 * B);
+        return static_cast<int>(e) >> (F ? 2 * B + 1 : 2 * B);
     }
 };
 
 // COARSE: 16 tables x 2^k buckets x 64-bit {cum | f << 16, z}; runtime b.
 struct CoarseLut {
-    uint32_t lut_s;
-    uint32_t b, mmask, sh, nb_shift;  // bucket = slot >> sh; table stride = 8 << nb_shift
-    const uint16_t* fq;               // global frequencies
+    static constexpr int kB = 0;
+    uint32_t lut_s;  // shared address
+    uint32_t b, mmask, sh, nb_shift;
+    const uint16_t* fq;  // global frequencies
     const int* s_min;
     const uint32_t* s_A;
     const uint32_t* s_off;
@@ -287,16 +423,15 @@ struct CoarseLut {
     template <int K>
     __device__ __forceinline__ int decode(uint32_t& x, uint32_t cb, bool& bad) const {
         const uint32_t slot = x & mmask;
-        const uint2 e = lds_u64(cb + (uint32_t)(2 * (K - 1)) * (8u << nb_shift) + (slot >> sh) * 8u);
+        const uint2 e = ld_s64(cb + ((uint32_t)(2 * (K - 1)) << (nb_shift + 3)) + ((slot >> sh) << 3));
         uint32_t c0 = e.x & 0xFFFFu, f = e.x >> 16;
         int z = static_cast<int>(e.y);
         if (slot >= c0 + f) {
-            // table index of this lane: from the coset base
             const int t = 1 + 2 * (K - 1) + (int)((cb - lut_s) >> (nb_shift + 3));
             const int mn = s_min[t];
             const uint32_t A = s_A[t], off = s_off[t];
-            // the walk may cross zero-frequency symbols (unobserved values inside
-            // the alphabet), so it is bounded by the alphabet, not by the bucket width
+            // the walk may cross zero-frequency symbols (unobserved values inside the
+            // alphabet), so it is bounded by the alphabet, not by the bucket width
             while (slot >= c0 + f) {
                 c0 += f;
                 ++z;
@@ -315,286 +450,242 @@ struct CoarseLut {
     }
 };
 
-// ------------------------------------------------------------- LUT builders
+// ------------------------------------------------------ per-warp payload ring
 
-__device__ __forceinline__ uint32_t warp_incl_scan(uint32_t v, int lane) {
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-        const uint32_t u = __shfl_up_sync(kFull, v, o);
-        if (lane >= o) v += u;
+struct Ring {
+    uint8_t* ring;    // this warp's ring (generic pointer into shared memory)
+    uint32_t ring_s;  // its shared address
+    uint32_t bar_s;   // shared address of its two mbarriers
+    uint32_t seq;     // chunks issued so far (all tiles)
+    uint32_t waited;  // chunks waited for so far
+    bool timed_out;
+};
+
+// Issue the next chunk: words [src, src + n) into ring half seq & 1 (and its
+// first 288 words to the mirror when that half is the first one).
+__device__ __forceinline__ void ring_issue(Ring& rg, const uint16_t* src, uint32_t n, int lane) {
+    const uint32_t half = rg.seq & 1u;
+    const uint32_t bar = rg.bar_s + 8u * half;
+    const uint32_t mirror = half == 0 ? (n < (uint32_t)kRoundWords ? n : (uint32_t)kRoundWords) : 0u;
+    if (lane == 0) {
+        mbar_arrive_expect_tx(bar, 2u * (n + mirror));
+        bulk_g2s(rg.ring_s + 2u * kChunkWords * half, src, 2u * n, bar);
+        if (mirror) bulk_g2s(rg.ring_s + 2u * kRingWords, src, 2u * mirror, bar);
     }
-    return v;
+    rg.seq += 1;
 }
 
-// PACKED build.  Phase 1 (warps 0..15, table w+1): cumulative frequencies into a
-// u16 scratch area of shared memory and, per 32-slot block, the symbol holding
-// the block's first slot.  Phase 2 (all threads): entries of 4 consecutive slots
-// per thread, written as one 16-byte store (a warp writes 512 contiguous bytes).
-template <int B>
-__device__ void build_packed(uint8_t* smem, const uint16_t* fq, const int* s_min, const uint32_t* s_A,
-                             const uint32_t* s_off, volatile int* s_bad) {
-    constexpr uint32_t M = 1u << B;
-    constexpr uint32_t kBlocks = M / 32;
-    uint16_t* cum_all = reinterpret_cast<uint16_t*>(smem + kOffRing);
-    uint16_t* blk_all = cum_all + 16 * (M + 1);  // cum area sized for A <= M per table
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    if (warp < 16) {
-        const int t = warp + 1;
-        const uint32_t A = s_A[t], off = s_off[t];
-        uint16_t* cum = cum_all + (t - 1) * (M + 1);
-        uint16_t* blk = blk_all + (t - 1) * kBlocks;
-        uint32_t carry = 0;
-        for (uint32_t base = 0; base < A; base += 32) {
-            const uint32_t s = base + lane;
-            const uint32_t f = s < A ? fq[off + s] : 0u;
-            const uint32_t incl = warp_incl_scan(f, lane);
-            const uint32_t c0 = carry + incl - f;
-            if (s < A) cum[s] = (uint16_t)(c0 < M ? c0 : M);
-            if (f > 0 && c0 < M) {
-                uint32_t end = c0 + f < M ? c0 + f : M;
-                for (uint32_t j = (c0 + 31) >> 5; (j << 5) < end; ++j) blk[j] = (uint16_t)s;
-            }
-            carry += __shfl_sync(kFull, incl, 31);
-        }
-        if (lane == 0) {
-            cum[A] = (uint16_t)(carry <= M ? carry : M);
-            if (A > 0 && carry != M) *s_bad = 1;
-        }
-    }
-    __syncthreads();
-    if (*s_bad) return;
-    uint32_t* lut = reinterpret_cast<uint32_t*>(smem + kOffLut);
-    for (uint32_t q = threadIdx.x; q < 16u * (M / 4); q += kThreads) {
-        const int t = (int)(q / (M / 4)) + 1;
-        const uint32_t slot0 = (q % (M / 4)) * 4;
-        const uint32_t A = s_A[t];
-        uint4 v = make_uint4(0, 0, 0, 0);
-        if (A > 0) {
-            const uint16_t* cum = cum_all + (t - 1) * (M + 1);
-            const uint16_t* blk = blk_all + (t - 1) * kBlocks;
-            const int mn = s_min[t];
-            uint32_t s = blk[slot0 >> 5];
-            uint32_t e[4];
-#pragma unroll
-            for (int k = 0; k < 4; ++k) {
-                const uint32_t slot = slot0 + k;
-                while (s + 1 < A && cum[s + 1] <= slot) ++s;
-                const uint32_t c0 = cum[s], f = cum[s + 1] - c0;
-                e[k] = (slot - c0) | ((f - 1) << B) | ((uint32_t)((int)s + mn) << (2 * B));
-            }
-            v = make_uint4(e[0], e[1], e[2], e[3]);
-        }
-        reinterpret_cast<uint4*>(lut)[q] = v;
-    }
-}
-
-// COARSE build (warps 0..15, table w+1): bucket j of 2^sh slots holds the symbol
-// that owns slot j << sh, with its cum, f and value.
-__device__ void build_coarse(uint8_t* smem, const uint16_t* fq, uint32_t b, uint32_t sh, uint32_t nb_shift,
-                             const int* s_min, const uint32_t* s_A, const uint32_t* s_off, volatile int* s_bad) {
-    const uint32_t M = 1u << b;
-    const uint32_t NB = 1u << nb_shift;
-    uint2* lut = reinterpret_cast<uint2*>(smem + kOffLut);
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    if (warp >= 16) return;
-    const int t = warp + 1;
-    const uint32_t A = s_A[t], off = s_off[t];
-    const int mn = s_min[t];
-    uint2* tl = lut + (size_t)(t - 1) * NB;
-    if (A == 0) {
-        for (uint32_t j = lane; j < NB; j += 32) tl[j] = make_uint2(0u, 0u);
-        return;
-    }
-    uint32_t carry = 0;
-    for (uint32_t base = 0; base < A; base += 32) {
-        const uint32_t s = base + lane;
-        const uint32_t f = s < A ? fq[off + s] : 0u;
-        const uint32_t incl = warp_incl_scan(f, lane);
-        const uint32_t c0 = carry + incl - f;
-        if (f > 0 && c0 < M) {
-            const uint32_t end = c0 + f < M ? c0 + f : M;
-            const uint32_t w = 1u << sh;
-            for (uint32_t j = (c0 + w - 1) >> sh; (j << sh) < end; ++j)
-                tl[j] = make_uint2(c0 | (f << 16), (uint32_t)((int)s + mn));
-        }
-        carry += __shfl_sync(kFull, incl, 31);
-    }
-    if (lane == 0 && carry != M) *s_bad = 1;
+__device__ __forceinline__ void ring_wait_one(Ring& rg) {
+    const uint32_t s = rg.waited;
+    if (!mbar_wait(rg.bar_s + 8u * (s & 1u), (s >> 1) & 1u)) rg.timed_out = true;
+    rg.waited = s + 1;
 }
 
 // ------------------------------------------------------------ the decode loop
 
 struct TileCtx {
     int64_t nvec;
-    uint32_t V, T, nq;
+    uint32_t V, T, nq, total;
     uint32_t f0c, f1c, cmin;  // coset table: f of symbol 0, of symbol 1, its min
     uint32_t b;
 };
 
-template <typename Lut, int B_CT>
-__device__ __forceinline__ uint32_t xshift(uint32_t x, uint32_t b) {
-    if constexpr (B_CT > 0) return x >> B_CT;
-    else return x >> b;
+// One tile's bookkeeping: record, staging state and every lane's row.
+struct Tile {
+    uint32_t t;
+    int64_t v0;
+    uint32_t vt, rounds;
+    uint32_t base, fend, nchunks, seq0, org;
+    uint32_t off0, off1;
+    uint32_t x;
+    uint32_t ql, rowl;
+    bool ok;
+};
+
+__device__ __forceinline__ void tile_issue_chunk(const uint16_t* tiles, Ring& rg, const Tile& tl, uint32_t ci,
+                                                 int lane) {
+    const uint32_t w0 = tl.base + ci * kChunkWords;
+    const uint32_t n = tl.fend - w0 < (uint32_t)kChunkWords ? tl.fend - w0 : (uint32_t)kChunkWords;
+    ring_issue(rg, tiles + w0, n, lane);
 }
 
-// One renormalisation step for all lanes of the warp.
-__device__ __forceinline__ void renorm(uint32_t& x, uint32_t xn, bool act, uint32_t& pbyte, uint32_t lt) {
-    const bool need = act && xn < kStateLow;
+// Read the tile record, check it, and start staging its first two chunks.
+__device__ __forceinline__ void tile_begin(const TileCtx& tc, const uint16_t* tiles, const uint32_t* tix, Ring& rg,
+                                           Tile& tl, uint32_t t, int lane) {
+    tl.t = t;
+    tl.v0 = (int64_t)t * tc.V;
+    tl.vt = (uint32_t)((tc.nvec - tl.v0) < (int64_t)tc.V ? (tc.nvec - tl.v0) : (int64_t)tc.V);
+    tl.rounds = (tl.vt + 31) >> 5;
+    const uint32_t* rec = tix + (size_t)kTileWords * t;
+    tl.off0 = rec[0];
+    tl.off1 = rec[kTileWords];
+    tl.x = rec[1 + lane];
+    const bool bad = !(tl.off0 <= tl.off1 && tl.off1 <= tc.total) || tl.x < kStateLow || tl.x >= 0x80000000u;
+    tl.ok = !__any_sync(kFull, bad);
+    tl.base = tl.off0 & ~7u;
+    tl.fend = (tl.off1 + 7u) & ~7u;
+    tl.nchunks = tl.ok ? (tl.fend - tl.base + kChunkWords - 1) >> kChunkShift : 0u;
+    tl.seq0 = rg.seq;
+    tl.org = (tl.seq0 & 1u) * kChunkWords;
+    if (tl.nchunks > 0) tile_issue_chunk(tiles, rg, tl, 0, lane);
+    if (tl.nchunks > 1) tile_issue_chunk(tiles, rg, tl, 1, lane);
+    const int64_t rowbase = tl.v0 / tc.nq;
+    tl.ql = (uint32_t)(tl.v0 - rowbase * tc.nq) + lane;
+    tl.rowl = (uint32_t)rowbase;
+    while (tl.ql >= tc.nq) {
+        tl.ql -= tc.nq;
+        ++tl.rowl;
+    }
+}
+
+// Renormalisation of every lane after one symbol: the lanes whose state fell
+// below 2^15 take the next words in ascending lane order.  pb is the shared
+// byte address of the next unread word.
+template <bool FULL>
+__device__ __forceinline__ void renorm(uint32_t& x, uint32_t xn, bool act, uint32_t& pb, uint32_t lt) {
+    const bool need = (FULL || act) && xn < kStateLow;
     const uint32_t bal = __ballot_sync(kFull, need);
-    const uint32_t rank = __popc(bal & lt);
-    const uint32_t w = lds_u16(pbyte + 2u * rank);
-    const uint32_t xr = need ? ((xn << 16) | w) : xn;
-    x = act ? xr : x;
-    pbyte += 2u * __popc(bal);
+    const uint32_t w = ld_s16(pb + 2u * __popc(bal & lt));
+    if (FULL) {
+        x = need ? ((xn << 16) | w) : xn;
+    } else if (act) {
+        x = need ? ((xn << 16) | w) : xn;
+    }
+    pb += 2u * __popc(bal);
 }
 
-template <int DT, typename Lut, int B_CT>
-__device__ void decode_tiles(const Params& p, const Lut& lut, const TileCtx& tc, uint8_t* smem) {
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+template <int DT, typename Lut, bool FULL>
+__device__ __forceinline__ void decode_round(void* out, const float sigma, const Lut& lut, const TileCtx& tc,
+                                             Tile& tl, uint32_t& pb, uint32_t r, uint32_t lt, int lane,
+                                             bool& corrupt) {
+    const uint32_t u = (r << 5) + lane;
+    const bool act = FULL || u < tl.vt;
+    const int64_t g = tl.v0 + u;
+    uint32_t x = tl.x;
+
+    // ---- a4: field 0, the coset bit (a two-symbol table: one compare)
+    const uint32_t mmask = (Lut::kB > 0 ? (1u << Lut::kB) : (1u << tc.b)) - 1u;
+    const uint32_t slot = x & mmask;
+    const uint32_t cs = slot >= tc.f0c ? 1u : 0u;
+    {
+        const uint32_t f = cs ? tc.f1c : tc.f0c;
+        const uint32_t bias = cs ? slot - tc.f0c : slot;
+        const uint32_t xn = f * (Lut::kB > 0 ? (x >> Lut::kB) : (x >> tc.b)) + bias;
+        renorm<FULL>(x, xn, act, pb, lt);
+    }
+    const int c = (int)(tc.cmin + cs);
+    const auto cb = lut.coset_base(c & 1);
+    bool badsym = false;
+    int z[8];
+    uint32_t xn;
+#define EP_FIELD(K)                                    \
+    xn = x;                                            \
+    z[K - 1] = lut.template decode<K>(xn, cb, badsym); \
+    renorm<FULL>(x, xn, act, pb, lt);
+    EP_FIELD(1)
+    EP_FIELD(2)
+    EP_FIELD(3)
+    EP_FIELD(4)
+    EP_FIELD(5)
+    EP_FIELD(6)
+    EP_FIELD(7)
+    EP_FIELD(8)
+#undef EP_FIELD
+    tl.x = x;
+    if (badsym && act) corrupt = true;
+
+    // ---- a5: z8 = 2m + parity(z1..z7)
+    const int s7 = z[0] + z[1] + z[2] + z[3] + z[4] + z[5] + z[6];
+    z[7] = 2 * z[7] + (s7 & 1);
+
+    if (act) {
+        if constexpr (DT == EP_LATTICE_I32) {
+            int4* o = reinterpret_cast<int4*>(out) + 2 * g;
+            o[0] = make_int4(2 * z[0] + c, 2 * z[1] + c, 2 * z[2] + c, 2 * z[3] + c);
+            o[1] = make_int4(2 * z[4] + c, 2 * z[5] + c, 2 * z[6] + c, 2 * z[7] + c);
+        } else {
+            // ---- a6: w = fl32(sigma * y), y = z + c/2 formed exactly from the bits of
+            // 1.5 * 2^22 + (2z + c)/2 (|2z + c| < 2^22), then one FMUL: one rounding
+            // for every sigma (zero, subnormal and negative included)
+            float w[8];
+#pragma unroll
+            for (int k = 0; k < 8; ++k)
+                w[k] = sigma * (__int_as_float(0x4AC00000 + 2 * z[k] + c) - 6291456.0f);
+            // ---- a7: conversion + one vector store per lane
+            Out<DT>::store(out, g, w);
+        }
+    }
+}
+
+// Decode the tiles of this warp; the first one was begun in the prologue.
+template <int DT, typename Lut>
+__device__ void decode_tiles(const uint16_t* tiles, const uint32_t* tix, const float* scales, void* out,
+                             const Lut& lut, const TileCtx& tc, Ring& rg, Tile& tl, uint32_t first_i) {
+    const int lane = threadIdx.x & 31;
     const uint32_t lt = lanemask_lt();
     const uint32_t G = gridDim.x;
-    const uint32_t M = 1u << tc.b;
-    const uint32_t mmask = M - 1;
-
-    Ring rg;
-    rg.ring_s = smem_u32(smem + kOffRing + warp * kRingAllocBytes);
-    rg.bar_s = smem_u32(smem + kOffBar + warp * 16);
-    rg.seq = 0;
-    rg.waited = 0;
-    rg.timed_out = false;
-    if (lane == 0) {
-        mbar_init(rg.bar_s, 1);
-        mbar_init(rg.bar_s + 8, 1);
-        fence_barrier_init();
-    }
-    __syncwarp();
-
-    const uint32_t total = p.tix[(size_t)kTileWords * tc.T];
     bool corrupt = false;
+    bool have = tl.t != 0xFFFFFFFFu;
 
-    for (uint32_t i = warp;; i += kWarps) {
-        const uint64_t t64 = (uint64_t)blockIdx.x + (uint64_t)i * G;
-        if (t64 >= tc.T) break;
-        const uint32_t t = (uint32_t)t64;
-        const int64_t v0 = (int64_t)t * tc.V;
-        const uint32_t vt = (uint32_t)((tc.nvec - v0) < (int64_t)tc.V ? (tc.nvec - v0) : (int64_t)tc.V);
-        const uint32_t* rec = p.tix + (size_t)kTileWords * t;
-        const uint32_t off0 = rec[0], off1 = rec[kTileWords];
-        uint32_t x = rec[1 + lane];
-        const bool bad_rec = !(off0 <= off1 && off1 <= total) || x < kStateLow || x >= 0x80000000u;
-        if (__any_sync(kFull, bad_rec)) {
+    for (uint32_t i = first_i; have;) {
+        if (!tl.ok) {
             corrupt = true;
-            continue;
-        }
-        // payload staging bookkeeping (warp-uniform)
-        const uint32_t base = off0 & ~7u;
-        const uint32_t fend = (off1 + 7u) & ~7u;
-        const uint32_t nchunks = (fend - base + kChunkWords - 1) >> kChunkShift;
-        const uint32_t seq0 = rg.seq;
-        const uint32_t org = (seq0 & 1u) * kChunkWords;
-        auto issue = [&](uint32_t ci) {
-            const uint32_t w0 = base + ci * kChunkWords;
-            const uint32_t n = fend - w0 < (uint32_t)kChunkWords ? fend - w0 : (uint32_t)kChunkWords;
-            ring_issue(rg, p.tiles + w0, n, lane);
-        };
-        if (nchunks > 0) issue(0);
-        if (nchunks > 1) issue(1);
-        uint32_t cur = off0 - base;  // tile-relative word cursor
-
-        // row of every lane's vector: vector g = v0 + 32r + lane
-        const int64_t rowbase = v0 / tc.nq;
-        uint32_t ql = (uint32_t)(v0 - rowbase * tc.nq) + lane;
-        uint32_t rowl = (uint32_t)rowbase;
-        while (ql >= tc.nq) {
-            ql -= tc.nq;
-            ++rowl;
-        }
-
-        const uint32_t rounds = (vt + 31) >> 5;
-        for (uint32_t r = 0; r < rounds; ++r) {
-            // ---- a3: staging: issue the chunk after the current one, wait for what this round may read
-            const uint32_t ci = cur >> kChunkShift;
-            if (ci + 1 < nchunks && ci + 1 >= rg.seq - seq0) issue(ci + 1);
-            uint32_t last = (cur + kRoundWords - 1) >> kChunkShift;
-            const uint32_t issued = rg.seq - seq0;
-            if (last >= issued) last = issued - 1;  // never wait on a chunk that was not issued
-            while (issued > 0 && rg.waited - seq0 <= last) ring_wait_one(rg);
-            uint32_t pbyte = rg.ring_s + 2u * ((org + cur) & (kRingWords - 1));
-            const uint32_t p_start = pbyte;
-
-            const uint32_t u = (r << 5) + lane;
-            const bool act = u < vt;
-            const int64_t g = v0 + u;
-            const float sigma = act ? __ldg(p.scales + rowl) : 0.0f;
-
-            // ---- a4: field 0, the coset bit (two-symbol table, no LUT)
-            uint32_t slot = x & mmask;
-            const uint32_t cs = slot >= tc.f0c ? 1u : 0u;
-            {
-                const uint32_t f = cs ? tc.f1c : tc.f0c;
-                const uint32_t bias = cs ? slot - tc.f0c : slot;
-                const uint32_t xn = f * xshift<Lut, B_CT>(x, tc.b) + bias;
-                renorm(x, xn, act, pbyte, lt);
-            }
-            const int c = (int)(tc.cmin + cs);
-            const uint32_t cb = lut.coset_base(c & 1);
-            bool badsym = false;
-            int z[8];
-            uint32_t xn;
-#define EP_FIELD(K)                                        \
-    xn = x;                                                \
-    z[K - 1] = lut.template decode<K>(xn, cb, badsym);     \
-    renorm(x, xn, act, pbyte, lt);
-            EP_FIELD(1)
-            EP_FIELD(2)
-            EP_FIELD(3)
-            EP_FIELD(4)
-            EP_FIELD(5)
-            EP_FIELD(6)
-            EP_FIELD(7)
-            EP_FIELD(8)
-#undef EP_FIELD
-            corrupt |= badsym && act;
-            cur += (pbyte - p_start) >> 1;
-
-            // ---- a5: z8 = 2m + parity(z1..z7)
-            const int s7 = z[0] + z[1] + z[2] + z[3] + z[4] + z[5] + z[6];
-            z[7] = 2 * z[7] + (s7 & 1);
-
-            if (act) {
-                if constexpr (DT == EP_LATTICE_I32) {
-                    int4* o = reinterpret_cast<int4*>(p.out) + 2 * g;
-                    o[0] = make_int4(2 * z[0] + c, 2 * z[1] + c, 2 * z[2] + c, 2 * z[3] + c);
-                    o[1] = make_int4(2 * z[4] + c, 2 * z[5] + c, 2 * z[6] + c, 2 * z[7] + c);
-                } else {
-                    // ---- a6: w = fl32(sigma * (z + c/2)) with one rounding
-                    float w[8];
-                    if (fabsf(sigma) >= 0x1p-124f) {
-                        const float add = c ? sigma * 0.5f : -0.0f;
-#pragma unroll
-                        for (int k = 0; k < 8; ++k) w[k] = fmaf(sigma, __int2float_rn(z[k]), add);
-                    } else {
-                        const float hc = c ? 0.5f : 0.0f;
-#pragma unroll
-                        for (int k = 0; k < 8; ++k) w[k] = sigma * (__int2float_rn(z[k]) + hc);
+        } else {
+            uint32_t cur = tl.off0 - tl.base;  // tile-relative word cursor
+            // a3: the staging state changes only when the cursor crosses `thr`:
+            // at the start of a chunk (issue the one after it) or within one round
+            // of a chunk not yet waited for (wait for it)
+            uint32_t thr = 0;
+            // every lane's row for round 0, its row scale, and the row of round 1
+            float sig_next = tl.vt > (uint32_t)lane ? __ldg(scales + tl.rowl) : 1.0f;
+            auto round = [&](auto full, uint32_t r) {
+                constexpr bool FULL = decltype(full)::value;
+                if (cur >= thr) {
+                    const uint32_t ci = cur >> kChunkShift;
+                    if (ci + 1 < tl.nchunks && ci + 1 >= rg.seq - tl.seq0)
+                        tile_issue_chunk(tiles, rg, tl, ci + 1, lane);
+                    const uint32_t issued = rg.seq - tl.seq0;
+                    if (issued > 0) {
+                        uint32_t last = (cur + kRoundWords - 1) >> kChunkShift;
+                        if (last >= issued) last = issued - 1;  // never wait on a chunk that was not issued
+                        while (rg.waited - tl.seq0 <= last) ring_wait_one(rg);
                     }
-                    // ---- a7: conversion + one vector store per lane
-                    Out<DT>::store(p.out, g, w);
+                    const uint32_t nw = rg.waited - tl.seq0, ni = rg.seq - tl.seq0;
+                    const uint32_t t_issue = ni < tl.nchunks ? (ni - 1) << kChunkShift : 0xFFFFFFFFu;
+                    const uint32_t t_wait = nw < ni ? (nw << kChunkShift) - (kRoundWords - 1) : 0xFFFFFFFFu;
+                    thr = t_issue < t_wait ? t_issue : t_wait;
                 }
-            }
-            // advance every lane's row by 32 vectors
-            ql += 32;
-            while (ql >= tc.nq) {
-                ql -= tc.nq;
-                ++rowl;
-            }
+                uint32_t pb = rg.ring_s + 2u * ((tl.org + cur) & (kRingWords - 1));
+                const uint32_t p_start = pb;
+                const float sigma = sig_next;
+                // advance every lane's row by 32 vectors and prefetch the next round's scale
+                tl.ql += 32;
+                if (tc.nq >= 32) {
+                    const bool wrap = tl.ql >= tc.nq;
+                    tl.ql -= wrap ? tc.nq : 0u;
+                    tl.rowl += wrap ? 1u : 0u;
+                } else {
+                    while (tl.ql >= tc.nq) {
+                        tl.ql -= tc.nq;
+                        ++tl.rowl;
+                    }
+                }
+                if (FULL) sig_next = ((r + 1) << 5) + lane < tl.vt ? __ldg(scales + tl.rowl) : 1.0f;
+                decode_round<DT, Lut, FULL>(out, sigma, lut, tc, tl, pb, r, lt, lane, corrupt);
+                cur += (pb - p_start) >> 1;
+            };
+            for (uint32_t r = 0; r + 1 < tl.rounds; ++r) round(std::true_type{}, r);
+            round(std::false_type{}, tl.rounds - 1);
+            // tile end: every lane back at 2^15 and the cursor on the next offset
+            if (!__all_sync(kFull, tl.x == kStateLow) || cur != tl.off1 - tl.base) corrupt = true;
         }
-        // tile end: every lane back at 2^15 and the cursor on the next offset
-        const bool lane_ok = x == kStateLow;
-        if (!__all_sync(kFull, lane_ok) || cur != off1 - base) corrupt = true;
-        // drain the copies of this tile before the ring is reused
-        while (rg.waited < rg.seq) ring_wait_one(rg);
+        // drain this tile's copies before the ring is reused
+        while (rg.waited < rg.seq && !rg.timed_out) ring_wait_one(rg);
         if (rg.timed_out) break;
+        i += kWarps;
+        const uint64_t t64 = (uint64_t)blockIdx.x + (uint64_t)i * G;
+        have = t64 < tc.T;
+        if (have) tile_begin(tc, tiles, tix, rg, tl, (uint32_t)t64, lane);
     }
     while (rg.waited < rg.seq && !rg.timed_out) ring_wait_one(rg);
     if (lane == 0) {
@@ -607,144 +698,233 @@ __device__ void decode_tiles(const Params& p, const Lut& lut, const TileCtx& tc,
 
 // ---------------------------------------------------------------- the kernel
 
+struct Params {
+    const uint16_t* tiles;
+    const uint32_t* tix;
+    const uint8_t* ft;
+    const float* scales;
+    void* out;
+    uint8_t* ws;  // LUT image + grid-barrier state
+    int64_t rows, cols;
+};
+
 template <int DT>
 __global__ void __launch_bounds__(kThreads, 1) decode_kernel(Params p) {
     extern __shared__ __align__(1024) uint8_t smem[];
+    __shared__ int s_ok;
     int* s_min = reinterpret_cast<int*>(smem + kOffDesc);
     uint32_t* s_A = reinterpret_cast<uint32_t*>(smem + kOffDesc + 128);
     uint32_t* s_off = reinterpret_cast<uint32_t*>(smem + kOffDesc + 256);
-    volatile int* s_flag = reinterpret_cast<volatile int*>(smem + kOffFlag);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
-    // ---- header (every thread reads the same words, so every decision is uniform)
-    const uint32_t* h = reinterpret_cast<const uint32_t*>(p.ft);
-    const int64_t* h64 = reinterpret_cast<const int64_t*>(p.ft);
-    const uint32_t b = h[kHB], V = h[kHV], T = h[kHT];
-    const int64_t nvec = p.rows * (p.cols / 8);
-    bool ok = h[kHMagic] == kMagic && h[kHVersion] == kVersion && h[kHJ] == (uint32_t)kLanes && b >= (uint32_t)kMinB &&
-              b <= (uint32_t)kMaxB && V >= 1 && h64[kHRows64] == p.rows && h64[kHCols64] == p.cols;
-    ok = ok && (int64_t)T == (nvec + V - 1) / V;
-    const bool unsupported = ok && (h[kHNTab] != (uint32_t)kTables || h[kHFlags] != 0u);
-    if (!ok || unsupported) {
-        if (threadIdx.x == 0 && blockIdx.x == 0) raise_status(ok ? kStUnsupported : kStHeader);
+    // ---- prologue: header, descriptors, barriers, the first chunks of every warp's first tile
+    Geo g;
+    const unsigned hs = parse_header(p.ft, p.rows, p.cols, g);
+    if (hs) {  // every CTA reads the same header, so every CTA leaves here
+        if (threadIdx.x == 0 && blockIdx.x == 0) raise_status(hs);
         return;
     }
-    if (blockIdx.x >= T) return;
-    const uint32_t M = 1u << b;
-
-    // ---- a2: table descriptors, validation, mode
+    const uint32_t* h = reinterpret_cast<const uint32_t*>(p.ft);
+    const uint16_t* fq = reinterpret_cast<const uint16_t*>(p.ft + table_header_bytes(kTables));
     if (threadIdx.x < 32) {
         const int t = threadIdx.x;
-        int mn = 0;
-        uint32_t A = 0;
-        if (t < kTables) {
-            mn = static_cast<int>(h[12 + 2 * t]);
-            A = h[13 + 2 * t];
+        const uint32_t A = t < kTables ? h[13 + 2 * t] : 0u;
+        uint32_t incl = A;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const uint32_t v = __shfl_up_sync(kFull, incl, o);
+            if (t >= o) incl += v;
         }
-        const uint32_t incl = warp_incl_scan(A, t);
         if (t < kTables) {
-            s_min[t] = mn;
+            s_min[t] = static_cast<int>(h[12 + 2 * t]);
             s_A[t] = A;
             s_off[t] = incl - A;
         }
-        bool bad = t < kTables && A > M;
-        if (t == 0) bad = bad || A < 1 || A > 2 || mn < 0 || mn + (int)A > 2;
-        int packed = 0;
-        if (b <= 11) {
-            const int64_t zlim = 1ll << (31 - 2 * b);
-            const bool fits = t == 0 || t >= kTables || A == 0 || (mn >= -zlim && (int64_t)mn + A - 1 < zlim);
-            packed = __all_sync(kFull, fits) ? 1 : 0;
-        }
-        const bool anybad = __any_sync(kFull, bad);
-        if (t == 0) {
-            s_flag[0] = anybad ? 1 : 0;
-            s_flag[1] = packed ? (int)b : kModeCoarse;
-        }
     }
-    __syncthreads();
-    if (s_flag[0]) {
-        if (threadIdx.x == 0) raise_status(kStHeader);
-        return;
-    }
-    const int mode = s_flag[1];
-    const uint16_t* fq = reinterpret_cast<const uint16_t*>(p.ft + table_header_bytes(kTables));
-
     TileCtx tc;
-    tc.nvec = nvec;
-    tc.V = V;
-    tc.T = T;
+    tc.nvec = g.nvec;
+    tc.V = g.V;
+    tc.T = g.T;
     tc.nq = (uint32_t)(p.cols / 8);
-    tc.b = b;
-    tc.cmin = (uint32_t)s_min[0];
-    tc.f0c = fq[0];
-    tc.f1c = s_A[0] == 2 ? (uint32_t)fq[1] : 0u;
-    if (s_A[0] == 1) tc.f0c = M;  // one-symbol coset table: every slot is that symbol
-    const bool bad_c = tc.f0c + tc.f1c != M;
+    tc.b = g.b;
+    tc.total = p.tix[(size_t)kTileWords * g.T];
+    tc.cmin = h[12];
+    if (h[13] == 1) {  // one-symbol coset table: every slot is that symbol
+        tc.f0c = g.M;
+        tc.f1c = 0;
+    } else {
+        tc.f0c = fq[0];
+        tc.f1c = fq[1];
+    }
+    const bool bad_c = tc.f0c + tc.f1c != g.M;
 
-    // cooperative LUT build
-    switch (mode) {
-        case kModePacked9: build_packed<9>(smem, fq, s_min, s_A, s_off, s_flag); break;
-        case kModePacked10: build_packed<10>(smem, fq, s_min, s_A, s_off, s_flag); break;
-        case kModePacked11: build_packed<11>(smem, fq, s_min, s_A, s_off, s_flag); break;
-        default: {
-            const uint32_t k = b < (uint32_t)kCoarseBits ? b : (uint32_t)kCoarseBits;
-            build_coarse(smem, fq, b, b - k, k, s_min, s_A, s_off, s_flag);
+    Ring rg;
+    rg.ring = smem + kOffRing + warp * kRingAllocBytes;
+    rg.ring_s = smem_u32(rg.ring);
+    rg.bar_s = smem_u32(smem + kOffBar + warp * 16);
+    rg.seq = 0;
+    rg.waited = 0;
+    rg.timed_out = false;
+    const uint32_t lut_bar = smem_u32(smem + kOffBar + kWarps * 16);
+    if (lane == 0) {
+        mbar_init(rg.bar_s, 1);
+        mbar_init(rg.bar_s + 8, 1);
+        if (warp == 0) mbar_init(lut_bar, 1);
+        fence_barrier_init();
+    }
+    __syncthreads();  // barrier initialisation and descriptors visible to every warp
+
+    Tile tl;
+    tl.t = 0xFFFFFFFFu;
+    const uint32_t first_i = (uint32_t)warp;
+    {
+        const uint64_t t64 = (uint64_t)blockIdx.x + (uint64_t)first_i * gridDim.x;
+        if (t64 < g.T && !bad_c) tile_begin(tc, p.tiles, p.tix, rg, tl, (uint32_t)t64, lane);
+    }
+
+    // ---- a2: this CTA's slice of the LUT image, a grid-wide arrival, the image into shared memory
+    bool bad = build_lut_slice(g, fq, s_min, s_A, s_off, p.ws, reinterpret_cast<uint16_t*>(smem + kOffLut));
+    __threadfence();          // this thread's image stores, device-wide, before the arrival
+    fence_proxy_async_shared();  // the scratch writes before the bulk copy overwrites them
+    bad = __syncthreads_or(bad) != 0;
+    uint32_t* counter = reinterpret_cast<uint32_t*>(p.ws + kWsCountOffset);
+    uint32_t* badcount = reinterpret_cast<uint32_t*>(p.ws + kWsBadCountOffset);
+    uint32_t* gen = reinterpret_cast<uint32_t*>(p.ws + kWsGenOffset);
+    uint32_t* result = reinterpret_cast<uint32_t*>(p.ws + kWsResultOffset);
+    if (threadIdx.x == 0) {
+        // self-resetting barrier: the last arrival publishes the bad count of this
+        // generation, clears the counters and advances the generation
+        const uint32_t my_gen = ld_acquire_gpu(gen);
+        if (bad) atomicAdd(badcount, 1u);
+        __threadfence();
+        const uint32_t old = atomicInc(counter, gridDim.x - 1);
+        uint32_t spins = 0;
+        if (old == gridDim.x - 1) {
+            result[my_gen & 1u] = atomicExch(badcount, 0u);
+            __threadfence();
+            atomicAdd(gen, 1u);
+        } else {
+            // every CTA of the (cooperative, hence co-resident) grid arrives; bounded wait
+            while (ld_acquire_gpu(gen) == my_gen && spins < kGridSpins) {
+                __nanosleep(32);
+                ++spins;
+            }
+        }
+        const bool arrived = spins < kGridSpins;
+        if (!arrived) raise_status(kStTimeout);
+        s_ok = arrived && ld_acquire_gpu(result + (my_gen & 1u)) == 0u && !bad_c;
+        if (s_ok && blockIdx.x < g.T) {
+            fence_proxy_async_global();  // generic-proxy image stores before the bulk-copy reads
+            mbar_arrive_expect_tx(lut_bar, g.image_bytes);
+            for (uint32_t o = 0; o < g.image_bytes; o += 16384u)
+                bulk_g2s(smem_u32(smem + kOffLut) + o, p.ws + o,
+                         g.image_bytes - o < 16384u ? g.image_bytes - o : 16384u, lut_bar);
         }
     }
-    fence_proxy_async_smem();  // generic writes to the ring area happen before its bulk copies
     __syncthreads();
-    if (s_flag[0] || bad_c) {
-        if (threadIdx.x == 0) raise_status(kStHeader);
+    if (blockIdx.x >= g.T) return;  // no tile for this CTA
+    bool lut_ok = s_ok != 0;
+    if (lut_ok && !mbar_wait(lut_bar, 0)) {
+        lut_ok = false;
+        raise_status(kStTimeout);
+    }
+    lut_ok = __syncthreads_and(lut_ok) != 0;  // one decision for the whole CTA
+    if (!lut_ok) {
+        if (threadIdx.x == 0 && blockIdx.x == 0) raise_status(kStHeader);
+        while (rg.waited < rg.seq && !rg.timed_out) ring_wait_one(rg);  // drain the prologue's copies
         return;
     }
 
-    switch (mode) {
-        case kModePacked9: decode_tiles<DT, PackedLut<9>, 9>(p, PackedLut<9>{smem_u32(smem + kOffLut)}, tc, smem); break;
-        case kModePacked10:
-            decode_tiles<DT, PackedLut<10>, 10>(p, PackedLut<10>{smem_u32(smem + kOffLut)}, tc, smem);
-            break;
-        case kModePacked11:
-            decode_tiles<DT, PackedLut<11>, 11>(p, PackedLut<11>{smem_u32(smem + kOffLut)}, tc, smem);
-            break;
+    const uint32_t lut_s = smem_u32(smem + kOffLut);
+#define EP_PACKED(BB, FF) \
+    decode_tiles<DT>(p.tiles, p.tix, p.scales, p.out, PackedLut<BB, FF>{lut_s}, tc, rg, tl, first_i)
+    switch (g.mode) {
+        case 9: EP_PACKED(9, false); break;
+        case 10: EP_PACKED(10, false); break;
+        case 11: EP_PACKED(11, false); break;
+        case kModeF + 9: EP_PACKED(9, true); break;
+        case kModeF + 10: EP_PACKED(10, true); break;
+        case kModeF + 11: EP_PACKED(11, true); break;
         default: {
-            const uint32_t k = b < (uint32_t)kCoarseBits ? b : (uint32_t)kCoarseBits;
             CoarseLut cl;
-            cl.lut_s = smem_u32(smem + kOffLut);
-            cl.b = b;
-            cl.mmask = M - 1;
-            cl.sh = b - k;
-            cl.nb_shift = k;
+            cl.lut_s = lut_s;
+            cl.b = g.b;
+            cl.mmask = g.M - 1;
+            cl.sh = g.b - g.k;
+            cl.nb_shift = g.k;
             cl.fq = fq;
             cl.s_min = s_min;
             cl.s_A = s_A;
             cl.s_off = s_off;
-            decode_tiles<DT, CoarseLut, 0>(p, cl, tc, smem);
+            decode_tiles<DT>(p.tiles, p.tix, p.scales, p.out, cl, tc, rg, tl, first_i);
         }
     }
+#undef EP_PACKED
 }
 
 // ------------------------------------------------------------- host side
 
-int g_num_sms[64];
-bool g_attr_done[64][8];
+struct DevState {
+    int num_sms = 0;
+    bool attr_done[8] = {};
+    uint8_t* ws = nullptr;         // the LUT workspace of this device
+    cudaEvent_t ws_free = nullptr;  // recorded after every decode that used it
+};
+DevState g_dev[64];
 std::mutex g_mu;
 
 template <int DT>
-cudaError_t launch(const Params& prm, cudaStream_t st, int dev) {
-    {
-        std::lock_guard<std::mutex> lk(g_mu);
-        if (!g_num_sms[dev]) {
-            cudaError_t e = cudaDeviceGetAttribute(&g_num_sms[dev], cudaDevAttrMultiProcessorCount, dev);
-            if (e != cudaSuccess) return e;
-        }
-        if (!g_attr_done[dev][DT]) {
-            cudaError_t e =
-                cudaFuncSetAttribute(decode_kernel<DT>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
-            if (e != cudaSuccess) return e;
-            g_attr_done[dev][DT] = true;
-        }
+cudaError_t set_decode_attr() {
+    return cudaFuncSetAttribute(decode_kernel<DT>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+}
+
+cudaError_t dev_setup(int dev, int dt, DevState*& ds) {
+    std::lock_guard<std::mutex> lk(g_mu);
+    ds = &g_dev[dev];
+    cudaError_t e;
+    if (!ds->num_sms) {
+        e = cudaDeviceGetAttribute(&ds->num_sms, cudaDevAttrMultiProcessorCount, dev);
+        if (e != cudaSuccess) return e;
     }
-    decode_kernel<DT><<<g_num_sms[dev], kThreads, kSmemBytes, st>>>(prm);
-    return cudaGetLastError();
+    if (!ds->ws) {
+        // one workspace per device, zeroed once; the grid barrier in it resets itself
+        void* w = nullptr;
+        e = cudaMalloc(&w, kWsBytes);
+        if (e != cudaSuccess) return e;
+        e = cudaMemset(w, 0, kWsBytes);
+        if (e != cudaSuccess) return e;
+        e = cudaEventCreateWithFlags(&ds->ws_free, cudaEventDisableTiming);
+        if (e != cudaSuccess) return e;
+        ds->ws = static_cast<uint8_t*>(w);
+    }
+    if (!ds->attr_done[dt]) {
+        switch (dt) {
+            case EP_BF16: e = set_decode_attr<EP_BF16>(); break;
+            case EP_FP16: e = set_decode_attr<EP_FP16>(); break;
+            case EP_FP8_E4M3: e = set_decode_attr<EP_FP8_E4M3>(); break;
+            case EP_INT8: e = set_decode_attr<EP_INT8>(); break;
+            case EP_FP32: e = set_decode_attr<EP_FP32>(); break;
+            default: e = set_decode_attr<EP_LATTICE_I32>(); break;
+        }
+        if (e != cudaSuccess) return e;
+        ds->attr_done[dt] = true;
+    }
+    return cudaSuccess;
+}
+
+template <int DT>
+cudaError_t launch_decode(const Params& prm, cudaStream_t st, int num_sms) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)num_sms);  // one CTA per SM; all co-resident (cooperative launch)
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = kSmemBytes;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeCooperative;
+    attr[0].val.cooperative = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, decode_kernel<DT>, prm);
 }
 
 }  // namespace
@@ -768,17 +948,28 @@ ep_status ep_decode_tensor(void* stream, const uint16_t* tiles, const uint32_t* 
         return EP_EINVAL;
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return EP_ECUDA;
-    Params prm{tiles, tile_index, freq_tables, row_scales, out, rows, cols};
+    DevState* ds = nullptr;
+    if (dev_setup(dev, (int)out_dtype, ds) != cudaSuccess) return EP_ECUDA;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
-    cudaError_t e;
-    switch (out_dtype) {
-        case EP_BF16: e = launch<EP_BF16>(prm, st, dev); break;
-        case EP_FP16: e = launch<EP_FP16>(prm, st, dev); break;
-        case EP_FP8_E4M3: e = launch<EP_FP8_E4M3>(prm, st, dev); break;
-        case EP_INT8: e = launch<EP_INT8>(prm, st, dev); break;
-        case EP_FP32: e = launch<EP_FP32>(prm, st, dev); break;
-        default: e = launch<EP_LATTICE_I32>(prm, st, dev); break;
+    // decodes on the device share its workspace: a decode waits (on the GPU)
+    // for the previous one, whatever stream that ran on
+    std::lock_guard<std::mutex> lk(g_mu);
+    cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
+    cudaError_t e = cudaStreamIsCapturing(st, &cap);
+    const bool capturing = e == cudaSuccess && cap != cudaStreamCaptureStatusNone;
+    if (e == cudaSuccess && !capturing) e = cudaStreamWaitEvent(st, ds->ws_free, 0);
+    if (e == cudaSuccess) {
+        Params prm{tiles, tile_index, freq_tables, row_scales, out, ds->ws, rows, cols};
+        switch (out_dtype) {
+            case EP_BF16: e = launch_decode<EP_BF16>(prm, st, ds->num_sms); break;
+            case EP_FP16: e = launch_decode<EP_FP16>(prm, st, ds->num_sms); break;
+            case EP_FP8_E4M3: e = launch_decode<EP_FP8_E4M3>(prm, st, ds->num_sms); break;
+            case EP_INT8: e = launch_decode<EP_INT8>(prm, st, ds->num_sms); break;
+            case EP_FP32: e = launch_decode<EP_FP32>(prm, st, ds->num_sms); break;
+            default: e = launch_decode<EP_LATTICE_I32>(prm, st, ds->num_sms); break;
+        }
     }
+    if (e == cudaSuccess && !capturing) e = cudaEventRecord(ds->ws_free, st);
     return e == cudaSuccess ? EP_OK : EP_ECUDA;
 }
 
@@ -792,14 +983,23 @@ ep_status ep_decode_status(void* stream) {
         cudaSuccess)
         return EP_ECUDA;
     if (cudaStreamSynchronize(st) != cudaSuccess) return EP_ECUDA;
+    if (v & ep::kStTimeout) {
+        // a wait that ran out may leave the grid barrier half-counted: start it afresh
+        int dev = 0;
+        if (cudaGetDevice(&dev) == cudaSuccess && dev >= 0 && dev < 64) {
+            std::lock_guard<std::mutex> lk(ep::g_mu);
+            if (ep::g_dev[dev].ws &&
+                cudaMemset(ep::g_dev[dev].ws + ep::kWsCountOffset, 0, ep::kWsBytes - ep::kWsCountOffset) !=
+                    cudaSuccess)
+                return EP_ECUDA;
+        }
+    }
     if (v & (ep::kStHeader | ep::kStCorrupt | ep::kStTimeout)) return EP_ECORRUPT;
     if (v & ep::kStUnsupported) return EP_EUNSUPPORTED;
     return EP_OK;
 }
 
-}  // extern "C"
-
-extern "C" const char* ep_status_string(ep_status s) {
+const char* ep_status_string(ep_status s) {
     switch (s) {
         case EP_OK: return "ok";
         case EP_EINVAL: return "invalid argument";
@@ -811,3 +1011,5 @@ extern "C" const char* ep_status_string(ep_status s) {
     }
     return "unknown status";
 }
+
+}  // extern "C"

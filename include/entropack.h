@@ -120,14 +120,20 @@ void ep_free_blob(ep_blob* blob);
  *   rows, cols   the matrix shape; must match the header.
  *   out_dtype    one of ep_dtype.
  *   out          device, rows*cols elements of out_dtype, row-major, 16-byte aligned.
- * All buffers belong to the caller; the library allocates no device memory.
- * The call is asynchronous: it validates the arguments on the host, launches
- * one kernel on the stream and returns.  Argument errors return at once
- * (EP_EINVAL, EP_EUNSUPPORTED), launch errors as EP_ECUDA.  The stream itself
- * is checked on the device without trapping: a corrupt payload, state, offset
- * or table raises a device-side status word that ep_decode_status reads.
- * Outputs of a corrupt tile are unspecified; no access leaves the buffers
- * described above.
+ * All buffers belong to the caller.  The library keeps one 128 KB workspace
+ * per device (allocated with cudaMalloc and zeroed on the first call on that
+ * device, so make the first call before any stream capture); every CTA writes
+ * its share of the decode lookup table there and reads the whole table back.
+ * Decodes on one device are ordered through that workspace: a call waits on
+ * the GPU for the previous call, whatever stream it ran on (not applied while
+ * the stream is being captured).
+ * The call is asynchronous: it validates the arguments on the host and makes
+ * one cooperative launch on the stream (one CTA per SM).  Argument errors
+ * return at once (EP_EINVAL, EP_EUNSUPPORTED), launch errors as EP_ECUDA.  The
+ * stream itself is checked on the device without trapping: a corrupt payload,
+ * state, offset or table raises a device-side status word that
+ * ep_decode_status reads.  Outputs of a corrupt tile are unspecified; no access
+ * leaves the buffers described above.
  */
 ep_status ep_decode_tensor(void* stream, const uint16_t* tiles, const uint32_t* tile_index,
                            const uint8_t* freq_tables, const float* row_scales, int64_t rows,
