@@ -85,6 +85,8 @@ def lib() -> C.CDLL:
         L.ep_free_blob.restype = None
         L.ep_decode_tensor.argtypes = [P, P, P, P, P, C.c_int64, C.c_int64, C.c_int, P]
         L.ep_decode_tensor.restype = C.c_int
+        L.ep_decode_tensor_noalloc.argtypes = [P, P, P, P, P, C.c_int64, C.c_int64, C.c_int, P]
+        L.ep_decode_tensor_noalloc.restype = C.c_int
         L.ep_decode_status.argtypes = [P]
         L.ep_decode_status.restype = C.c_int
         L.ep_status_string.argtypes = [C.c_int]
@@ -93,7 +95,8 @@ def lib() -> C.CDLL:
     return _lib
 
 
-EXPORTED = ("ep_encode_tensor", "ep_free_blob", "ep_decode_tensor", "ep_decode_status", "ep_status_string")
+EXPORTED = ("ep_encode_tensor", "ep_free_blob", "ep_decode_tensor", "ep_decode_tensor_noalloc", "ep_decode_status",
+            "ep_status_string")
 
 
 @dataclass
@@ -195,6 +198,22 @@ def decode_tensor(db: DeviceBlob, out_dtype: int = BF16, out=None, stream=None):
                                 int(out_dtype), out.data_ptr())
     if rc:
         raise EntroPackError(rc, "ep_decode_tensor")
+    return out
+
+
+def decode_tensor_noalloc(db: DeviceBlob, out_dtype: int = BF16, out=None, stream=None):
+    """ep_decode_tensor_noalloc: the same decode with the library's fixed device scratch array
+    (no device allocation by the library); calls that overlap on the GPU must be ordered by the caller."""
+    import torch
+
+    if out is None:
+        out = torch.empty((db.rows, db.cols), dtype=_torch_dtype(out_dtype), device=db.payload.device)
+    st = stream if stream is not None else torch.cuda.current_stream(db.payload.device)
+    rc = lib().ep_decode_tensor_noalloc(C.c_void_p(st.cuda_stream), db.payload.data_ptr(), db.tile_index.data_ptr(),
+                                        db.freq_tables.data_ptr(), db.row_scales.data_ptr(), db.rows, db.cols,
+                                        int(out_dtype), out.data_ptr())
+    if rc:
+        raise EntroPackError(rc, "ep_decode_tensor_noalloc")
     return out
 
 

@@ -1013,3 +1013,97 @@ const char* ep_status_string(ep_status s) {
 }
 
 }  // extern "C"
+
+// ----------------------------------------------- decode without allocation
+//
+// ep_decode_tensor_noalloc: the same decode, with its scratch (the decode
+// lookup-table image and the grid-barrier words) in a file-scope device array
+// instead of the workspace ep_decode_tensor allocates.  The array is a
+// host-side stand-in in host code: its device address is taken with
+// cudaGetSymbolAddress once per device, with that device current, on the
+// first call there.
+
+namespace ep {
+namespace {
+
+// 128 KiB of lookup-table image (the largest any stream needs, b <= 15) plus
+// the 32 bytes of barrier state; every GPU that loads the library keeps it.
+constexpr size_t kNoAllocScratchBytes = (size_t)kWsBytes;
+static __device__ __align__(256) uint8_t g_noalloc_scratch[kNoAllocScratchBytes];
+static_assert(kLutBytes + 32 <= (int)kNoAllocScratchBytes, "scratch array too small for the table image");
+
+struct NoAllocState {
+    int num_sms = 0;
+    bool attr_done[8] = {};
+    uint8_t* scratch = nullptr;  // device address of g_noalloc_scratch on this device
+};
+NoAllocState g_noalloc[64];
+std::mutex g_noalloc_mu;
+
+cudaError_t noalloc_setup(int dev, int dt, NoAllocState*& ns) {
+    std::lock_guard<std::mutex> lk(g_noalloc_mu);
+    ns = &g_noalloc[dev];
+    cudaError_t e;
+    if (!ns->num_sms) {
+        e = cudaDeviceGetAttribute(&ns->num_sms, cudaDevAttrMultiProcessorCount, dev);
+        if (e != cudaSuccess) return e;
+    }
+    if (!ns->scratch) {
+        void* ptr = nullptr;
+        e = cudaGetSymbolAddress(&ptr, g_noalloc_scratch);
+        if (e != cudaSuccess) return e;
+        ns->scratch = static_cast<uint8_t*>(ptr);
+    }
+    if (!ns->attr_done[dt]) {
+        switch (dt) {
+            case EP_BF16: e = set_decode_attr<EP_BF16>(); break;
+            case EP_FP16: e = set_decode_attr<EP_FP16>(); break;
+            case EP_FP8_E4M3: e = set_decode_attr<EP_FP8_E4M3>(); break;
+            case EP_INT8: e = set_decode_attr<EP_INT8>(); break;
+            case EP_FP32: e = set_decode_attr<EP_FP32>(); break;
+            default: e = set_decode_attr<EP_LATTICE_I32>(); break;
+        }
+        if (e != cudaSuccess) return e;
+        ns->attr_done[dt] = true;
+    }
+    return cudaSuccess;
+}
+
+}  // namespace
+}  // namespace ep
+
+extern "C" ep_status ep_decode_tensor_noalloc(void* stream, const uint16_t* tiles, const uint32_t* tile_index,
+                                              const uint8_t* freq_tables, const float* row_scales, int64_t rows,
+                                              int64_t cols, ep_dtype out_dtype, void* out) {
+    using namespace ep;
+    if (!tiles || !tile_index || !freq_tables || !row_scales || !out) return EP_EINVAL;
+    if (rows <= 0 || cols <= 0) return EP_EINVAL;
+    if (cols % 8) return EP_EUNSUPPORTED;
+    if ((int)out_dtype < EP_BF16 || (int)out_dtype > EP_LATTICE_I32) return EP_EUNSUPPORTED;
+    // the largest tensor this entry point takes: fewer than 2^31 vectors of eight
+    const int64_t nvec = rows * (cols / 8);
+    if (nvec >= (1ll << 31) || rows >= (1ll << 31)) return EP_EINVAL;
+    auto misaligned = [](const void* q, uintptr_t a) { return (reinterpret_cast<uintptr_t>(q) & (a - 1)) != 0; };
+    if (misaligned(tiles, 16) || misaligned(freq_tables, 16) || misaligned(tile_index, 4) ||
+        misaligned(row_scales, 4) || misaligned(out, 16))
+        return EP_EINVAL;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return EP_ECUDA;
+    NoAllocState* ns = nullptr;
+    if (noalloc_setup(dev, (int)out_dtype, ns) != cudaSuccess) return EP_ECUDA;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    // the barrier words must start at zero; the array keeps whatever the last call left
+    cudaError_t e = cudaMemsetAsync(ns->scratch + kWsCountOffset, 0, kNoAllocScratchBytes - kWsCountOffset, st);
+    if (e == cudaSuccess) {
+        Params prm{tiles, tile_index, freq_tables, row_scales, out, ns->scratch, rows, cols};
+        switch (out_dtype) {
+            case EP_BF16: e = launch_decode<EP_BF16>(prm, st, ns->num_sms); break;
+            case EP_FP16: e = launch_decode<EP_FP16>(prm, st, ns->num_sms); break;
+            case EP_FP8_E4M3: e = launch_decode<EP_FP8_E4M3>(prm, st, ns->num_sms); break;
+            case EP_INT8: e = launch_decode<EP_INT8>(prm, st, ns->num_sms); break;
+            case EP_FP32: e = launch_decode<EP_FP32>(prm, st, ns->num_sms); break;
+            default: e = launch_decode<EP_LATTICE_I32>(prm, st, ns->num_sms); break;
+        }
+    }
+    return e == cudaSuccess ? EP_OK : EP_ECUDA;
+}

@@ -140,6 +140,30 @@ ep_status ep_decode_tensor(void* stream, const uint16_t* tiles, const uint32_t* 
                            int64_t cols, ep_dtype out_dtype, void* out);
 
 /*
+ * ep_decode_tensor_noalloc -- the same decode as ep_decode_tensor, for callers
+ * that cannot allocate device memory: code whose memory is owned by another
+ * allocator (a framework's caching allocator, a memory budget fixed at start-up),
+ * code that must not take the implicit device synchronisation of cudaMalloc
+ * (latency-critical serving loops), and code that runs where allocation is not
+ * permitted.  There is no counterpart in the EntroPack paper; the arguments,
+ * alignment rules, output and status reporting are those of ep_decode_tensor.
+ * Its scratch (the decode lookup-table image and 32 bytes of grid-barrier state,
+ * 131,104 bytes in all: enough for any stream with b <= 15) lives in a
+ * fixed-size device array inside the library; every GPU that loads the library
+ * keeps that array until the process exits.  The call allocates and frees
+ * nothing: on the first call on a device (which must come before any stream
+ * capture) it looks up the array's device address; each call then clears the
+ * barrier words with cudaMemsetAsync and makes one cooperative launch.
+ * Every call shares the array and it keeps the last call's contents, so calls
+ * whose executions overlap on the GPU (for instance on two streams) race on it
+ * and must be ordered by the caller.  Tensors of 2^31 vectors (of 8 weights) or
+ * more are rejected with EP_EINVAL, like every other size error.
+ */
+ep_status ep_decode_tensor_noalloc(void* stream, const uint16_t* tiles, const uint32_t* tile_index,
+                                   const uint8_t* freq_tables, const float* row_scales, int64_t rows,
+                                   int64_t cols, ep_dtype out_dtype, void* out);
+
+/*
  * ep_decode_status -- synchronise `stream`, read and clear the status word of
  * the current device: EP_OK, EP_ECORRUPT (an inconsistent stream or header),
  * or EP_EUNSUPPORTED (a header variant the GPU decoder does not handle).
