@@ -71,13 +71,8 @@ constexpr int kOffDesc = kOffBar + kWarps * 16 + 16;
 constexpr int kSmemBytes = kOffDesc + 3 * 32 * 4;
 
 // LUT workspace (global, one per device, zeroed once): the image, then the
-// state of a self-resetting grid barrier: arrival counter (wraps to 0 on the
-// last arrival), bad-table count of the current generation, generation, and
-// the bad-table result of the last two generations
+// grid barrier's 64-bit arrival counter, which only grows (by G per launch)
 constexpr int kWsCountOffset = kLutBytes;
-constexpr int kWsBadCountOffset = kLutBytes + 4;
-constexpr int kWsGenOffset = kLutBytes + 8;
-constexpr int kWsResultOffset = kLutBytes + 16;  // 2 words
 constexpr int kWsBytes = kLutBytes + 32;
 constexpr uint32_t kGridSpins = 1u << 22;  // bound on the grid-barrier polls
 
@@ -139,9 +134,9 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity) {
 }
 __device__ __forceinline__ void fence_proxy_async_shared() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
 __device__ __forceinline__ void fence_proxy_async_global() { asm volatile("fence.proxy.async.global;" ::: "memory"); }
-__device__ __forceinline__ uint32_t ld_acquire_gpu(const uint32_t* p) {
-    uint32_t v;
-    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+__device__ __forceinline__ unsigned long long ld_acquire_gpu(const unsigned long long* p) {
+    unsigned long long v;
+    asm volatile("ld.acquire.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
     return v;
 }
 __device__ __forceinline__ uint32_t lanemask_lt() {
@@ -241,9 +236,19 @@ __device__ bool build_lut_slice(const Geo& g, const uint16_t* fq, const int* s_m
     const bool fstored = g.mode >= kModeF;
     const uint32_t E = coarse ? (1u << g.k) : g.M;
     const uint32_t sh = coarse ? g.b - g.k : 0u;
-    const uint32_t all = 16u * E;
-    const uint32_t per = (all + gridDim.x - 1) / gridDim.x;
-    const uint32_t e0 = min(all, blockIdx.x * per), e1 = min(all, e0 + per);
+    uint32_t e0, e1;
+    if (gridDim.x >= 16) {
+        // CTAs [ceil(tG/16), ceil((t+1)G/16)) share table t + 1, so no CTA builds two tables
+        const uint32_t G = gridDim.x, t0 = blockIdx.x * 16u / G;
+        const uint32_t bf = (t0 * G + 15u) / 16u, n = ((t0 + 1u) * G + 15u) / 16u - bf, j = blockIdx.x - bf;
+        e0 = t0 * E + (uint32_t)((uint64_t)j * E / n);
+        e1 = t0 * E + (uint32_t)((uint64_t)(j + 1u) * E / n);
+    } else {
+        const uint32_t all = 16u * E;
+        const uint32_t per = (all + gridDim.x - 1) / gridDim.x;
+        e0 = min(all, blockIdx.x * per);
+        e1 = min(all, e0 + per);
+    }
     const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
     bool bad = false;
     if (e0 >= e1) return false;
@@ -306,8 +311,8 @@ __device__ bool build_lut_slice(const Geo& g, const uint16_t* fq, const int* s_m
                 const uint32_t b = g.b;
                 uint32_t e = 0;
                 if (A > 0 && valid)
-                    e = fstored ? (slot - c0) | (f << b) | ((uint32_t)((int)s + mn) << (2 * b + 1))
-                                : (slot - c0) | ((f - 1) << b) | ((uint32_t)((int)s + mn) << (2 * b));
+                    e = fstored ? (slot - c0) | (f << b) | ((uint32_t)((int)s + mn + (1 << (30 - 2 * b))) << (2 * b + 1))
+                                : (slot - c0) | ((f - 1) << b) | ((uint32_t)((int)s + mn + (1 << (31 - 2 * b))) << (2 * b));
                 reinterpret_cast<uint32_t*>(ws)[idx] = e;
             }
         }
@@ -394,25 +399,35 @@ template <int B, bool F>
 struct PackedLut {
     static constexpr uint32_t kM = 1u << B;
     static constexpr int kB = B;
+    static constexpr int kZSh = F ? 2 * B + 1 : 2 * B;
+    static constexpr uint32_t kZBias = F ? (1u << (30 - 2 * B)) : (1u << (31 - 2 * B));
     uint32_t lut_s;
+    uint32_t four;  // 4, 2^32 - 4 * 2^B, -2^(B+1) or -2^B: run-time values, so that the
+    uint32_t m4;    // products below stay integer multiply-adds
+    uint32_t fz;
     __device__ __forceinline__ uint32_t coset_base(int c) const { return lut_s + ((uint32_t)c << (B + 2)); }
     template <int K>
-    __device__ __forceinline__ int decode(uint32_t& x, uint32_t cb, bool& bad) const {
-        const uint32_t e = ld_s32<(2 * (K - 1)) * (int)kM * 4>(cb + ((x & (kM - 1)) << 2));
+    __device__ __forceinline__ uint32_t decode(uint32_t& x, uint32_t cb, bool& bad) const {
         const uint32_t xs = x >> B;
+        const uint32_t a = xs * m4 + (x * four + cb);  // cb + 4 (x mod 2^B)
+        const uint32_t e = ld_s32<(2 * (K - 1)) * (int)kM * 4>(a);
+        const uint32_t zb = e >> kZSh;
+        const uint32_t f = zb * fz + (e >> B);  // f, or f - 1
+        const uint32_t bias = e & (kM - 1);
         if constexpr (F) {
-            x = ((e >> B) & (2 * kM - 1)) * xs + (e & (kM - 1));
+            x = f * xs + bias;
         } else {
-            x = ((e >> B) & (kM - 1)) * xs + (xs + (e & (kM - 1)));
+            x = f * xs + (xs + bias);
         }
         (void)bad;
-        return static_cast<int>(e) >> (F ? 2 * B + 1 : 2 * B);
+        return zb;
     }
 };
 
 // COARSE: 16 tables x 2^k buckets x 64-bit {cum | f << 16, z}; runtime b.
 struct CoarseLut {
     static constexpr int kB = 0;
+    static constexpr uint32_t kZBias = 0;
     uint32_t lut_s;  // shared address
     uint32_t b, mmask, sh, nb_shift;
     const uint16_t* fq;  // global frequencies
@@ -421,7 +436,7 @@ struct CoarseLut {
     const uint32_t* s_off;
     __device__ __forceinline__ uint32_t coset_base(int c) const { return lut_s + ((uint32_t)c << (nb_shift + 3)); }
     template <int K>
-    __device__ __forceinline__ int decode(uint32_t& x, uint32_t cb, bool& bad) const {
+    __device__ __forceinline__ uint32_t decode(uint32_t& x, uint32_t cb, bool& bad) const {
         const uint32_t slot = x & mmask;
         const uint2 e = ld_s64(cb + ((uint32_t)(2 * (K - 1)) << (nb_shift + 3)) + ((slot >> sh) << 3));
         uint32_t c0 = e.x & 0xFFFFu, f = e.x >> 16;
@@ -446,7 +461,7 @@ struct CoarseLut {
             }
         }
         x = f * (x >> b) + (slot - c0);
-        return z;
+        return (uint32_t)z;
     }
 };
 
@@ -488,6 +503,9 @@ struct TileCtx {
     uint32_t V, T, nq, total;
     uint32_t f0c, f1c, cmin;  // coset table: f of symbol 0, of symbol 1, its min
     uint32_t b;
+    // 2, 4, 2^16, -2^b, f1c - f0c, -f0c: run-time multipliers (integer multiply-adds run
+    // beside the shift / logic / compare unit instead of on it)
+    uint32_t two, four, k64, mneg, df, nf0;
 };
 
 // One tile's bookkeeping: record, staging state and every lane's row.
@@ -542,16 +560,18 @@ __device__ __forceinline__ void tile_begin(const TileCtx& tc, const uint16_t* ti
 // below 2^15 take the next words in ascending lane order.  pb is the shared
 // byte address of the next unread word.
 template <bool FULL>
-__device__ __forceinline__ void renorm(uint32_t& x, uint32_t xn, bool act, uint32_t& pb, uint32_t lt) {
+__device__ __forceinline__ void renorm(uint32_t& x, uint32_t xn, bool act, uint32_t& pb, uint32_t lt,
+                                       const TileCtx& tc) {
     const bool need = (FULL || act) && xn < kStateLow;
     const uint32_t bal = __ballot_sync(kFull, need);
-    const uint32_t w = ld_s16(pb + 2u * __popc(bal & lt));
+    const uint32_t w = ld_s16(__popc(bal & lt) * tc.two + pb);
+    const uint32_t xr = xn * tc.k64 + w;  // (xn << 16) | w
     if (FULL) {
-        x = need ? ((xn << 16) | w) : xn;
+        x = need ? xr : xn;
     } else if (act) {
-        x = need ? ((xn << 16) | w) : xn;
+        x = need ? xr : xn;
     }
-    pb += 2u * __popc(bal);
+    pb = __popc(bal) * tc.two + pb;
 }
 
 template <int DT, typename Lut, bool FULL>
@@ -564,24 +584,23 @@ __device__ __forceinline__ void decode_round(void* out, const float sigma, const
     uint32_t x = tl.x;
 
     // ---- a4: field 0, the coset bit (a two-symbol table: one compare)
-    const uint32_t mmask = (Lut::kB > 0 ? (1u << Lut::kB) : (1u << tc.b)) - 1u;
-    const uint32_t slot = x & mmask;
+    const uint32_t xs = Lut::kB > 0 ? (x >> Lut::kB) : (x >> tc.b);
+    const uint32_t slot = xs * tc.mneg + x;
     const uint32_t cs = slot >= tc.f0c ? 1u : 0u;
     {
-        const uint32_t f = cs ? tc.f1c : tc.f0c;
-        const uint32_t bias = cs ? slot - tc.f0c : slot;
-        const uint32_t xn = f * (Lut::kB > 0 ? (x >> Lut::kB) : (x >> tc.b)) + bias;
-        renorm<FULL>(x, xn, act, pb, lt);
+        const uint32_t f = cs * tc.df + tc.f0c;
+        const uint32_t bias = cs * tc.nf0 + slot;
+        renorm<FULL>(x, f * xs + bias, act, pb, lt, tc);
     }
     const int c = (int)(tc.cmin + cs);
     const auto cb = lut.coset_base(c & 1);
     bool badsym = false;
-    int z[8];
+    uint32_t zb[8];
     uint32_t xn;
-#define EP_FIELD(K)                                    \
-    xn = x;                                            \
-    z[K - 1] = lut.template decode<K>(xn, cb, badsym); \
-    renorm<FULL>(x, xn, act, pb, lt);
+#define EP_FIELD(K)                                     \
+    xn = x;                                             \
+    zb[K - 1] = lut.template decode<K>(xn, cb, badsym); \
+    renorm<FULL>(x, xn, act, pb, lt, tc);
     EP_FIELD(1)
     EP_FIELD(2)
     EP_FIELD(3)
@@ -594,23 +613,29 @@ __device__ __forceinline__ void decode_round(void* out, const float sigma, const
     tl.x = x;
     if (badsym && act) corrupt = true;
 
-    // ---- a5: z8 = 2m + parity(z1..z7)
-    const int s7 = z[0] + z[1] + z[2] + z[3] + z[4] + z[5] + z[6];
-    z[7] = 2 * z[7] + (s7 & 1);
+    // ---- a5: z8 = 2m + parity(z1..z7); the bits of 1.5 * 2^22 + (2z + c)/2 for every
+    // coordinate (fields come with an even bias, which leaves the parity alone)
+    const uint32_t s7 = zb[0] + zb[1] + zb[2] + zb[3] + zb[4] + zb[5] + zb[6];
+    const uint32_t magic = 0x4AC00000u + (uint32_t)c - 2u * Lut::kZBias;
+    uint32_t yb[8];
+#pragma unroll
+    for (int k = 0; k < 7; ++k) yb[k] = zb[k] * tc.two + magic;
+    yb[7] = zb[7] * tc.four + ((s7 & 1u) * tc.two + (magic - 2u * Lut::kZBias));
 
     if (act) {
         if constexpr (DT == EP_LATTICE_I32) {
             int4* o = reinterpret_cast<int4*>(out) + 2 * g;
-            o[0] = make_int4(2 * z[0] + c, 2 * z[1] + c, 2 * z[2] + c, 2 * z[3] + c);
-            o[1] = make_int4(2 * z[4] + c, 2 * z[5] + c, 2 * z[6] + c, 2 * z[7] + c);
+            o[0] = make_int4((int)(yb[0] - 0x4AC00000u), (int)(yb[1] - 0x4AC00000u), (int)(yb[2] - 0x4AC00000u),
+                             (int)(yb[3] - 0x4AC00000u));
+            o[1] = make_int4((int)(yb[4] - 0x4AC00000u), (int)(yb[5] - 0x4AC00000u), (int)(yb[6] - 0x4AC00000u),
+                             (int)(yb[7] - 0x4AC00000u));
         } else {
             // ---- a6: w = fl32(sigma * y), y = z + c/2 formed exactly from the bits of
             // 1.5 * 2^22 + (2z + c)/2 (|2z + c| < 2^22), then one FMUL: one rounding
             // for every sigma (zero, subnormal and negative included)
             float w[8];
 #pragma unroll
-            for (int k = 0; k < 8; ++k)
-                w[k] = sigma * (__int_as_float(0x4AC00000 + 2 * z[k] + c) - 6291456.0f);
+            for (int k = 0; k < 8; ++k) w[k] = sigma * (__uint_as_float(yb[k]) - 6291456.0f);
             // ---- a7: conversion + one vector store per lane
             Out<DT>::store(out, g, w);
         }
@@ -706,6 +731,7 @@ struct Params {
     void* out;
     uint8_t* ws;  // LUT image + grid-barrier state
     int64_t rows, cols;
+    uint32_t one;  // 1, set by the host (see TileCtx)
 };
 
 template <int DT>
@@ -747,6 +773,10 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(Params p) {
     tc.T = g.T;
     tc.nq = (uint32_t)(p.cols / 8);
     tc.b = g.b;
+    tc.two = p.one << 1;
+    tc.four = p.one << 2;
+    tc.k64 = p.one << 16;
+    tc.mneg = 0u - (p.one << g.b);
     tc.total = p.tix[(size_t)kTileWords * g.T];
     tc.cmin = h[12];
     if (h[13] == 1) {  // one-symbol coset table: every slot is that symbol
@@ -757,6 +787,8 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(Params p) {
         tc.f1c = fq[1];
     }
     const bool bad_c = tc.f0c + tc.f1c != g.M;
+    tc.df = tc.f1c - tc.f0c;
+    tc.nf0 = 0u - tc.f0c;
 
     Ring rg;
     rg.ring = smem + kOffRing + warp * kRingAllocBytes;
@@ -783,36 +815,27 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(Params p) {
     }
 
     // ---- a2: this CTA's slice of the LUT image, a grid-wide arrival, the image into shared memory
-    bool bad = build_lut_slice(g, fq, s_min, s_A, s_off, p.ws, reinterpret_cast<uint16_t*>(smem + kOffLut));
-    __threadfence();          // this thread's image stores, device-wide, before the arrival
+    // A table that does not sum to 2^b gets zero entries (decoding with them stays in
+    // bounds) and raises the status word; the decode goes on, its output unspecified.
+    const bool bad = build_lut_slice(g, fq, s_min, s_A, s_off, p.ws, reinterpret_cast<uint16_t*>(smem + kOffLut));
+    if (bad && threadIdx.x == 0) raise_status(kStHeader);
     fence_proxy_async_shared();  // the scratch writes before the bulk copy overwrites them
-    bad = __syncthreads_or(bad) != 0;
-    uint32_t* counter = reinterpret_cast<uint32_t*>(p.ws + kWsCountOffset);
-    uint32_t* badcount = reinterpret_cast<uint32_t*>(p.ws + kWsBadCountOffset);
-    uint32_t* gen = reinterpret_cast<uint32_t*>(p.ws + kWsGenOffset);
-    uint32_t* result = reinterpret_cast<uint32_t*>(p.ws + kWsResultOffset);
+    __syncthreads();
     if (threadIdx.x == 0) {
-        // self-resetting barrier: the last arrival publishes the bad count of this
-        // generation, clears the counters and advances the generation
-        const uint32_t my_gen = ld_acquire_gpu(gen);
-        if (bad) atomicAdd(badcount, 1u);
-        __threadfence();
-        const uint32_t old = atomicInc(counter, gridDim.x - 1);
+        __threadfence();  // the CTA's image stores (ordered by the barrier above) before the arrival
+        // the counter grows by G per launch, so the arrival that returns `old` belongs to
+        // the launch that ends at the next multiple of G
+        unsigned long long* arrivals = reinterpret_cast<unsigned long long*>(p.ws + kWsCountOffset);
+        const unsigned long long old = atomicAdd(arrivals, 1ull);
+        const unsigned long long target = (old / gridDim.x + 1ull) * gridDim.x;
         uint32_t spins = 0;
-        if (old == gridDim.x - 1) {
-            result[my_gen & 1u] = atomicExch(badcount, 0u);
-            __threadfence();
-            atomicAdd(gen, 1u);
-        } else {
-            // every CTA of the (cooperative, hence co-resident) grid arrives; bounded wait
-            while (ld_acquire_gpu(gen) == my_gen && spins < kGridSpins) {
-                __nanosleep(32);
-                ++spins;
-            }
+        // every CTA of the (cooperative, hence co-resident) grid arrives; bounded wait
+        while (ld_acquire_gpu(arrivals) < target && spins < kGridSpins) {
+            __nanosleep(32);
+            ++spins;
         }
-        const bool arrived = spins < kGridSpins;
-        if (!arrived) raise_status(kStTimeout);
-        s_ok = arrived && ld_acquire_gpu(result + (my_gen & 1u)) == 0u && !bad_c;
+        s_ok = spins < kGridSpins;
+        if (!s_ok) raise_status(kStTimeout);
         if (s_ok && blockIdx.x < g.T) {
             fence_proxy_async_global();  // generic-proxy image stores before the bulk-copy reads
             mbar_arrive_expect_tx(lut_bar, g.image_bytes);
@@ -829,15 +852,17 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(Params p) {
         raise_status(kStTimeout);
     }
     lut_ok = __syncthreads_and(lut_ok) != 0;  // one decision for the whole CTA
-    if (!lut_ok) {
-        if (threadIdx.x == 0 && blockIdx.x == 0) raise_status(kStHeader);
+    if (!lut_ok || bad_c) {
+        if (bad_c && threadIdx.x == 0 && blockIdx.x == 0) raise_status(kStHeader);
         while (rg.waited < rg.seq && !rg.timed_out) ring_wait_one(rg);  // drain the prologue's copies
         return;
     }
 
     const uint32_t lut_s = smem_u32(smem + kOffLut);
 #define EP_PACKED(BB, FF) \
-    decode_tiles<DT>(p.tiles, p.tix, p.scales, p.out, PackedLut<BB, FF>{lut_s}, tc, rg, tl, first_i)
+    decode_tiles<DT>(p.tiles, p.tix, p.scales, p.out,                                              \
+                     PackedLut<BB, FF>{lut_s, tc.four, 0u - (p.one << (BB + 2)), 0u - (p.one << (FF ? BB + 1 : BB))}, \
+                     tc, rg, tl, first_i)
     switch (g.mode) {
         case 9: EP_PACKED(9, false); break;
         case 10: EP_PACKED(10, false); break;
@@ -959,7 +984,7 @@ ep_status ep_decode_tensor(void* stream, const uint16_t* tiles, const uint32_t* 
     const bool capturing = e == cudaSuccess && cap != cudaStreamCaptureStatusNone;
     if (e == cudaSuccess && !capturing) e = cudaStreamWaitEvent(st, ds->ws_free, 0);
     if (e == cudaSuccess) {
-        Params prm{tiles, tile_index, freq_tables, row_scales, out, ds->ws, rows, cols};
+        Params prm{tiles, tile_index, freq_tables, row_scales, out, ds->ws, rows, cols, 1u};
         switch (out_dtype) {
             case EP_BF16: e = launch_decode<EP_BF16>(prm, st, ds->num_sms); break;
             case EP_FP16: e = launch_decode<EP_FP16>(prm, st, ds->num_sms); break;
@@ -1095,7 +1120,7 @@ extern "C" ep_status ep_decode_tensor_noalloc(void* stream, const uint16_t* tile
     // the barrier words must start at zero; the array keeps whatever the last call left
     cudaError_t e = cudaMemsetAsync(ns->scratch + kWsCountOffset, 0, kNoAllocScratchBytes - kWsCountOffset, st);
     if (e == cudaSuccess) {
-        Params prm{tiles, tile_index, freq_tables, row_scales, out, ns->scratch, rows, cols};
+        Params prm{tiles, tile_index, freq_tables, row_scales, out, ns->scratch, rows, cols, 1u};
         switch (out_dtype) {
             case EP_BF16: e = launch_decode<EP_BF16>(prm, st, ns->num_sms); break;
             case EP_FP16: e = launch_decode<EP_FP16>(prm, st, ns->num_sms); break;
