@@ -1,6 +1,7 @@
 """Benchmark of the fused EntroPack decode on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+    python bench.py --sweep      (every workload, one GPU: a table, not the bench line)
 
 One step = one ep_decode_tensor call: the whole hot path (tile setup, table
 staging, payload staging, rANS decode, lattice reconstruction, row rescale,
@@ -365,6 +366,154 @@ def run_reference(args):
             "e2e": {"value": round(value, 5), "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
 
 
+def _timed_decodes(ep, db, dtype, out, runs: int = 15):
+    """Min and median ms of `runs` decodes, each after an L2 flush (a 256 MiB write), timed with
+    CUDA events on the launching stream after 3 warm-ups."""
+    import torch
+
+    st = torch.cuda.current_stream()
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=out.device)
+    for _ in range(3):
+        ep.decode_tensor(db, dtype, out=out, stream=st)
+    ts = []
+    for _ in range(runs):
+        flush.zero_()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(st)
+        ep.decode_tensor(db, dtype, out=out, stream=st)
+        b.record(st)
+        torch.cuda.synchronize()
+        ts.append(a.elapsed_time(b))
+    if ep.decode_status(st) != 0:
+        raise RuntimeError("decode reported a corrupt stream")
+    return min(ts), statistics.median(ts)
+
+
+def _timed_matmul(rows: int, cols: int, tokens: int = 4096, runs: int = 15):
+    """Min ms of a torch bf16 matmul X[tokens, cols] @ W[rows, cols]^T, same protocol."""
+    import torch
+
+    X = torch.randn(tokens, cols, dtype=torch.bfloat16, device="cuda")
+    W = torch.randn(rows, cols, dtype=torch.bfloat16, device="cuda")
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
+    for _ in range(3):
+        torch.matmul(X, W.t())
+    ts = []
+    for _ in range(runs):
+        flush.zero_()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        torch.matmul(X, W.t())
+        b.record()
+        torch.cuda.synchronize()
+        ts.append(a.elapsed_time(b))
+    return min(ts)
+
+
+def run_sweep(args):
+    """Decode throughput on every workload: the headline's tile-size sweep, the attention
+    projection (BF16, FP16), the FP8 / INT8 containers, the LLM-prefill rate sweep (with
+    rel-L2), the DiT stack (one layer of every kind at every rate, against a bf16 matmul of the
+    same shape with 4096 tokens, and the 30-block total from the per-layer rate allocation), and
+    the oracle decoder on one and on all host cores.  Prints a markdown table and JSON lines."""
+    import torch
+
+    import dit_weight_compression_ep_b200 as ep
+    from dit_weight_compression_ep_b200 import build, synth
+    from dit_weight_compression_ep_b200._lib import _torch_dtype
+
+    build.build()
+    peak, peak_kind = _peaks()
+    out_bytes = {ep.BF16: 2, ep.FP16: 2, ep.FP8_E4M3: 1, ep.INT8: 1, ep.FP32: 4}
+    names = {ep.BF16: "bf16", ep.FP16: "fp16", ep.FP8_E4M3: "e4m3", ep.INT8: "int8", ep.FP32: "fp32"}
+    rows_out = []
+
+    def case(label, blob, dtype, extra=None):
+        db = ep.DeviceBlob(blob)
+        out = torch.empty((blob.rows, blob.cols), dtype=_torch_dtype(dtype), device="cuda")
+        tmin, tmed = _timed_decodes(ep, db, dtype, out)
+        numel = blob.rows * blob.cols
+        nbytes = blob.stored_device_bytes() + numel * out_bytes[dtype]
+        r = {"case": label, "shape": f"{blob.rows}x{blob.cols}", "out": names[dtype], "stored_bpp":
+             round(blob.stored_bpp, 3), "b": blob.b, "V": blob.V, "tiles": blob.ntiles,
+             "us_min": round(tmin * 1e3, 2), "us_median": round(tmed * 1e3, 2),
+             "gweights_s": round(numel / (tmin * 1e-3) / 1e9, 1), "gb_s": round(nbytes / (tmin * 1e-3) / 1e9, 1),
+             "hbm_frac": round(nbytes / (tmin * 1e-3) / 1e9 / peak, 4)}
+        if extra:
+            r.update(extra(out))
+        rows_out.append(r)
+        print(json.dumps(r), flush=True)
+        del db, out
+        return r
+
+    W = synth.generate(synth.headline())
+    for V in (512, 910, 1820, 3640):
+        case(f"headline 4 bpp, V={V}", ep.encode_tensor(W, 4.0, tile_vectors=V), ep.BF16)
+    case("256x512 fp32 t5, 4 bpp, V=512, b=12", ep.encode_tensor(synth.generate(synth.small_fp32()), 4.0,
+                                                                   tile_vectors=512, prob_bits=12), ep.BF16)
+    blob = ep.encode_tensor(synth.generate(synth.dit_attn_proj()), 5.0)
+    for dt in (ep.BF16, ep.FP16):
+        case("DiT attention projection, 5 bpp", blob, dt)
+    src = synth.generate(synth.lowp_source())
+    for kind, dt in (("e4m3", ep.FP8_E4M3), ("int8", ep.INT8)):
+        vals, _ = synth.to_e4m3_container(src) if kind == "e4m3" else synth.to_int8_container(src)
+        case(f"{kind} container, 5 bpp", ep.encode_tensor(vals, 5.0, has_container_scales=True), dt)
+    del src
+    for wide in (True, False):
+        W = synth.generate(synth.llm_prefill(wide))
+        Wt = torch.from_numpy(W).cuda()
+        nrm = float(torch.linalg.vector_norm(Wt))
+
+        def rel_l2(out, Wt=Wt, nrm=nrm):
+            return {"rel_l2": round(float(torch.linalg.vector_norm(out.float() - Wt)) / nrm, 5)}
+
+        for bpp in (2, 3, 4, 5, 6, 7, 8):
+            case(f"LLM prefill, {bpp} bpp", ep.encode_tensor(W, float(bpp)), ep.BF16, rel_l2)
+        del Wt, W
+        torch.cuda.empty_cache()
+    # DiT stack: every kind at every rate (decode speed depends on shape and rate, not on the
+    # block's seed), then the 30-block total from the per-layer rate allocation
+    alloc = synth.dit_stack_bpp()
+    per = {}
+    for kind, (r_, c_) in synth.DIT_KINDS.items():
+        Wk = synth.generate(synth.dit_stack_layer(0, kind))
+        mm = _timed_matmul(r_, c_)
+        for bpp in synth.DIT_BPP_CHOICES:
+            r = case(f"DiT stack {kind}, {bpp} bpp", ep.encode_tensor(Wk, bpp), ep.BF16,
+                     lambda out, mm=mm: {"matmul_4096_us": round(mm * 1e3, 2)})
+            per[(kind, bpp)] = (r["us_min"], mm * 1e3)
+    dec_total = sum(per[(k, bpp)][0] for (_, k), bpp in alloc.items())
+    mm_total = sum(per[(k, bpp)][1] for (_, k), bpp in alloc.items())
+    tot = {"case": "DiT stack, 30 blocks (sum over the allocation)", "decode_ms": round(dec_total / 1e3, 3),
+           "matmul_4096_ms": round(mm_total / 1e3, 3), "decode_over_matmul": round(dec_total / mm_total, 4)}
+    print(json.dumps(tot), flush=True)
+    # the oracle decoder on the headline: one thread and all host cores, bounded samples
+    import oracle
+
+    oracle.build()
+    blob = ep.encode_tensor(synth.generate(synth.headline()), 4.0)
+    cores = os.cpu_count() or 1
+    orc = {}
+    for nth in (1, cores):
+        per_t = max(1, blob.ntiles // (4 * nth))
+        ranges = [(t, min(t + per_t, blob.ntiles)) for t in range(0, blob.ntiles, per_t)][: 2 * nth]
+        t0 = time.time()
+        wts = _oracle_threads(blob, ranges, nth, oracle.BF16)
+        orc[nth] = wts / (time.time() - t0) / 1e9
+    oc = {"case": "oracle decoder, headline sample", "gweights_s_1_thread": round(orc[1], 4),
+          f"gweights_s_{cores}_threads": round(orc[cores], 4)}
+    print(json.dumps(oc), flush=True)
+
+    print("\n| case | shape | out | bpp | V | µs (min / median) | G w/s | GB/s | of HBM | extra |")
+    print("|---|---|---|---|---|---|---|---|---|---|")
+    for r in rows_out:
+        extra = ", ".join(f"{k} {v}" for k, v in r.items() if k in ("rel_l2", "matmul_4096_us"))
+        print(f"| {r['case']} | {r['shape']} | {r['out']} | {r['stored_bpp']} | {r['V']} | {r['us_min']} / "
+              f"{r['us_median']} | {r['gweights_s']} | {r['gb_s']} | {100 * r['hbm_frac']:.1f} % | {extra} |")
+    print(f"\nDiT stack total: decode {tot['decode_ms']} ms vs bf16 matmul (4096 tokens) {tot['matmul_4096_ms']} ms "
+          f"= {100 * tot['decode_over_matmul']:.1f} %; oracle: {oc}; HBM peak {peak} GB/s ({peak_kind})")
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -372,6 +521,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    ap.add_argument("--sweep", action="store_true", help="every workload's decode throughput (one GPU)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
@@ -379,6 +529,9 @@ def main():
     world = int(os.environ.get("WORLD_SIZE", "1"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
 
+    if args.sweep:
+        run_sweep(args)
+        return
     if args.impl == "reference":
         if rank != 0:
             return

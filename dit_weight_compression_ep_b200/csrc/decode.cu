@@ -595,12 +595,26 @@ __device__ __forceinline__ void decode_round(void* out, const float sigma, const
     const int c = (int)(tc.cmin + cs);
     const auto cb = lut.coset_base(c & 1);
     bool badsym = false;
-    uint32_t zb[8];
+    const uint32_t magic = 0x4AC00000u + (uint32_t)c - 2u * Lut::kZBias;
+    uint32_t yb[8];
+    float wf[8];
+    uint32_t s7 = 0;
     uint32_t xn;
-#define EP_FIELD(K)                                     \
-    xn = x;                                             \
-    zb[K - 1] = lut.template decode<K>(xn, cb, badsym); \
-    renorm<FULL>(x, xn, act, pb, lt, tc);
+    // each coordinate's bits as soon as its field is known, so that this work can fill
+    // the gaps of the state chain
+#define EP_FIELD(K)                                               \
+    xn = x;                                                       \
+    {                                                             \
+        const uint32_t z_ = lut.template decode<K>(xn, cb, badsym); \
+        renorm<FULL>(x, xn, act, pb, lt, tc);                     \
+        if (K < 8) {                                              \
+            yb[K - 1] = z_ * tc.two + magic;                      \
+            wf[K - 1] = sigma * (__uint_as_float(yb[K - 1]) - 6291456.0f); \
+            s7 += z_;                                             \
+        } else {                                                  \
+            yb[7] = z_ * tc.four + ((s7 & 1u) * tc.two + (magic - 2u * Lut::kZBias)); \
+        }                                                         \
+    }
     EP_FIELD(1)
     EP_FIELD(2)
     EP_FIELD(3)
@@ -613,15 +627,6 @@ __device__ __forceinline__ void decode_round(void* out, const float sigma, const
     tl.x = x;
     if (badsym && act) corrupt = true;
 
-    // ---- a5: z8 = 2m + parity(z1..z7); the bits of 1.5 * 2^22 + (2z + c)/2 for every
-    // coordinate (fields come with an even bias, which leaves the parity alone)
-    const uint32_t s7 = zb[0] + zb[1] + zb[2] + zb[3] + zb[4] + zb[5] + zb[6];
-    const uint32_t magic = 0x4AC00000u + (uint32_t)c - 2u * Lut::kZBias;
-    uint32_t yb[8];
-#pragma unroll
-    for (int k = 0; k < 7; ++k) yb[k] = zb[k] * tc.two + magic;
-    yb[7] = zb[7] * tc.four + ((s7 & 1u) * tc.two + (magic - 2u * Lut::kZBias));
-
     if (act) {
         if constexpr (DT == EP_LATTICE_I32) {
             int4* o = reinterpret_cast<int4*>(out) + 2 * g;
@@ -630,14 +635,8 @@ __device__ __forceinline__ void decode_round(void* out, const float sigma, const
             o[1] = make_int4((int)(yb[4] - 0x4AC00000u), (int)(yb[5] - 0x4AC00000u), (int)(yb[6] - 0x4AC00000u),
                              (int)(yb[7] - 0x4AC00000u));
         } else {
-            // ---- a6: w = fl32(sigma * y), y = z + c/2 formed exactly from the bits of
-            // 1.5 * 2^22 + (2z + c)/2 (|2z + c| < 2^22), then one FMUL: one rounding
-            // for every sigma (zero, subnormal and negative included)
-            float w[8];
-#pragma unroll
-            for (int k = 0; k < 8; ++k) w[k] = sigma * (__uint_as_float(yb[k]) - 6291456.0f);
-            // ---- a7: conversion + one vector store per lane
-            Out<DT>::store(out, g, w);
+            wf[7] = sigma * (__uint_as_float(yb[7]) - 6291456.0f);
+            Out<DT>::store(out, g, wf);
         }
     }
 }
