@@ -68,7 +68,11 @@ constexpr int kOffLut = 0;
 constexpr int kOffRing = kOffLut + kLutBytes;
 constexpr int kOffBar = kOffRing + kWarps * kRingAllocBytes;  // 2 per warp + 1 for the LUT
 constexpr int kOffDesc = kOffBar + kWarps * 16 + 16;
-constexpr int kSmemBytes = kOffDesc + 3 * 32 * 4;
+constexpr int kOffDesc2 = kOffDesc + 3 * 32 * 4;  // TWO: per table {record address, min}
+constexpr int kSmemBytes = kOffDesc2 + 16 * 8;
+// TWO: slot table in the first 64 KiB of the LUT region, cumulative-count records after it
+constexpr int kTwoRec = 64 * 1024;
+constexpr uint32_t kTwoRecMax = 32 * 1024;  // u16 records: sum over tables 1..16 of (A + 1), + 1
 
 // LUT workspace (global, one per device, zeroed once): the image, then the
 // grid barrier's 64-bit arrival counter, which only grows (by G per launch)
@@ -87,7 +91,7 @@ constexpr uint32_t kWaitSpins = 1u << 20;  // bound on mbarrier polls
 
 // PACKED modes: b (entries hold f - 1) or 16 + b (entries hold f; one add fewer
 // per symbol, needs one more bit); COARSE otherwise.
-enum : int { kModeCoarse = 1, kModeF = 16 };
+enum : int { kModeCoarse = 1, kModeTwo = 2, kModeTwoPair = 3, kModeF = 16 };
 
 }  // namespace
 
@@ -215,9 +219,17 @@ __device__ unsigned parse_header(const uint8_t* ft, int64_t rows, int64_t cols, 
         }
     }
     if (bad) return kStHeader;
-    g.mode = fstored ? kModeF + (int)g.b : (packed ? (int)g.b : kModeCoarse);
+    uint32_t nrec = 1;  // TWO: records of tables 1..16 (A + 1 each) and one pad entry
+#pragma unroll
+    for (int t = 1; t < kTables; ++t) nrec += h[13 + 2 * t] + 1u;
+    const bool two = g.b <= 12 && nrec <= kTwoRecMax;
+    g.mode = fstored ? kModeF + (int)g.b
+                     : (packed ? (int)g.b : (two ? (g.b == 12 ? kModeTwoPair : kModeTwo) : kModeCoarse));
     g.k = g.b < (uint32_t)kCoarseBits ? g.b : (uint32_t)kCoarseBits;
-    g.image_bytes = packed ? 16u * g.M * 4u : 16u * (1u << g.k) * 8u;
+    if (g.mode == kModeTwo || g.mode == kModeTwoPair)
+        g.image_bytes = (uint32_t)kTwoRec + ((2u * nrec + 15u) & ~15u);
+    else
+        g.image_bytes = packed ? 16u * g.M * 4u : 16u * (1u << g.k) * 8u;
     return 0;
 }
 
@@ -234,7 +246,8 @@ __device__ bool build_lut_slice(const Geo& g, const uint16_t* fq, const int* s_m
     __shared__ uint32_t part_sum[kWarps];
     const bool coarse = g.mode == kModeCoarse;
     const bool fstored = g.mode >= kModeF;
-    const uint32_t E = coarse ? (1u << g.k) : g.M;
+    const bool two = g.mode == kModeTwo || g.mode == kModeTwoPair, pair = g.mode == kModeTwoPair;
+    const uint32_t E = coarse ? (1u << g.k) : (pair ? g.M / 2u : g.M);
     const uint32_t sh = coarse ? g.b - g.k : 0u;
     uint32_t e0, e1;
     if (gridDim.x >= 16) {
@@ -289,6 +302,39 @@ __device__ bool build_lut_slice(const Geo& g, const uint16_t* fq, const int* s_m
         bad |= !valid;
         // entries of this table inside [e0, e1)
         const uint32_t lo = max(e0, (uint32_t)(t - 1) * E), hi = min(e1, (uint32_t)t * E);
+        if (two && lo == (uint32_t)(t - 1) * E) {
+            // the CTA holding the table's first entry writes its records: cum_0 .. cum_{A-1}, M
+            // (tables 1..16 back to back, A + 1 records each)
+            uint16_t* rec = reinterpret_cast<uint16_t*>(ws + kTwoRec) + (s_off[t] - s_A[0] + (uint32_t)(t - 1));
+            for (uint32_t q = tid; q <= A; q += kThreads) rec[q] = q < A ? cum[q] : (uint16_t)g.M;
+            if (t == 16 && tid == 0) rec[A + 1] = (uint16_t)g.M;  // pad: a zero entry of the last table reads it
+        }
+        if (two) {
+            for (uint32_t idx = lo + tid; idx < hi; idx += kThreads) {
+                const uint32_t j = idx - (uint32_t)(t - 1) * E;
+                uint32_t e = 0;
+                if (A > 0 && valid) {
+                    // the largest s with cum[s] <= slot owns the slot (zero-frequency symbols
+                    // share their successor's count and are passed over)
+                    const uint32_t slot = pair ? 2u * j : j;
+                    uint32_t l = 0, r = A;
+                    while (r - l > 1) {
+                        const uint32_t mid = (l + r) >> 1;
+                        if (cum[mid] <= slot) l = mid;
+                        else r = mid;
+                    }
+                    e = l;
+                    if (pair) {  // the odd slot's owner, as an offset of at most 15 (15: look further)
+                        uint32_t so = l;
+                        while (so + 1 < A && so < l + 15u && cum[so + 1] <= slot + 1u) ++so;
+                        e |= (so - l) << 12;
+                    }
+                }
+                reinterpret_cast<uint16_t*>(ws)[idx] = (uint16_t)e;
+            }
+            __syncthreads();  // the scratch is reused by the next table
+            continue;
+        }
         for (uint32_t idx = lo + tid; idx < hi; idx += kThreads) {
             const uint32_t j = idx - (uint32_t)(t - 1) * E;  // slot (PACKED) or bucket (COARSE)
             const uint32_t slot = j << sh;
@@ -421,6 +467,46 @@ struct PackedLut {
         }
         (void)bad;
         return zb;
+    }
+};
+
+// TWO: a u16 per slot (b <= 11) or per slot pair (b = 12, PAIR) holding the table-local
+// symbol index s (and, for a pair, the odd slot's offset from it, 15 meaning "at least
+// 15"), then the table's u16 cumulative counts cum[s], cum[s + 1]: f = cum[s + 1] - cum[s],
+// slot - cum[s], z = s + min.  Runtime b.
+template <bool PAIR>
+struct TwoLut {
+    static constexpr int kB = 0;
+    static constexpr uint32_t kZBias = 0;
+    uint32_t lut_s;  // slot table (tables in the order 2(k-1) + c)
+    uint32_t b, mmask, half;  // b, 2^b - 1, 2 * entries per table (bytes per table)
+    uint32_t desc_s;          // shared address of {record address, min} per table (same order)
+    const uint32_t* s_A;      // alphabet sizes, for the escape walk
+    __device__ __forceinline__ uint32_t coset_base(int c) const { return (uint32_t)c; }
+    template <int K>
+    __device__ __forceinline__ uint32_t decode(uint32_t& x, uint32_t c, bool& bad) const {
+        const uint32_t tix = 2u * (K - 1) + c;  // table t - 1
+        const uint2 d = ld_s64<8 * 2 * (K - 1)>(desc_s + 8u * c);
+        const uint32_t slot = x & mmask;
+        const uint32_t xs = x >> b;
+        uint32_t s;
+        if constexpr (PAIR) {
+            const uint32_t e = ld_s16(lut_s + tix * half + (x & (mmask - 1u)));
+            const uint32_t odd = x & 1u;
+            const uint32_t dl = e >> 12;
+            s = odd * dl + (e & 4095u);
+            if (odd && dl == 15u) {  // a run of unused symbols: walk on (bounded by the alphabet)
+                const uint32_t A = s_A[1 + tix];
+                while (s + 1u < A && ld_s16(d.x + 2u * (s + 1u)) <= slot) ++s;
+            }
+        } else {
+            s = ld_s16(lut_s + tix * half + 2u * slot);
+        }
+        const uint32_t ra = d.x + 2u * s;
+        const uint32_t c0 = ld_s16(ra), c1 = ld_s16(ra + 2u);
+        x = (c1 - c0) * xs + (slot - c0);
+        (void)bad;
+        return s + d.y;
     }
 };
 
@@ -765,6 +851,11 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(Params p) {
             s_A[t] = A;
             s_off[t] = incl - A;
         }
+        // TWO: table t's records start after those of tables 1..t-1 (A + 1 each)
+        const uint32_t A0 = __shfl_sync(kFull, A, 0);
+        if (t >= 1 && t < kTables)
+            reinterpret_cast<uint2*>(smem + kOffDesc2)[t - 1] =
+                make_uint2(smem_u32(smem + kOffLut + kTwoRec) + 2u * (incl - A - A0 + (uint32_t)(t - 1)), h[12 + 2 * t]);
     }
     TileCtx tc;
     tc.nvec = g.nvec;
@@ -869,6 +960,18 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(Params p) {
         case kModeF + 9: EP_PACKED(9, true); break;
         case kModeF + 10: EP_PACKED(10, true); break;
         case kModeF + 11: EP_PACKED(11, true); break;
+        case kModeTwo:
+        case kModeTwoPair: {
+            const bool pair = g.mode == kModeTwoPair;
+            const uint32_t desc2 = smem_u32(smem + kOffDesc2);
+            if (pair)
+                decode_tiles<DT>(p.tiles, p.tix, p.scales, p.out,
+                                 TwoLut<true>{lut_s, g.b, g.M - 1u, g.M, desc2, s_A}, tc, rg, tl, first_i);
+            else
+                decode_tiles<DT>(p.tiles, p.tix, p.scales, p.out,
+                                 TwoLut<false>{lut_s, g.b, g.M - 1u, 2u * g.M, desc2, s_A}, tc, rg, tl, first_i);
+            break;
+        }
         default: {
             CoarseLut cl;
             cl.lut_s = lut_s;
