@@ -179,18 +179,28 @@ struct Geo {
     int64_t nvec;
 };
 
-// Parse and check the table header (every thread reads the same words, so the
-// result is uniform).  Returns 0, kStHeader or kStUnsupported.
-__device__ unsigned parse_header(const uint8_t* ft, int64_t rows, int64_t cols, Geo& g) {
-    // the 192 header bytes in twelve independent 16-byte loads (one round trip)
-    uint32_t h[48];
+// Parse and check the table header.  Every warp reads the same words and takes
+// the same decisions, so the result is uniform; lane t (t < 17) also returns
+// table t's {min, A}.  The checks are lane-parallel and division-free: this
+// code runs once per CTA, cold, so its length is what it costs.  Returns 0,
+// kStHeader or kStUnsupported.
+__device__ unsigned parse_header(const uint8_t* ft, int64_t rows, int64_t cols, Geo& g, int& mn, uint32_t& A) {
+    const int lane = threadIdx.x & 31;
+    uint32_t h[12];
 #pragma unroll
-    for (int i = 0; i < 12; ++i) {
+    for (int i = 0; i < 3; ++i) {
         const uint4 v = __ldg(reinterpret_cast<const uint4*>(ft) + i);
         h[4 * i] = v.x;
         h[4 * i + 1] = v.y;
         h[4 * i + 2] = v.z;
         h[4 * i + 3] = v.w;
+    }
+    mn = 0;
+    A = 0;
+    if (lane < kTables) {
+        const uint2 d = __ldg(reinterpret_cast<const uint2*>(ft + kHeaderFixedBytes) + lane);
+        mn = static_cast<int>(d.x);
+        A = d.y;
     }
     g.b = h[kHB];
     g.V = h[kHV];
@@ -199,29 +209,28 @@ __device__ unsigned parse_header(const uint8_t* ft, int64_t rows, int64_t cols, 
     const int64_t hrows = (int64_t)(((uint64_t)h[2 * kHRows64 + 1] << 32) | h[2 * kHRows64]);
     const int64_t hcols = (int64_t)(((uint64_t)h[2 * kHCols64 + 1] << 32) | h[2 * kHCols64]);
     bool ok = h[kHMagic] == kMagic && h[kHVersion] == kVersion && h[kHJ] == (uint32_t)kLanes &&
-              g.b >= (uint32_t)kMinB && g.b <= (uint32_t)kMaxB && g.V >= 1 && hrows == rows && hcols == cols;
-    ok = ok && (int64_t)g.T == (g.nvec + g.V - 1) / g.V;
+              g.b >= (uint32_t)kMinB && g.b <= (uint32_t)kMaxB && g.V >= 1 && g.T >= 1 && hrows == rows &&
+              hcols == cols;
+    // T = ceil(nvec / V): (T - 1) V < nvec <= T V
+    ok = ok && (uint64_t)g.T * g.V >= (uint64_t)g.nvec && (uint64_t)(g.T - 1) * g.V < (uint64_t)g.nvec;
     if (!ok) return kStHeader;
     if (h[kHNTab] != (uint32_t)kTables || h[kHFlags] != 0u) return kStUnsupported;
     g.M = 1u << g.b;
-    bool packed = g.b <= 11, fstored = g.b <= 11, bad = false;
+    // per table (one lane each): alphabet within 2^b, the coset table {0, 1}-valued; whether
+    // z fits the packed entry with (fstored) and without the extra f bit
     const int bb = g.b <= 11 ? (int)g.b : 11;
     const int64_t zlim = 1ll << (31 - 2 * bb), zlim_f = 1ll << (30 - 2 * bb);
-#pragma unroll
-    for (int t = 0; t < kTables; ++t) {
-        const int mn = static_cast<int>(h[12 + 2 * t]);
-        const uint32_t A = h[13 + 2 * t];
-        bad |= A > g.M;
-        if (t == 0) bad |= A < 1 || A > 2 || mn < 0 || mn + (int)A > 2;
-        if (t > 0 && A > 0) {
-            packed &= mn >= -zlim && (int64_t)mn + A - 1 < zlim;
-            fstored &= mn >= -zlim_f && (int64_t)mn + A - 1 < zlim_f;
-        }
-    }
-    if (bad) return kStHeader;
-    uint32_t nrec = 1;  // TWO: records of tables 1..16 (A + 1 each) and one pad entry
-#pragma unroll
-    for (int t = 1; t < kTables; ++t) nrec += h[13 + 2 * t] + 1u;
+    bool badt = A > g.M;
+    if (lane == 0) badt |= A < 1 || A > 2 || mn < 0 || mn + (int)A > 2;
+    const bool coord = lane >= 1 && lane < kTables && A > 0;
+    const int64_t zhi = (int64_t)mn + A - 1;
+    const bool pk = !coord || (mn >= -zlim && zhi < zlim);
+    const bool fs = !coord || (mn >= -zlim_f && zhi < zlim_f);
+    if (__any_sync(kFull, badt)) return kStHeader;
+    const bool packed = g.b <= 11 && __all_sync(kFull, pk);
+    const bool fstored = g.b <= 11 && __all_sync(kFull, fs);
+    // TWO: records of tables 1..16 (A + 1 each) and one pad entry
+    const uint32_t nrec = 1u + __reduce_add_sync(kFull, lane >= 1 && lane < kTables ? A + 1u : 0u);
     const bool two = g.b <= 12 && nrec <= kTwoRecMax;
     g.mode = fstored ? kModeF + (int)g.b
                      : (packed ? (int)g.b : (two ? (g.b == 12 ? kModeTwoPair : kModeTwo) : kModeCoarse));
@@ -241,8 +250,11 @@ __device__ unsigned parse_header(const uint8_t* ft, int64_t rows, int64_t cols, 
 // CTA scans the frequencies into cumulative counts (u16; M <= 2^15) in shared
 // scratch and finds the owner of every slot by binary search.  Returns true
 // when a touched table does not sum to 2^b.
-__device__ bool build_lut_slice(const Geo& g, const uint16_t* fq, const int* s_min, const uint32_t* s_A,
-                                const uint32_t* s_off, uint8_t* ws, uint16_t* scratch) {
+constexpr int kPre = 6;  // a table of up to kPre * kThreads symbols comes in with the prologue's loads
+
+__device__ __forceinline__ bool build_lut_slice(const Geo& g, const uint16_t* fq, const int* s_min,
+                                                const uint32_t* s_A, const uint32_t* s_off, uint8_t* ws,
+                                                uint16_t* scratch, int t_pre, const uint32_t (&fr)[kPre]) {
     __shared__ uint32_t part_sum[kWarps];
     const bool coarse = g.mode == kModeCoarse;
     const bool fstored = g.mode >= kModeF;
@@ -254,8 +266,8 @@ __device__ bool build_lut_slice(const Geo& g, const uint16_t* fq, const int* s_m
         // CTAs [ceil(tG/16), ceil((t+1)G/16)) share table t + 1, so no CTA builds two tables
         const uint32_t G = gridDim.x, t0 = blockIdx.x * 16u / G;
         const uint32_t bf = (t0 * G + 15u) / 16u, n = ((t0 + 1u) * G + 15u) / 16u - bf, j = blockIdx.x - bf;
-        e0 = t0 * E + (uint32_t)((uint64_t)j * E / n);
-        e1 = t0 * E + (uint32_t)((uint64_t)(j + 1u) * E / n);
+        e0 = t0 * E + j * E / n;  // j < n <= G, E <= 2^15
+        e1 = t0 * E + (j + 1u) * E / n;
     } else {
         const uint32_t all = 16u * E;
         const uint32_t per = (all + gridDim.x - 1) / gridDim.x;
@@ -271,7 +283,15 @@ __device__ bool build_lut_slice(const Geo& g, const uint16_t* fq, const int* s_m
         const uint32_t A = s_A[t], off = s_off[t];
         const int mn = s_min[t];
         // frequencies into shared memory, then an in-place exclusive scan by contiguous chunks
-        for (uint32_t q = tid; q < A; q += kThreads) cum[q] = fq[off + q];
+        if (t == t_pre) {  // frequencies already in registers
+#pragma unroll
+            for (int k = 0; k < kPre; ++k) {
+                const uint32_t q = (uint32_t)tid + (uint32_t)k * kThreads;
+                if (q < A) cum[q] = (uint16_t)fr[k];
+            }
+        } else {
+            for (uint32_t q = tid; q < A; q += kThreads) cum[q] = fq[off + q];
+        }
         __syncthreads();
         const uint32_t chunk = (A + kThreads - 1) / kThreads;
         const uint32_t q0 = min(A, tid * chunk), q1 = min(A, q0 + chunk);
@@ -633,9 +653,10 @@ __device__ __forceinline__ void tile_begin(const TileCtx& tc, const uint16_t* ti
     tl.org = (tl.seq0 & 1u) * kChunkWords;
     if (tl.nchunks > 0) tile_issue_chunk(tiles, rg, tl, 0, lane);
     if (tl.nchunks > 1) tile_issue_chunk(tiles, rg, tl, 1, lane);
-    const int64_t rowbase = tl.v0 / tc.nq;
-    tl.ql = (uint32_t)(tl.v0 - rowbase * tc.nq) + lane;
-    tl.rowl = (uint32_t)rowbase;
+    const uint32_t v0 = (uint32_t)tl.v0;  // < nvec < 2^31
+    const uint32_t rowbase = v0 / tc.nq;
+    tl.ql = v0 - rowbase * tc.nq + lane;
+    tl.rowl = rowbase;
     while (tl.ql >= tc.nq) {
         tl.ql -= tc.nq;
         ++tl.rowl;
@@ -830,16 +851,35 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(Params p) {
 
     // ---- prologue: header, descriptors, barriers, the first chunks of every warp's first tile
     Geo g;
-    const unsigned hs = parse_header(p.ft, p.rows, p.cols, g);
+    int lane_mn;
+    uint32_t lane_A;
+    const unsigned hs = parse_header(p.ft, p.rows, p.cols, g, lane_mn, lane_A);
     if (hs) {  // every CTA reads the same header, so every CTA leaves here
         if (threadIdx.x == 0 && blockIdx.x == 0) raise_status(hs);
         return;
     }
-    const uint32_t* h = reinterpret_cast<const uint32_t*>(p.ft);
     const uint16_t* fq = reinterpret_cast<const uint16_t*>(p.ft + table_header_bytes(kTables));
+    // This CTA's table (one per CTA when G >= 16): its frequencies into registers now, so
+    // that these loads, the coset table's, the tile records and the first payload chunks are
+    // in flight together.
+    uint32_t fr[kPre];
+    int t_pre = 0;
+    if (gridDim.x >= 16 && g.mode != kModeCoarse) {
+        const int t = 1 + (int)(blockIdx.x * 16u / gridDim.x);
+        const uint32_t At = __shfl_sync(kFull, lane_A, t);
+        const uint32_t offt = __reduce_add_sync(kFull, lane < t ? lane_A : 0u);
+        if (At <= (uint32_t)(kPre * kThreads)) {
+            t_pre = t;
+#pragma unroll
+            for (int k = 0; k < kPre; ++k) {
+                const uint32_t q = threadIdx.x + (uint32_t)k * kThreads;
+                fr[k] = q < At ? fq[offt + q] : 0u;
+            }
+        }
+    }
     if (threadIdx.x < 32) {
         const int t = threadIdx.x;
-        const uint32_t A = t < kTables ? h[13 + 2 * t] : 0u;
+        const uint32_t A = lane_A;
         uint32_t incl = A;
 #pragma unroll
         for (int o = 1; o < 32; o <<= 1) {
@@ -847,7 +887,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(Params p) {
             if (t >= o) incl += v;
         }
         if (t < kTables) {
-            s_min[t] = static_cast<int>(h[12 + 2 * t]);
+            s_min[t] = lane_mn;
             s_A[t] = A;
             s_off[t] = incl - A;
         }
@@ -855,7 +895,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(Params p) {
         const uint32_t A0 = __shfl_sync(kFull, A, 0);
         if (t >= 1 && t < kTables)
             reinterpret_cast<uint2*>(smem + kOffDesc2)[t - 1] =
-                make_uint2(smem_u32(smem + kOffLut + kTwoRec) + 2u * (incl - A - A0 + (uint32_t)(t - 1)), h[12 + 2 * t]);
+                make_uint2(smem_u32(smem + kOffLut + kTwoRec) + 2u * (incl - A - A0 + (uint32_t)(t - 1)), (uint32_t)lane_mn);
     }
     TileCtx tc;
     tc.nvec = g.nvec;
@@ -868,8 +908,8 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(Params p) {
     tc.k64 = p.one << 16;
     tc.mneg = 0u - (p.one << g.b);
     tc.total = p.tix[(size_t)kTileWords * g.T];
-    tc.cmin = h[12];
-    if (h[13] == 1) {  // one-symbol coset table: every slot is that symbol
+    tc.cmin = (uint32_t)__shfl_sync(kFull, lane_mn, 0);
+    if (__shfl_sync(kFull, lane_A, 0) == 1u) {  // one-symbol coset table: every slot is that symbol
         tc.f0c = g.M;
         tc.f1c = 0;
     } else {
@@ -901,13 +941,14 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(Params p) {
     const uint32_t first_i = (uint32_t)warp;
     {
         const uint64_t t64 = (uint64_t)blockIdx.x + (uint64_t)first_i * gridDim.x;
-        if (t64 < g.T && !bad_c) tile_begin(tc, p.tiles, p.tix, rg, tl, (uint32_t)t64, lane);
+        if (t64 < g.T) tile_begin(tc, p.tiles, p.tix, rg, tl, (uint32_t)t64, lane);
     }
 
     // ---- a2: this CTA's slice of the LUT image, a grid-wide arrival, the image into shared memory
     // A table that does not sum to 2^b gets zero entries (decoding with them stays in
     // bounds) and raises the status word; the decode goes on, its output unspecified.
-    const bool bad = build_lut_slice(g, fq, s_min, s_A, s_off, p.ws, reinterpret_cast<uint16_t*>(smem + kOffLut));
+    const bool bad = build_lut_slice(g, fq, s_min, s_A, s_off, p.ws, reinterpret_cast<uint16_t*>(smem + kOffLut),
+                                     t_pre, fr);
     if (bad && threadIdx.x == 0) raise_status(kStHeader);
     fence_proxy_async_shared();  // the scratch writes before the bulk copy overwrites them
     __syncthreads();
@@ -917,7 +958,12 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(Params p) {
         // the launch that ends at the next multiple of G
         unsigned long long* arrivals = reinterpret_cast<unsigned long long*>(p.ws + kWsCountOffset);
         const unsigned long long old = atomicAdd(arrivals, 1ull);
-        const unsigned long long target = (old / gridDim.x + 1ull) * gridDim.x;
+        // old / G without a 64-bit integer division: a double quotient (old < 2^53), corrected
+        const unsigned long long G = gridDim.x;
+        unsigned long long q = (unsigned long long)((double)old / (double)G);
+        q -= q * G > old ? 1ull : 0ull;
+        q += (q + 1ull) * G <= old ? 1ull : 0ull;
+        const unsigned long long target = (q + 1ull) * G;
         uint32_t spins = 0;
         // every CTA of the (cooperative, hence co-resident) grid arrives; bounded wait
         while (ld_acquire_gpu(arrivals) < target && spins < kGridSpins) {
