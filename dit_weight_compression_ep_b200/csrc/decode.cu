@@ -305,11 +305,9 @@ __device__ __forceinline__ bool build_lut_slice(const Geo& g, const uint16_t* fq
         }
         if (lane == 31) part_sum[wid] = incl;
         __syncthreads();
-        uint32_t before = 0, total = 0;
-        for (int w = 0; w < kWarps; ++w) {
-            if (w < wid) before += part_sum[w];
-            total += part_sum[w];
-        }
+        const uint32_t ps = lane < kWarps ? part_sum[lane] : 0u;
+        const uint32_t before = __reduce_add_sync(kFull, lane < wid ? ps : 0u);
+        const uint32_t total = __reduce_add_sync(kFull, ps);
         uint32_t run = before + incl - local;
         for (uint32_t q = q0; q < q1; ++q) {
             const uint32_t f = cum[q];
@@ -377,8 +375,8 @@ __device__ __forceinline__ bool build_lut_slice(const Geo& g, const uint16_t* fq
                 const uint32_t b = g.b;
                 uint32_t e = 0;
                 if (A > 0 && valid)
-                    e = fstored ? (slot - c0) | (f << b) | ((uint32_t)((int)s + mn + (1 << (30 - 2 * b))) << (2 * b + 1))
-                                : (slot - c0) | ((f - 1) << b) | ((uint32_t)((int)s + mn + (1 << (31 - 2 * b))) << (2 * b));
+                    e = fstored ? f | ((uint32_t)((int)s + mn + (1 << (30 - 2 * b))) << (b + 1)) | ((slot - c0) << (32 - b))
+                                : (f - 1) | ((uint32_t)((int)s + mn + (1 << (31 - 2 * b))) << b) | ((slot - c0) << (32 - b));
                 reinterpret_cast<uint32_t*>(ws)[idx] = e;
             }
         }
@@ -459,27 +457,26 @@ struct Out<EP_FP32> {
 // ------------------------------------------------------------- symbol LUTs
 
 // PACKED: 16 tables x 2^B slots x 32-bit entries at shared address lut_s;
-// table (2(k-1) + c).  F: the entry holds f in B+1 bits (z in 31 - 2B bits),
-// otherwise f - 1 in B bits (z in 32 - 2B bits).
+// table (2(k-1) + c).  Entry, low to high: f in B+1 bits (F) or f - 1 in B bits,
+// then z with an even bias (31 - 2B or 32 - 2B bits), then slot - cum in the top
+// B bits, so that f and slot - cum each come out in one operation.
 template <int B, bool F>
 struct PackedLut {
     static constexpr uint32_t kM = 1u << B;
     static constexpr int kB = B;
-    static constexpr int kZSh = F ? 2 * B + 1 : 2 * B;
     static constexpr uint32_t kZBias = F ? (1u << (30 - 2 * B)) : (1u << (31 - 2 * B));
     uint32_t lut_s;
-    uint32_t four;  // 4, 2^32 - 4 * 2^B, -2^(B+1) or -2^B: run-time values, so that the
-    uint32_t m4;    // products below stay integer multiply-adds
-    uint32_t fz;
+    uint32_t four;  // 4 and 2^32 - 4 * 2^B: run-time values, so that the address
+    uint32_t m4;    // arithmetic stays integer multiply-adds
     __device__ __forceinline__ uint32_t coset_base(int c) const { return lut_s + ((uint32_t)c << (B + 2)); }
     template <int K>
     __device__ __forceinline__ uint32_t decode(uint32_t& x, uint32_t cb, bool& bad) const {
         const uint32_t xs = x >> B;
         const uint32_t a = xs * m4 + (x * four + cb);  // cb + 4 (x mod 2^B)
         const uint32_t e = ld_s32<(2 * (K - 1)) * (int)kM * 4>(a);
-        const uint32_t zb = e >> kZSh;
-        const uint32_t f = zb * fz + (e >> B);  // f, or f - 1
-        const uint32_t bias = e & (kM - 1);
+        const uint32_t f = e & (F ? 2u * kM - 1u : kM - 1u);
+        const uint32_t bias = e >> (32 - B);
+        const uint32_t zb = (e << B) >> (F ? 2 * B + 1 : 2 * B);
         if constexpr (F) {
             x = f * xs + bias;
         } else {
@@ -633,9 +630,9 @@ __device__ __forceinline__ void tile_issue_chunk(const uint16_t* tiles, Ring& rg
     ring_issue(rg, tiles + w0, n, lane);
 }
 
-// Read the tile record, check it, and start staging its first two chunks.
-__device__ __forceinline__ void tile_begin(const TileCtx& tc, const uint16_t* tiles, const uint32_t* tix, Ring& rg,
-                                           Tile& tl, uint32_t t, int lane) {
+// Read the tile record (loads only: the caller may issue other loads before the
+// values are used).
+__device__ __forceinline__ void tile_load(const TileCtx& tc, const uint32_t* tix, Tile& tl, uint32_t t, int lane) {
     tl.t = t;
     tl.v0 = (int64_t)t * tc.V;
     tl.vt = (uint32_t)((tc.nvec - tl.v0) < (int64_t)tc.V ? (tc.nvec - tl.v0) : (int64_t)tc.V);
@@ -644,6 +641,10 @@ __device__ __forceinline__ void tile_begin(const TileCtx& tc, const uint16_t* ti
     tl.off0 = rec[0];
     tl.off1 = rec[kTileWords];
     tl.x = rec[1 + lane];
+}
+
+// Check the tile record and start staging its first two chunks.
+__device__ __forceinline__ void tile_start(const TileCtx& tc, const uint16_t* tiles, Ring& rg, Tile& tl, int lane) {
     const bool bad = !(tl.off0 <= tl.off1 && tl.off1 <= tc.total) || tl.x < kStateLow || tl.x >= 0x80000000u;
     tl.ok = !__any_sync(kFull, bad);
     tl.base = tl.off0 & ~7u;
@@ -661,6 +662,12 @@ __device__ __forceinline__ void tile_begin(const TileCtx& tc, const uint16_t* ti
         tl.ql -= tc.nq;
         ++tl.rowl;
     }
+}
+
+__device__ __forceinline__ void tile_begin(const TileCtx& tc, const uint16_t* tiles, const uint32_t* tix, Ring& rg,
+                                           Tile& tl, uint32_t t, int lane) {
+    tile_load(tc, tix, tl, t, lane);
+    tile_start(tc, tiles, rg, tl, lane);
 }
 
 // Renormalisation of every lane after one symbol: the lanes whose state fell
@@ -907,6 +914,12 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(Params p) {
     tc.four = p.one << 2;
     tc.k64 = p.one << 16;
     tc.mneg = 0u - (p.one << g.b);
+    // the first tile's record, in flight with the loads above and below
+    Tile tl;
+    tl.t = 0xFFFFFFFFu;
+    const uint32_t first_i = (uint32_t)warp;
+    const uint64_t t_first = (uint64_t)blockIdx.x + (uint64_t)first_i * gridDim.x;
+    if (t_first < g.T) tile_load(tc, p.tix, tl, (uint32_t)t_first, lane);
     tc.total = p.tix[(size_t)kTileWords * g.T];
     tc.cmin = (uint32_t)__shfl_sync(kFull, lane_mn, 0);
     if (__shfl_sync(kFull, lane_A, 0) == 1u) {  // one-symbol coset table: every slot is that symbol
@@ -916,9 +929,6 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(Params p) {
         tc.f0c = fq[0];
         tc.f1c = fq[1];
     }
-    const bool bad_c = tc.f0c + tc.f1c != g.M;
-    tc.df = tc.f1c - tc.f0c;
-    tc.nf0 = 0u - tc.f0c;
 
     Ring rg;
     rg.ring = smem + kOffRing + warp * kRingAllocBytes;
@@ -936,13 +946,10 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(Params p) {
     }
     __syncthreads();  // barrier initialisation and descriptors visible to every warp
 
-    Tile tl;
-    tl.t = 0xFFFFFFFFu;
-    const uint32_t first_i = (uint32_t)warp;
-    {
-        const uint64_t t64 = (uint64_t)blockIdx.x + (uint64_t)first_i * gridDim.x;
-        if (t64 < g.T) tile_begin(tc, p.tiles, p.tix, rg, tl, (uint32_t)t64, lane);
-    }
+    if (t_first < g.T) tile_start(tc, p.tiles, rg, tl, lane);
+    const bool bad_c = tc.f0c + tc.f1c != g.M;
+    tc.df = tc.f1c - tc.f0c;
+    tc.nf0 = 0u - tc.f0c;
 
     // ---- a2: this CTA's slice of the LUT image, a grid-wide arrival, the image into shared memory
     // A table that does not sum to 2^b gets zero entries (decoding with them stays in
@@ -997,7 +1004,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(Params p) {
     const uint32_t lut_s = smem_u32(smem + kOffLut);
 #define EP_PACKED(BB, FF) \
     decode_tiles<DT>(p.tiles, p.tix, p.scales, p.out,                                              \
-                     PackedLut<BB, FF>{lut_s, tc.four, 0u - (p.one << (BB + 2)), 0u - (p.one << (FF ? BB + 1 : BB))}, \
+                     PackedLut<BB, FF>{lut_s, tc.four, 0u - (p.one << (BB + 2))},                      \
                      tc, rg, tl, first_i)
     switch (g.mode) {
         case 9: EP_PACKED(9, false); break;
