@@ -55,10 +55,14 @@ def _peaks():
 
 
 def _kernel_sha():
+    """Hash of the decoder's source without comments and blank space (a comment edit keeps it)."""
+    import re
+
     h = hashlib.sha256()
     for p in ("dit_weight_compression_ep_b200/csrc/decode.cu", "dit_weight_compression_ep_b200/csrc/ep_format.h"):
-        with open(os.path.join(ROOT, p), "rb") as f:
-            h.update(f.read())
+        with open(os.path.join(ROOT, p), encoding="utf-8") as f:
+            code = re.sub(r"//[^\n]*", "", f.read())
+        h.update(" ".join(code.split()).encode())
     return h.hexdigest()[:16]
 
 

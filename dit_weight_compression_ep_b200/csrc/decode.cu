@@ -6,18 +6,25 @@
 // decoder lookup tables ("in shared memory or packed global memory").
 //
 // One call = one cooperative launch of decode_kernel on the caller's stream:
-// one persistent CTA of 24 warps per SM (all co-resident).  Its prologue reads
-// the header and starts staging every warp's first tile; then every CTA builds
-// 1/G of the decode-LUT image in a stream-ordered global workspace (binary
-// search of every slot in its table's cumulative frequencies):
-//   PACKED (b <= 11 and |z| small): 32-bit entry per slot, either
-//     [bias = slot - cum : b][f : b+1][z : 31 - 2b, signed] or
-//     [bias : b][f - 1 : b][z : 32 - 2b, signed] when z needs the extra bit;
-//   COARSE (otherwise): 64-bit entry per bucket of 2^(b-k) slots (k <= 10)
-//     {cum | f << 16, z} of the symbol owning the bucket's first slot;
-// arrives on a grid-wide counter, waits (bounded) for every CTA, and copies
-// the whole image into shared memory with cp.async.bulk.  Tile t goes to CTA
-// t mod G and, within the CTA, to warp (t / G) mod 24.
+// one persistent CTA of 24 warps per SM (all co-resident).  Its prologue parses
+// the header (lane-parallel checks: it runs once, from a cold instruction cache,
+// so its length is its cost) and loads, together, the tables' frequencies of
+// this CTA's table, the coset table and every warp's first tile record.  Then
+// the CTAs sharing a table (G/16 of them) build its part of the decode-LUT image
+// in a stream-ordered global workspace (binary search of every slot in the
+// table's cumulative frequencies), arrive on a 64-bit grid counter, wait
+// (bounded) for every CTA, and copy the whole image into shared memory with
+// cp.async.bulk.  Three image formats (16 coordinate tables, table 2(k-1) + c):
+//   PACKED (b <= 11, z fits): a 32-bit entry per slot, low to high
+//     [f : b+1][z + even bias][slot - cum : b], or [f - 1 : b][z][slot - cum : b]
+//     when z needs the extra bit;
+//   TWO (b <= 12 otherwise, the alphabets small enough): a u16 symbol index per
+//     slot (per slot pair at b = 12, the odd slot's offset in 4 bits) and the
+//     tables' u16 cumulative counts: f = cum[s+1] - cum[s], z = s + min;
+//   COARSE (otherwise): a 64-bit entry per bucket of 2^(b-k) slots (k <= 10)
+//     {cum | f << 16, z} of the symbol owning the bucket's first slot, and a
+//     bounded walk over the global frequencies.
+// Tile t goes to CTA t mod G and, within the CTA, to warp (t / G) mod 24.
 // Per warp and tile:
 //   a1  32 terminal states (one per lane), the tile's payload offsets;
 //   a3  payload words staged by cp.async.bulk into a double-buffered ring of
@@ -35,6 +42,9 @@
 //   a7  cvt.rn bf16x2 / f16x2, cvt.rn.satfinite e4m3x2, or rni + clamp for
 //       INT8, and one 16-byte (8-byte) store per lane, so a warp writes 512
 //       (256) contiguous bytes per round.
+// The integer arithmetic of a symbol step is split between the logic/shift
+// unit and integer multiply-adds (run-time multipliers, on the FMA pipe), and
+// each coordinate is formed as soon as its field is decoded.
 // Stream errors never fault or trap: every shared-memory index is masked or
 // bounded, every global read stays inside the buffers the header describes,
 // every wait is bounded, and inconsistencies raise bits in a device status word.
