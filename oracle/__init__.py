@@ -24,8 +24,9 @@ _SRC = os.path.join(_HERE, "ep_oracle.c")
 _SO = os.path.join(_HERE, "libep_oracle.so")
 
 # dtype codes of the oracle's decoder
-BF16, FP16, E4M3, INT8, FP32, LATTICE = 0, 1, 2, 3, 4, 5
-_NP_OUT = {BF16: np.uint16, FP16: np.uint16, E4M3: np.uint8, INT8: np.int8, FP32: np.float32, LATTICE: np.int32}
+BF16, FP16, E4M3, INT8, FP32, LATTICE, UINT8 = 0, 1, 2, 3, 4, 5, 6
+_NP_OUT = {BF16: np.uint16, FP16: np.uint16, E4M3: np.uint8, INT8: np.int8, FP32: np.float32, LATTICE: np.int32,
+           UINT8: np.uint8}
 
 
 def build(force: bool = False) -> str:

@@ -30,7 +30,8 @@
  *   pinned    quantize_e8 (brute force, covering radius, Q(y)=y), fields
  *             (exhaustive bijection), rANS coder (round trip, terminal states,
  *             cursor, code length near the entropy), tile layout (Table 5),
- *             dtype conversions (library conversions), splitmix64 (published
+ *             dtype conversions (library conversions; the INT8 and UINT8
+ *             readings on their own edge cases and numpy), splitmix64 (published
  *             outputs), refit (least-squares optimality), normalise_freqs (sum,
  *             support and rounding invariants), scale search (rate lands near
  *             target, bracket property), stored bytes (closed form).
@@ -883,13 +884,25 @@ int8_t epo_f32_to_int8(float x) {
     return (int8_t)r;
 }
 
+/* UINT8 container with its offset ([paper] App. B, Table 6: integer inputs are
+ * scaled per tensor before casting, "with an offset for unsigned values"; the
+ * errors are taken "with the UINT8 offset removed").  Reading: the codec codes
+ * the container's codes minus 128, and the decoder adds the 128 back: the
+ * nearest integer (ties to even), clamped to [-128, 127], plus 128. */
+uint8_t epo_f32_to_uint8(float x) {
+    double r = nearbyint((double)x);
+    if (r > 127.0) r = 127.0;
+    if (r < -128.0) r = -128.0;
+    return (uint8_t)(r + 128.0);
+}
+
 /* dtype codes shared with the Python wrapper of the oracle */
-enum { EPO_BF16 = 0, EPO_FP16 = 1, EPO_E4M3 = 2, EPO_INT8 = 3, EPO_FP32 = 4, EPO_LATTICE = 5 };
+enum { EPO_BF16 = 0, EPO_FP16 = 1, EPO_E4M3 = 2, EPO_INT8 = 3, EPO_FP32 = 4, EPO_LATTICE = 5, EPO_UINT8 = 6 };
 
 static int dtype_size(int dt) {
     switch (dt) {
         case EPO_BF16: case EPO_FP16: return 2;
-        case EPO_E4M3: case EPO_INT8: return 1;
+        case EPO_E4M3: case EPO_INT8: case EPO_UINT8: return 1;
         case EPO_FP32: case EPO_LATTICE: return 4;
         default: return 0;
     }
@@ -902,6 +915,7 @@ void epo_convert(const float* in, int64_t n, int dtype, void* out) {
             case EPO_FP16: ((uint16_t*)out)[i] = epo_f32_to_fp16(in[i]); break;
             case EPO_E4M3: ((uint8_t*)out)[i] = epo_f32_to_e4m3(in[i]); break;
             case EPO_INT8: ((int8_t*)out)[i] = epo_f32_to_int8(in[i]); break;
+            case EPO_UINT8: ((uint8_t*)out)[i] = epo_f32_to_uint8(in[i]); break;
             case EPO_FP32: ((float*)out)[i] = in[i]; break;
             default: break;
         }

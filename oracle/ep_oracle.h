@@ -53,6 +53,7 @@ uint16_t epo_f32_to_bf16(float x);
 uint16_t epo_f32_to_fp16(float x);
 uint8_t epo_f32_to_e4m3(float x);
 int8_t epo_f32_to_int8(float x);
+uint8_t epo_f32_to_uint8(float x);
 void epo_convert(const float* in, int64_t n, int dtype, void* out);
 
 int epo_decode_fields(const uint16_t* payload, const uint32_t* tile_index, const uint8_t* freq_tables,

@@ -1,6 +1,6 @@
 """Pins of the oracle's output conversions against the library conversions of
-PyTorch's CPU backend (round to nearest even), plus the saturating FP8 and
-symmetric INT8 readings checked on their own edge cases."""
+PyTorch's CPU backend (round to nearest even), plus the saturating FP8, the
+symmetric INT8 and the offset UINT8 readings checked on their own edge cases."""
 import numpy as np
 import torch
 
@@ -53,3 +53,19 @@ def test_int8_round_half_even_and_clamp():
     y = _samples()
     ref = np.clip(np.rint(y.astype(np.float64)), -127, 127).astype(np.int8)
     np.testing.assert_array_equal(oracle.convert(y, oracle.INT8), ref)
+
+
+def test_uint8_offset_round_half_even_and_clamp():
+    # [paper] App. B, Table 6: unsigned integer containers carry an offset; the decoder
+    # adds it back: nearest integer (ties to even), clamped to [-128, 127], plus 128
+    x = np.array([0.5, 1.5, -0.5, -1.5, 126.5, 127.5, 300, -127.5, -128.0, -128.5, -129.0, -1e9, 0.0, -0.0],
+                 np.float32)
+    got = oracle.convert(x, oracle.UINT8)
+    assert list(got) == [128, 130, 128, 126, 254, 255, 255, 0, 0, 0, 0, 0, 128, 128]
+    y = _samples()
+    ref = (np.clip(np.rint(y.astype(np.float64)), -128, 127) + 128).astype(np.uint8)
+    np.testing.assert_array_equal(oracle.convert(y, oracle.UINT8), ref)
+    # the offset removed, UINT8 and INT8 agree wherever INT8 does not clamp
+    z = y[(y > -127.5) & (y < 127.5)]
+    np.testing.assert_array_equal(oracle.convert(z, oracle.UINT8).astype(np.int16) - 128,
+                                  oracle.convert(z, oracle.INT8).astype(np.int16))
