@@ -428,8 +428,8 @@ def run_sweep(args):
 
     build.build()
     peak, peak_kind = _peaks()
-    out_bytes = {ep.BF16: 2, ep.FP16: 2, ep.FP8_E4M3: 1, ep.INT8: 1, ep.FP32: 4}
-    names = {ep.BF16: "bf16", ep.FP16: "fp16", ep.FP8_E4M3: "e4m3", ep.INT8: "int8", ep.FP32: "fp32"}
+    out_bytes = {ep.BF16: 2, ep.FP16: 2, ep.FP8_E4M3: 1, ep.INT8: 1, ep.FP32: 4, ep.UINT8: 1}
+    names = {ep.BF16: "bf16", ep.FP16: "fp16", ep.FP8_E4M3: "e4m3", ep.INT8: "int8", ep.FP32: "fp32", ep.UINT8: "uint8"}
     rows_out = []
 
     def case(label, blob, dtype, extra=None):
@@ -459,9 +459,10 @@ def run_sweep(args):
     for dt in (ep.BF16, ep.FP16):
         case("DiT attention projection, 5 bpp", blob, dt)
     src = synth.generate(synth.lowp_source())
-    for kind, dt in (("e4m3", ep.FP8_E4M3), ("int8", ep.INT8)):
-        vals, _ = synth.to_e4m3_container(src) if kind == "e4m3" else synth.to_int8_container(src)
-        case(f"{kind} container, 5 bpp", ep.encode_tensor(vals, 5.0, has_container_scales=True), dt)
+    for kind, dt in (("e4m3", ep.FP8_E4M3), ("int8", ep.INT8), ("uint8", ep.UINT8)):
+        conv = {"e4m3": synth.to_e4m3_container, "int8": synth.to_int8_container, "uint8": synth.to_uint8_container}
+        vals, _ = conv[kind](src)
+        case(f"{kind} container, 5 bpp", ep.encode_tensor(vals, 5.0, has_container_scales=kind != "uint8"), dt)
     del src
     for wide in (True, False):
         W = synth.generate(synth.llm_prefill(wide))

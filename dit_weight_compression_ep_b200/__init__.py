@@ -6,5 +6,5 @@ This package is a thin ctypes binding over it; nothing here computes the codec.
 Importing the package does not load the library; the first call does, and it
 raises if the library has not been built.
 """
-from ._lib import (BF16, FP16, FP8_E4M3, INT8, FP32, LATTICE_I32, Blob, DeviceBlob, EntroPackError,  # noqa: F401
+from ._lib import (BF16, FP16, FP8_E4M3, INT8, FP32, LATTICE_I32, UINT8, Blob, DeviceBlob, EntroPackError,  # noqa: F401
                    check_status, decode_status, decode_tensor, encode_tensor, lib)

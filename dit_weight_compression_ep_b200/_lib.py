@@ -17,10 +17,10 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 SO_PATH = os.path.join(_HERE, "libentropack.so")
 
 # ep_dtype
-BF16, FP16, FP8_E4M3, INT8, FP32, LATTICE_I32 = 0, 1, 2, 3, 4, 5
+BF16, FP16, FP8_E4M3, INT8, FP32, LATTICE_I32, UINT8 = 0, 1, 2, 3, 4, 5, 6
 DTYPE_NAMES = {"bf16": BF16, "fp16": FP16, "e4m3": FP8_E4M3, "fp8_e4m3": FP8_E4M3, "int8": INT8, "fp32": FP32,
-               "lattice": LATTICE_I32}
-OUT_BYTES = {BF16: 2, FP16: 2, FP8_E4M3: 1, INT8: 1, FP32: 4, LATTICE_I32: 4}
+               "lattice": LATTICE_I32, "uint8": UINT8}
+OUT_BYTES = {BF16: 2, FP16: 2, FP8_E4M3: 1, INT8: 1, FP32: 4, LATTICE_I32: 4, UINT8: 1}
 
 # ep_status
 STATUS = {0: "EP_OK", 1: "EP_EINVAL", 2: "EP_EUNSUPPORTED", 3: "EP_EALPHABET", 4: "EP_ECUDA", 5: "EP_ECORRUPT",
@@ -183,7 +183,7 @@ def _torch_dtype(dt: int):
     import torch
 
     return {BF16: torch.bfloat16, FP16: torch.float16, FP8_E4M3: torch.float8_e4m3fn, INT8: torch.int8,
-            FP32: torch.float32, LATTICE_I32: torch.int32}[dt]
+            FP32: torch.float32, LATTICE_I32: torch.int32, UINT8: torch.uint8}[dt]
 
 
 def decode_tensor(db: DeviceBlob, out_dtype: int = BF16, out=None, stream=None):

@@ -40,7 +40,7 @@
 //       bits of 1.5*2^22 + (2z + c)/2) and multiplied once by sigma, so every
 //       weight gets a single rounding, whatever sigma;
 //   a7  cvt.rn bf16x2 / f16x2, cvt.rn.satfinite e4m3x2, or rni + clamp for
-//       INT8, and one 16-byte (8-byte) store per lane, so a warp writes 512
+//       INT8 (and + 128 for UINT8), and one 16-byte (8-byte) store per lane, so a warp writes 512
 //       (256) contiguous bytes per round.
 // The integer arithmetic of a symbol step is split between the logic/shift
 // unit and integer multiply-adds (run-time multipliers, on the FMA pipe), and
@@ -449,6 +449,18 @@ struct Out<EP_INT8> {
         int q[8];
 #pragma unroll
         for (int i = 0; i < 8; ++i) q[i] = __float2int_rn(fminf(fmaxf(w[i], -127.0f), 127.0f));
+        uint2 v;
+        v.x = __byte_perm(__byte_perm(q[0], q[1], 0x0040), __byte_perm(q[2], q[3], 0x0040), 0x5410);
+        v.y = __byte_perm(__byte_perm(q[4], q[5], 0x0040), __byte_perm(q[6], q[7], 0x0040), 0x5410);
+        reinterpret_cast<uint2*>(out)[g] = v;
+    }
+};
+template <>
+struct Out<EP_UINT8> {
+    __device__ static void store(void* out, int64_t g, const float w[8]) {
+        int q[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) q[i] = __float2int_rn(fminf(fmaxf(w[i], -128.0f), 127.0f)) + 128;
         uint2 v;
         v.x = __byte_perm(__byte_perm(q[0], q[1], 0x0040), __byte_perm(q[2], q[3], 0x0040), 0x5410);
         v.y = __byte_perm(__byte_perm(q[4], q[5], 0x0040), __byte_perm(q[6], q[7], 0x0040), 0x5410);
@@ -1093,6 +1105,7 @@ cudaError_t dev_setup(int dev, int dt, DevState*& ds) {
             case EP_FP16: e = set_decode_attr<EP_FP16>(); break;
             case EP_FP8_E4M3: e = set_decode_attr<EP_FP8_E4M3>(); break;
             case EP_INT8: e = set_decode_attr<EP_INT8>(); break;
+            case EP_UINT8: e = set_decode_attr<EP_UINT8>(); break;
             case EP_FP32: e = set_decode_attr<EP_FP32>(); break;
             default: e = set_decode_attr<EP_LATTICE_I32>(); break;
         }
@@ -1129,7 +1142,7 @@ ep_status ep_decode_tensor(void* stream, const uint16_t* tiles, const uint32_t* 
     if (!tiles || !tile_index || !freq_tables || !row_scales || !out) return EP_EINVAL;
     if (rows <= 0 || cols <= 0) return EP_EINVAL;
     if (cols % 8) return EP_EUNSUPPORTED;
-    if ((int)out_dtype < EP_BF16 || (int)out_dtype > EP_LATTICE_I32) return EP_EUNSUPPORTED;
+    if ((int)out_dtype < EP_BF16 || (int)out_dtype > EP_UINT8) return EP_EUNSUPPORTED;
     const int64_t nvec = rows * (cols / 8);
     if (nvec >= (1ll << 31) || rows >= (1ll << 31)) return EP_EINVAL;
     auto misaligned = [](const void* q, uintptr_t a) { return (reinterpret_cast<uintptr_t>(q) & (a - 1)) != 0; };
@@ -1155,6 +1168,7 @@ ep_status ep_decode_tensor(void* stream, const uint16_t* tiles, const uint32_t* 
             case EP_FP16: e = launch_decode<EP_FP16>(prm, st, ds->num_sms); break;
             case EP_FP8_E4M3: e = launch_decode<EP_FP8_E4M3>(prm, st, ds->num_sms); break;
             case EP_INT8: e = launch_decode<EP_INT8>(prm, st, ds->num_sms); break;
+            case EP_UINT8: e = launch_decode<EP_UINT8>(prm, st, ds->num_sms); break;
             case EP_FP32: e = launch_decode<EP_FP32>(prm, st, ds->num_sms); break;
             default: e = launch_decode<EP_LATTICE_I32>(prm, st, ds->num_sms); break;
         }
@@ -1250,6 +1264,7 @@ cudaError_t noalloc_setup(int dev, int dt, NoAllocState*& ns) {
             case EP_FP16: e = set_decode_attr<EP_FP16>(); break;
             case EP_FP8_E4M3: e = set_decode_attr<EP_FP8_E4M3>(); break;
             case EP_INT8: e = set_decode_attr<EP_INT8>(); break;
+            case EP_UINT8: e = set_decode_attr<EP_UINT8>(); break;
             case EP_FP32: e = set_decode_attr<EP_FP32>(); break;
             default: e = set_decode_attr<EP_LATTICE_I32>(); break;
         }
@@ -1269,7 +1284,7 @@ extern "C" ep_status ep_decode_tensor_noalloc(void* stream, const uint16_t* tile
     if (!tiles || !tile_index || !freq_tables || !row_scales || !out) return EP_EINVAL;
     if (rows <= 0 || cols <= 0) return EP_EINVAL;
     if (cols % 8) return EP_EUNSUPPORTED;
-    if ((int)out_dtype < EP_BF16 || (int)out_dtype > EP_LATTICE_I32) return EP_EUNSUPPORTED;
+    if ((int)out_dtype < EP_BF16 || (int)out_dtype > EP_UINT8) return EP_EUNSUPPORTED;
     // the largest tensor this entry point takes: fewer than 2^31 vectors of eight
     const int64_t nvec = rows * (cols / 8);
     if (nvec >= (1ll << 31) || rows >= (1ll << 31)) return EP_EINVAL;
@@ -1291,6 +1306,7 @@ extern "C" ep_status ep_decode_tensor_noalloc(void* stream, const uint16_t* tile
             case EP_FP16: e = launch_decode<EP_FP16>(prm, st, ns->num_sms); break;
             case EP_FP8_E4M3: e = launch_decode<EP_FP8_E4M3>(prm, st, ns->num_sms); break;
             case EP_INT8: e = launch_decode<EP_INT8>(prm, st, ns->num_sms); break;
+            case EP_UINT8: e = launch_decode<EP_UINT8>(prm, st, ns->num_sms); break;
             case EP_FP32: e = launch_decode<EP_FP32>(prm, st, ns->num_sms); break;
             default: e = launch_decode<EP_LATTICE_I32>(prm, st, ns->num_sms); break;
         }

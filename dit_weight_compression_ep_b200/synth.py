@@ -84,6 +84,16 @@ def to_e4m3_container(a: np.ndarray):
     return q.to(torch.float32).numpy(), scale
 
 
+def to_uint8_container(a: np.ndarray):
+    """Per-tensor UINT8 container with offset 128: scale = amax/127, code = nearest + 128, clamped
+    to [0, 255].  Returns (the codes minus the offset as fp32 -- what the codec codes --, scale)."""
+    a = np.ascontiguousarray(a, np.float32)
+    amax = float(np.abs(a).max())
+    scale = np.float32(amax / 127.0) if amax > 0 else np.float32(1.0)
+    q = np.clip(np.rint(a / scale) + 128, 0, 255)
+    return (q - 128).astype(np.float32), scale
+
+
 def to_int8_container(a: np.ndarray):
     """Per-channel (row) symmetric INT8 container: scale = amax/127, nearest, clamp +-127."""
     a = np.ascontiguousarray(a, np.float32)

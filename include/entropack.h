@@ -47,7 +47,10 @@ typedef enum {
     EP_FP8_E4M3 = 2,    /* OCP FP8 E4M3 ("fn"), round to nearest even, saturating to +-448 */
     EP_INT8 = 3,        /* nearest-even integer, clamped to [-127, 127] */
     EP_FP32 = 4,        /* the FP32 product itself */
-    EP_LATTICE_I32 = 5  /* int32 2y (twice the lattice coordinates), for verification */
+    EP_LATTICE_I32 = 5, /* int32 2y (twice the lattice coordinates), for verification */
+    EP_UINT8 = 6        /* the UINT8 container with its offset: nearest-even integer, clamped to
+                           [-128, 127], plus 128 (App. B, Table 6: unsigned integer inputs carry an
+                           offset, which the codec removes before coding and adds back here) */
 } ep_dtype;
 
 typedef enum {

@@ -5,9 +5,9 @@ import oracle
 import dit_weight_compression_ep_b200 as ep
 
 ORACLE_DT = {ep.BF16: oracle.BF16, ep.FP16: oracle.FP16, ep.FP8_E4M3: oracle.E4M3, ep.INT8: oracle.INT8,
-             ep.FP32: oracle.FP32, ep.LATTICE_I32: oracle.LATTICE}
+             ep.FP32: oracle.FP32, ep.LATTICE_I32: oracle.LATTICE, ep.UINT8: oracle.UINT8}
 RAW = {ep.BF16: np.uint16, ep.FP16: np.uint16, ep.FP8_E4M3: np.uint8, ep.INT8: np.uint8, ep.FP32: np.uint32,
-       ep.LATTICE_I32: np.uint32}
+       ep.LATTICE_I32: np.uint32, ep.UINT8: np.uint8}
 
 
 def to_raw(t):
@@ -17,7 +17,7 @@ def to_raw(t):
     a = t.detach().cpu().contiguous()
     if a.dtype in (torch.bfloat16, torch.float16):
         return a.view(torch.int16).numpy().view(np.uint16)
-    if a.dtype in (torch.float8_e4m3fn, torch.int8):
+    if a.dtype in (torch.float8_e4m3fn, torch.int8, torch.uint8):
         return a.view(torch.uint8).numpy()
     return a.view(torch.int32).numpy().view(np.uint32)
 

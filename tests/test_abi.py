@@ -54,9 +54,10 @@ def test_decode_rejects_bad_arguments_on_host(lib):
     a = list(args)
     a[6] = 60                   # cols % 8 != 0
     assert lib.ep_decode_tensor(*a) == EUNSUP
-    a = list(args)
-    a[7] = 9                    # unknown dtype
-    assert lib.ep_decode_tensor(*a) == EUNSUP
+    for dt in (7, 9, -1):       # unknown dtypes (EP_UINT8 = 6 is the last one)
+        a = list(args)
+        a[7] = dt
+        assert lib.ep_decode_tensor(*a) == EUNSUP
     a = list(args)
     a[5] = 0                    # rows <= 0
     assert lib.ep_decode_tensor(*a) == EINVAL

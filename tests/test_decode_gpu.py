@@ -17,7 +17,7 @@ from gpu_util import as_lib_blob, assert_parity, oracle_decode, to_raw
 
 pytestmark = pytest.mark.gpu
 
-ALL_DT = [ep.BF16, ep.FP16, ep.FP8_E4M3, ep.INT8, ep.FP32, ep.LATTICE_I32]
+ALL_DT = [ep.BF16, ep.FP16, ep.FP8_E4M3, ep.INT8, ep.FP32, ep.LATTICE_I32, ep.UINT8]
 
 
 @pytest.fixture(scope="module", autouse=True)
@@ -62,7 +62,7 @@ def test_precisions_and_tile_sizes(b, V):
     W = (rng.standard_normal((96, 1024)) * 0.02 * np.exp(rng.normal(0, 0.4, (96, 1)))).astype(np.float32)
     ob = oracle.encode(W, 4.0 if b <= 11 else 7.5, prob_bits=b, tile_vectors=V)
     assert ob.b == b
-    _check(as_lib_blob(ob), [ep.BF16, ep.INT8, ep.LATTICE_I32], f"b={b} V={V}")
+    _check(as_lib_blob(ob), [ep.BF16, ep.INT8, ep.LATTICE_I32, ep.UINT8], f"b={b} V={V}")
 
 
 @pytest.mark.parametrize("rows,cols,V", [(1, 8, 32), (1, 256, 1), (3, 64, 32), (5, 24, 7), (17, 8, 50),
@@ -227,6 +227,21 @@ def test_fp8_and_int8_containers_5bpp():
         assert abs(blob.stored_bpp / 5.0 - 1) < 0.03
         dt = ep.FP8_E4M3 if kind == "e4m3" else ep.INT8
         _full_check(blob, [dt], kind)
+
+
+def test_uint8_container_5bpp():
+    """UINT8 container (per-tensor scale, offset 128): the codec codes the codes minus 128 and
+    the decoder adds it back; bit-exact against the oracle, and the round trip stays close."""
+    src = synth.generate(synth.lowp_source())
+    vals, _ = synth.to_uint8_container(src)
+    blob = ep.encode_tensor(vals, 5.0)
+    assert abs(blob.stored_bpp / 5.0 - 1) < 0.03
+    _full_check(blob, [ep.UINT8], "uint8")
+    import torch
+
+    out = ep.decode_tensor(ep.DeviceBlob(blob), ep.UINT8).cpu().numpy().astype(np.float64) - 128.0
+    rel = np.linalg.norm(out - vals) / np.linalg.norm(vals)
+    assert rel < 0.1, rel
 
 
 @pytest.mark.parametrize("wide", [True, False])
