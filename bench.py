@@ -2,6 +2,7 @@
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
     python bench.py --sweep      (every workload, one GPU: a table, not the bench line)
+    python bench.py --linear     (decode-then-GEMM against a resident weight, one GPU)
 
 One step = one ep_decode_tensor call: the whole hot path (tile setup, table
 staging, payload staging, rANS decode, lattice reconstruction, row rescale,
@@ -519,6 +520,89 @@ def run_sweep(args):
           f"= {100 * tot['decode_over_matmul']:.1f} %; oracle: {oc}; HBM peak {peak} GB/s ({peak_kind})")
 
 
+def run_linear(args):
+    """A linear layer whose weight is stored compressed: decode it with the library, then the
+    library GEMM (cuBLAS through torch), against the same GEMM with the weight resident
+    (BF16 X @ W^T; FP8-e4m3 `_scaled_mm` with per-row weight scales; INT8 `_int_mm`).  The
+    3840x10240 layer at 4 bpp, tokens 256 .. 16384; each time is the minimum of 15 runs, each
+    after a 256 MiB L2 flush.  Prints a markdown table and JSON lines."""
+    import torch
+
+    import dit_weight_compression_ep_b200 as ep
+    from dit_weight_compression_ep_b200 import build, synth
+
+    build.build()
+    dev = torch.device("cuda")
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+
+    def tmin(fn, runs=15):
+        for _ in range(3):
+            fn()
+        ts = []
+        for _ in range(runs):
+            flush.zero_()
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record()
+            fn()
+            b.record()
+            torch.cuda.synchronize()
+            ts.append(a.elapsed_time(b))
+        return min(ts) * 1e3
+
+    W = synth.generate(synth.headline())
+    rows, cols = W.shape
+    routes = []
+    # BF16
+    blob = ep.encode_tensor(W, TARGET)
+    db = ep.DeviceBlob(blob)
+    Wb = torch.from_numpy(W).to(dev).to(torch.bfloat16)
+    Wd = torch.empty_like(Wb)
+    routes.append(("bf16", db, ep.BF16, Wb, Wd))
+    # FP8-e4m3 container, per-row scales
+    vals, wsc = synth.to_e4m3_container(W)
+    blob8 = ep.encode_tensor(vals, TARGET, has_container_scales=True)
+    W8 = torch.from_numpy(vals).to(dev).to(torch.float8_e4m3fn)
+    routes.append(("fp8 e4m3", ep.DeviceBlob(blob8), ep.FP8_E4M3, W8, torch.empty_like(W8)))
+    wscale = torch.from_numpy(wsc).to(dev).view(1, -1)
+    # INT8 container, per-row scales
+    vali, _ = synth.to_int8_container(W)
+    blobi = ep.encode_tensor(vali, TARGET, has_container_scales=True)
+    Wi = torch.from_numpy(vali).to(dev).to(torch.int8)
+    routes.append(("int8", ep.DeviceBlob(blobi), ep.INT8, Wi, torch.empty_like(Wi)))
+    out = []
+    for tokens in (256, 1024, 4096, 16384):
+        X = (torch.randn(tokens, cols, device=dev) * 0.5)
+        Xb = X.to(torch.bfloat16)
+        X8 = X.clamp(-448, 448).to(torch.float8_e4m3fn)
+        Xi = X.mul(20).round().clamp(-127, 127).to(torch.int8)
+        xs = torch.ones(tokens, 1, device=dev)
+        for name, dbr, dt, Wres, Wdec in routes:
+            if name == "bf16":
+                gemm = lambda Wm: torch.matmul(Xb, Wm.t())
+            elif name == "fp8 e4m3":
+                gemm = lambda Wm: torch._scaled_mm(X8, Wm.t(), scale_a=xs, scale_b=wscale, out_dtype=torch.bfloat16)
+            else:
+                gemm = lambda Wm: torch._int_mm(Xi, Wm.t())
+            try:
+                t_res = tmin(lambda: gemm(Wres))
+            except Exception as exc:  # a route torch's GEMMs do not offer on this device
+                print(json.dumps({"route": name, "tokens": tokens, "unavailable": str(exc)[:160]}), flush=True)
+                continue
+            t_dec = tmin(lambda: ep.decode_tensor(dbr, dt, out=Wdec))
+            t_both = tmin(lambda: (ep.decode_tensor(dbr, dt, out=Wdec), gemm(Wdec)))
+            r = {"route": name, "tokens": tokens, "gemm_resident_us": round(t_res, 2), "decode_us": round(t_dec, 2),
+                 "decode_then_gemm_us": round(t_both, 2), "overhead": round(t_both / t_res - 1.0, 4)}
+            out.append(r)
+            print(json.dumps(r), flush=True)
+        if ep.decode_status() != 0:
+            raise RuntimeError("decode reported a corrupt stream")
+    print("\n| route | tokens | GEMM, weight resident (µs) | decode (µs) | decode then GEMM (µs) | overhead |")
+    print("|---|---|---|---|---|---|")
+    for r in out:
+        print(f"| {r['route']} | {r['tokens']} | {r['gemm_resident_us']} | {r['decode_us']} | {r['decode_then_gemm_us']} | "
+              f"{100 * r['overhead']:.1f} % |")
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -527,6 +611,7 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--sweep", action="store_true", help="every workload's decode throughput (one GPU)")
+    ap.add_argument("--linear", action="store_true", help="decode-then-GEMM against a resident weight (one GPU)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
@@ -536,6 +621,9 @@ def main():
 
     if args.sweep:
         run_sweep(args)
+        return
+    if args.linear:
+        run_linear(args)
         return
     if args.impl == "reference":
         if rank != 0:
