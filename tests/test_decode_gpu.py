@@ -200,6 +200,40 @@ def _full_check(blob, dts, what, sample_tiles=None):
         del out
 
 
+def _slot_pairs_past_15(blob):
+    """Host-side look at the stored tables: (b, slot pairs whose odd slot's symbol lies 15 or
+    more symbols past the even slot's, records the two-level LUT would need)."""
+    ft = blob.freq_tables
+    b = int(ft[:48].view(np.uint32)[2])
+    d = ft[48:48 + 17 * 8].view(np.int32).reshape(17, 2)
+    fq = ft[192:].view(np.uint16).astype(np.int64)
+    A = d[:, 1].astype(np.int64)
+    off = np.concatenate([[0], np.cumsum(A)[:-1]])
+    far, nrec = 0, 1
+    for t in range(1, 17):
+        cum = np.concatenate([[0], np.cumsum(fq[off[t]:off[t] + A[t]])])
+        nrec += int(A[t]) + 1
+        own = np.searchsorted(cum[:A[t]], np.arange(1 << b), side="right") - 1
+        far += int(np.sum(own[1::2] - own[0::2] >= 15))
+    return b, far, nrec
+
+
+@pytest.mark.parametrize("lo,hi,p,two", [(12.0, 40.0, 0.01, True), (20.0, 60.0, 0.02, False)])
+def test_sparse_outlier_alphabets_at_8bpp(lo, hi, p, two):
+    """b = 12 with sparse, widely spaced outliers: many slot pairs whose odd slot's symbol is 15
+    or more symbols on (the two-level LUT's bounded walk), and, with larger alphabets, the
+    bucketed LUT.  Bit-exact against the oracle."""
+    rng = np.random.default_rng(5)
+    W = rng.standard_normal((512, 1024)).astype(np.float32)
+    mask = rng.random(W.shape) < p
+    W[mask] = (rng.choice([-1, 1], mask.sum()) * rng.uniform(lo, hi, mask.sum())).astype(np.float32)
+    blob = ep.encode_tensor(W, 8.0)
+    b, far, nrec = _slot_pairs_past_15(blob)
+    assert b == 12 and far > 50
+    assert (nrec <= 32768) == two  # the header rule that picks the two-level LUT
+    _full_check(blob, [ep.BF16, ep.LATTICE_I32], f"sparse outliers {lo}-{hi}")
+
+
 def test_headline_3840x10240_bf16_4bpp():
     W = synth.generate(synth.headline())
     blob = ep.encode_tensor(W, 4.0)
