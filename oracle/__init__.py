@@ -54,6 +54,8 @@ class _Opts(C.Structure):
         ("has_container_scales", C.c_int),
         ("direct_z8", C.c_int),
         ("pooled", C.c_int),
+        ("rdo_candidates", C.c_int),
+        ("rdo_sweeps", C.c_int),
     ]
 
 
@@ -87,6 +89,7 @@ def lib() -> C.CDLL:
         L.epo_refit_row.argtypes = [P, P, I64]
         L.epo_refit_row.restype = C.c_float
         L.epo_encode.argtypes = [P, I64, I64, C.POINTER(_Opts), C.POINTER(P)]
+        L.epo_rdo_ratios.argtypes = [C.c_int, P]
         L.epo_encode.restype = C.c_int
         L.epo_encode_fields.argtypes = [P, I64, I64, P, C.c_int, C.c_int, C.c_int, C.POINTER(P)]
         L.epo_encode_fields.restype = C.c_int
@@ -151,12 +154,14 @@ def _blob_from_handle(h: int) -> Blob:
 
 def encode(W: np.ndarray, target_bpp: float, *, prob_bits: int = 0, tile_vectors: int = 0,
            sample_vectors: int = 0, search_steps: int = 0, seed: int = 0,
-           has_container_scales: bool = False, direct_z8: bool = False, pooled: bool = False) -> Blob:
-    """Full encoder (§3.1): normalise, search s, quantise, refit, tables, tiled rANS."""
+           has_container_scales: bool = False, direct_z8: bool = False, pooled: bool = False,
+           rdo_candidates: int = 0, rdo_sweeps: int = 0) -> Blob:
+    """Full encoder (§3.1): normalise, search s, quantise, refit, optional per-row RDO (§3.5,
+    App. C.2), tables, tiled rANS."""
     W = np.ascontiguousarray(W, dtype=np.float32)
     rows, cols = W.shape
     o = _Opts(target_bpp, prob_bits, tile_vectors, sample_vectors, search_steps, seed,
-              int(has_container_scales), int(direct_z8), int(pooled))
+              int(has_container_scales), int(direct_z8), int(pooled), int(rdo_candidates), int(rdo_sweeps))
     h = C.c_void_p()
     rc = lib().epo_encode(_p(W), rows, cols, C.byref(o), C.byref(h))
     if rc:
@@ -265,6 +270,13 @@ def fields_of(y: np.ndarray, c: np.ndarray, direct_z8: bool = False) -> np.ndarr
     f = np.zeros((y.shape[0], 9), np.int32)
     lib().epo_fields_batch(_p(y), _p(c), y.shape[0], int(direct_z8), _p(f))
     return f
+
+
+def rdo_ratios(K: int) -> np.ndarray:
+    """The K nested candidate ratios of the per-row refinement (App. C.2)."""
+    out = np.zeros(K, np.float64)
+    lib().epo_rdo_ratios(int(K), _p(out))
+    return out
 
 
 def points_of(fields: np.ndarray, direct_z8: bool = False) -> np.ndarray:

@@ -660,6 +660,155 @@ float epo_refit_row(const float* w, const double* y, int64_t cols) {
     return (float)(num / den);
 }
 
+/*
+ * A10 Per-row rate-distortion refinement ([paper] §3.5 "RDO compares several
+ * quantization resolutions per row and allocates them under a common storage
+ * budget"; App. C.2; Figs. 3-4).  Off unless asked for ([paper] §4.1: "RDO is
+ * disabled except in its dedicated ablations").
+ *
+ * Candidate ratios (§3.5): K ratios in [0.70, 1.45], starting from 1; each
+ * further ratio bisects, in log scale, the widest interval between neighbouring
+ * ratios and the ends of the range.  READING: the ends are not candidates
+ * themselves; ties between equally wide intervals go to the lower interval.
+ */
+void epo_rdo_ratios(int K, double* rho) {
+    double pts[2 + 64];
+    int n = 3;
+    pts[0] = 0.70;
+    pts[1] = 1.0;
+    pts[2] = 1.45;
+    rho[0] = 1.0;
+    for (int k = 1; k < K && k < 64; ++k) {
+        int best = 0;
+        double wbest = -1.0;
+        for (int i = 0; i + 1 < n; ++i) {
+            double w = log(pts[i + 1] / pts[i]);
+            if (w > wbest) {
+                wbest = w;
+                best = i;
+            }
+        }
+        double mid = sqrt(pts[best] * pts[best + 1]);
+        for (int i = n; i > best + 1; --i) pts[i] = pts[i - 1];
+        pts[best + 1] = mid;
+        ++n;
+        rho[k] = mid;
+    }
+}
+
+/* Ideal code length of one row's fields under the tables: sum over its symbols, in
+ * order, of b - log2 f, with f = 1 for a symbol the table gives no frequency
+ * (READING: an unseen symbol costs the minimum frequency, b bits). */
+static double row_bits(const int32_t* f, int64_t nq, const table_t* tabs, int b, int pooled) {
+    double bits = 0.0;
+    for (int64_t q = 0; q < nq; ++q) {
+        const int32_t* v = f + NFIELDS * q;
+        for (int k = 0; k < NFIELDS; ++k) {
+            const table_t* tb = &tabs[table_of(k, v[0], pooled)];
+            int64_t i = (int64_t)v[k] - tb->min;
+            uint32_t fr = (tb->A && i >= 0 && i < (int64_t)tb->A) ? tb->freq[i] : 0u;
+            bits += (double)b - log2((double)(fr ? fr : 1u));
+        }
+    }
+    return bits;
+}
+
+/*
+ * App. C.2 allocation.  READINGS: candidate k of row r quantises the row at
+ * rho_k s (the row normaliser unchanged) and refits its scale (A9); its
+ * distortion is sum_j (w_j - sigma y_j)^2 in weight units (sigma as stored, FP32).
+ * A candidate is admissible when every symbol lies in the baseline tables'
+ * alphabets (so the stored alphabets keep fitting 2^b).  Budget: the baseline's
+ * ideal code length under its own tables.  A sweep prices every admissible
+ * candidate under the current tables, finds the smallest common rate penalty
+ * lambda (64 bisection steps of log2 lambda on [-80, 80]) whose per-row choices
+ * argmin D + lambda R (ties: lowest k) fit the budget, and rebuilds the tables
+ * from the chosen fields.  In: fields at ratio 1; out: chosen fields and scales.
+ */
+static void rdo_refine(const shape_t* sh, const float* W, const double* norms, double s, int b, int K, int sweeps,
+                       int32_t* fields, float* scales) {
+    const int64_t rows = sh->rows, cols = sh->cols, nq = cols / 8, rowf = NFIELDS * nq;
+    double rho[64];
+    if (K > 64) K = 64;
+    epo_rdo_ratios(K, rho);
+    int32_t* cf = (int32_t*)malloc(sizeof(int32_t) * (size_t)(K * rows * rowf));
+    float* cs = (float*)malloc(sizeof(float) * (size_t)(K * rows));
+    double* cd = (double*)malloc(sizeof(double) * (size_t)(K * rows));
+    double* cr = (double*)malloc(sizeof(double) * (size_t)(K * rows));
+    unsigned char* ok = (unsigned char*)malloc((size_t)(K * rows));
+    int* sel = (int*)malloc(sizeof(int) * (size_t)rows);
+    double* y = (double*)malloc(sizeof(double) * (size_t)cols);
+    table_t base[MAX_TABLES], tabs[MAX_TABLES];
+    count_tables(fields, sh->nvec, sh->pooled, sh->ntab, UINT64_MAX, base);
+    build_freqs(base, sh->ntab, b);
+    for (int k = 0; k < K; ++k)
+        for (int64_t r = 0; r < rows; ++r) {
+            const float* w = W + r * cols;
+            int32_t* f = cf + (k * rows + r) * rowf;
+            quantize_row(w, cols, norms[r], rho[k] * s, sh->direct_z8, f, y);
+            float sg = epo_refit_row(w, y, cols);
+            double d = 0.0;
+            for (int64_t j = 0; j < cols; ++j) {
+                double e = (double)w[j] - (double)sg * y[j];
+                d += e * e;
+            }
+            cs[k * rows + r] = sg;
+            cd[k * rows + r] = d;
+            unsigned char in = 1;
+            for (int64_t q = 0; q < nq && in; ++q)
+                for (int m = 0; m < NFIELDS; ++m) {
+                    const table_t* tb = &base[table_of(m, f[NFIELDS * q], sh->pooled)];
+                    int64_t i = (int64_t)f[NFIELDS * q + m] - tb->min;
+                    if (!tb->A || i < 0 || i >= (int64_t)tb->A) in = 0;
+                }
+            ok[k * rows + r] = in;
+        }
+    double budget = 0.0;
+    for (int64_t r = 0; r < rows; ++r) budget += row_bits(cf + r * rowf, nq, base, b, sh->pooled);
+    for (int64_t r = 0; r < rows; ++r) sel[r] = 0;
+    const table_t* model = base;
+    for (int sw = 0; sw < sweeps; ++sw) {
+        for (int k = 0; k < K; ++k)
+            for (int64_t r = 0; r < rows; ++r)
+                cr[k * rows + r] = ok[k * rows + r] ? row_bits(cf + (k * rows + r) * rowf, nq, model, b, sh->pooled)
+                                                    : INFINITY;
+        double lo = -80.0, hi = 80.0;
+        for (int it = 0; it <= 64; ++it) {
+            double t = it < 64 ? 0.5 * (lo + hi) : hi; /* the last pass applies the final lambda */
+            double lam = exp2(t), total = 0.0;
+            for (int64_t r = 0; r < rows; ++r) {
+                int best = 0;
+                double jbest = cd[r] + lam * cr[r];
+                for (int k = 1; k < K; ++k) {
+                    double j = cd[k * rows + r] + lam * cr[k * rows + r];
+                    if (j < jbest) {
+                        jbest = j;
+                        best = k;
+                    }
+                }
+                sel[r] = best;
+                total += cr[best * rows + r];
+            }
+            if (it < 64) {
+                if (total <= budget) hi = t;
+                else lo = t;
+            }
+        }
+        for (int64_t r = 0; r < rows; ++r)
+            memcpy(fields + r * rowf, cf + (sel[r] * rows + r) * rowf, sizeof(int32_t) * (size_t)rowf);
+        if (model != base)
+            for (int t = 0; t < sh->ntab; ++t) table_free(&tabs[t]);
+        count_tables(fields, sh->nvec, sh->pooled, sh->ntab, UINT64_MAX, tabs);
+        build_freqs(tabs, sh->ntab, b);
+        model = tabs;
+    }
+    for (int64_t r = 0; r < rows; ++r) scales[r] = cs[sel[r] * rows + r];
+    for (int t = 0; t < sh->ntab; ++t) table_free(&base[t]);
+    if (model != base)
+        for (int t = 0; t < sh->ntab; ++t) table_free(&tabs[t]);
+    free(cf); free(cs); free(cd); free(cr); free(ok); free(sel); free(y);
+}
+
 int epo_encode(const float* W, int64_t rows, int64_t cols, const epo_opts* opts, epo_blob** out) {
     *out = NULL;
     if (rows <= 0 || cols <= 0 || cols % 8) return -1;
@@ -739,6 +888,9 @@ int epo_encode(const float* W, int64_t rows, int64_t cols, const epo_opts* opts,
     bl->s = s;
     bl->row_scales = (float*)malloc(sizeof(float) * (size_t)rows);
     for (int64_t r = 0; r < rows; ++r) bl->row_scales[r] = epo_refit_row(W + r * cols, ys + r * cols, cols);
+    if (opts->rdo_candidates > 1)
+        rdo_refine(&sh, W, norms, s, b, opts->rdo_candidates, opts->rdo_sweeps > 0 ? opts->rdo_sweeps : 1,
+                   bl->fields, bl->row_scales);
     int rc = code_fields(bl, sh.pooled);
     free(norms);
     free(srows);

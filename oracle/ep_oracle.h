@@ -22,9 +22,12 @@ typedef struct {
     int has_container_scales;
     int direct_z8;          /* App. A.3 ablation: store z8 instead of m */
     int pooled;             /* App. A.3 ablation: 9 tables, no coset conditioning */
+    int rdo_candidates;     /* App. C.2 per-row refinement: K candidate scales (0 or 1: off) */
+    int rdo_sweeps;         /* allocation sweeps (0: 1) */
 } epo_opts;
 
 void epo_splitmix64(uint64_t seed, int64_t n, uint64_t* out);
+void epo_rdo_ratios(int K, double* rho);
 uint64_t epo_shape_seed(int64_t rows, int64_t cols);
 int64_t epo_sample_rows(int64_t rows, int64_t cols, int64_t sample_vectors, uint64_t seed, int64_t* out_rows);
 double epo_row_norm(const float* w, int64_t cols);

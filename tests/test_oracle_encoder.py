@@ -167,3 +167,67 @@ def test_coarsening_at_maximum_precision():
     assert amax <= 1 << 15
     np.testing.assert_array_equal(
         oracle.decode_fields(a.payload, a.tile_index, a.freq_tables, a.rows, a.cols), a.fields)
+
+
+# ------------------------------------------------------------------ per-row RDO (§3.5, App. C.2)
+
+def _heterogeneous_rows(seed=1, rows=256, cols=512):
+    """Rows with different tails and scales: the case where per-row resolutions differ."""
+    rng = np.random.default_rng(seed)
+    W = np.empty((rows, cols), np.float32)
+    for r in range(rows):
+        W[r] = rng.standard_t([2.5, 4, 8, 30][r % 4], cols) * 0.02 * np.exp(rng.normal(0, 0.5))
+    return W
+
+
+def _rel_l2(ob, W):
+    dec = oracle.decode_blob(ob, oracle.FP32).reshape(W.shape)
+    return float(np.linalg.norm(dec - W) / np.linalg.norm(W))
+
+
+def test_rdo_candidate_ratios_are_nested_log_bisections():
+    # §3.5: ratios in [0.70, 1.45], starting from 1, each bisecting the widest remaining interval
+    # in log scale (the two halves of [1, 1.45] tie; the lower one goes first)
+    want = [1.0, 1.45 ** 0.5, 0.70 ** 0.5, 1.45 ** 0.25, 1.45 ** 0.75]
+    np.testing.assert_allclose(oracle.rdo_ratios(5), want, rtol=1e-15)
+    r20 = oracle.rdo_ratios(20)
+    for k in range(1, 20):
+        np.testing.assert_array_equal(oracle.rdo_ratios(k), r20[:k])  # nested
+    assert np.all((r20 > 0.70) & (r20 < 1.45)) and len(set(r20)) == 20
+    gaps = np.diff(np.log(np.sort(np.concatenate([[0.70, 1.45], r20]))))
+    assert gaps.max() <= 2 * gaps.min() + 1e-12  # bisection keeps the log spacing within a factor 2
+
+
+def test_rdo_off_and_one_candidate_leave_the_stream_unchanged():
+    W = _heterogeneous_rows(seed=2, rows=64)
+    a = oracle.encode(W, 4.0)
+    for kw in (dict(rdo_candidates=1), dict(rdo_candidates=1, rdo_sweeps=3), dict(rdo_candidates=0)):
+        b = oracle.encode(W, 4.0, **kw)
+        for f in ("payload", "tile_index", "freq_tables", "row_scales"):
+            np.testing.assert_array_equal(getattr(a, f), getattr(b, f))
+
+
+@pytest.mark.parametrize("target", [2.0, 3.0, 5.0])
+def test_rdo_lowers_distortion_within_the_budget(target):
+    # the allocation keeps the baseline's storage budget and, with more resolutions per row,
+    # reconstructs closer (the paper's Fig. 4 direction: 14.35 % -> 14.11 % at K = 5)
+    W = _heterogeneous_rows(seed=3)
+    base = oracle.encode(W, target)
+    e0 = _rel_l2(base, W)
+    k5 = oracle.encode(W, target, rdo_candidates=5)
+    k9 = oracle.encode(W, target, rdo_candidates=9)
+    assert k5.stored_bpp <= base.stored_bpp * 1.002 and k9.stored_bpp <= base.stored_bpp * 1.002
+    e5, e9 = _rel_l2(k5, W), _rel_l2(k9, W)
+    assert e5 < e0 and e9 <= e5 * 1.005, (e0, e5, e9)
+    # the stored fields decode to themselves and every row scale is the refit of its own points
+    y = oracle.decode_blob(k5, oracle.LATTICE).reshape(W.shape).astype(np.float64) / 2
+    for r in range(0, W.shape[0], 37):
+        assert k5.row_scales[r] == oracle.refit_row(W[r], y[r])
+
+
+def test_rdo_second_sweep_keeps_the_budget():
+    W = _heterogeneous_rows(seed=4)
+    base = oracle.encode(W, 3.0)
+    two = oracle.encode(W, 3.0, rdo_candidates=5, rdo_sweeps=2)
+    assert two.stored_bpp <= base.stored_bpp * 1.002
+    assert _rel_l2(two, W) < _rel_l2(base, W)
