@@ -43,6 +43,8 @@ class _Opts(C.Structure):
         ("seed", C.c_uint64),
         ("has_container_scales", C.c_int),
         ("num_threads", C.c_int),
+        ("rdo_candidates", C.c_int),
+        ("rdo_sweeps", C.c_int),
     ]
 
 
@@ -140,12 +142,15 @@ class Blob:
 
 def encode_tensor(W: np.ndarray, target_bpp: float, *, prob_bits: int = 0, tile_vectors: int = 0,
                   sample_vectors: int = 0, search_steps: int = 0, seed: int = 0,
-                  has_container_scales: bool = False, num_threads: int = 0) -> Blob:
-    """Compress a host float32 matrix with the library's CPU packer (ep_encode_tensor)."""
+                  has_container_scales: bool = False, num_threads: int = 0, rdo_candidates: int = 0,
+                  rdo_sweeps: int = 0) -> Blob:
+    """Compress a host float32 matrix with the library's CPU packer (ep_encode_tensor);
+    rdo_candidates > 1 turns on the per-row refinement (App. C.2)."""
     W = np.ascontiguousarray(W, np.float32)
     if W.ndim != 2:
         raise ValueError("W must be 2-D")
-    o = _Opts(prob_bits, tile_vectors, sample_vectors, search_steps, seed, int(has_container_scales), num_threads)
+    o = _Opts(prob_bits, tile_vectors, sample_vectors, search_steps, seed, int(has_container_scales), num_threads,
+              int(rdo_candidates), int(rdo_sweeps))
     out = C.POINTER(_Blob)()
     rc = lib().ep_encode_tensor(W.ctypes.data, W.shape[0], W.shape[1], float(target_bpp), C.byref(o), C.byref(out))
     if rc:

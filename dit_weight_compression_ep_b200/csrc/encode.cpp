@@ -268,6 +268,168 @@ void normalise(Table& tb, int b) {
     for (uint32_t s = 0; s < tb.A; ++s) tb.cum[s + 1] = tb.cum[s] + tb.freq[s];
 }
 
+// ------------------------------------------------- per-row refinement (RDO)
+
+// Paper §3.5, App. C.2: K candidate ratios in [0.70, 1.45]: 1 first, then the
+// log-midpoint of the widest interval between neighbours and the range ends
+// (ties: the lower interval); nested in K.
+void rdo_ratios(int K, double* rho) {
+    double pts[2 + 64];
+    int n = 3;
+    pts[0] = 0.70;
+    pts[1] = 1.0;
+    pts[2] = 1.45;
+    rho[0] = 1.0;
+    for (int k = 1; k < K && k < 64; ++k) {
+        int best = 0;
+        double wbest = -1.0;
+        for (int i = 0; i + 1 < n; ++i) {
+            const double w = std::log(pts[i + 1] / pts[i]);
+            if (w > wbest) {
+                wbest = w;
+                best = i;
+            }
+        }
+        const double mid = std::sqrt(pts[best] * pts[best + 1]);
+        for (int i = n; i > best + 1; --i) pts[i] = pts[i - 1];
+        pts[best + 1] = mid;
+        ++n;
+        rho[k] = mid;
+    }
+}
+
+// Ideal code length of one row's fields under the tables, symbols in order; a
+// symbol the tables give no frequency costs b bits.
+double row_bits(const int32_t* f, int64_t nq, const Table* tabs, int b) {
+    double bits = 0.0;
+    for (int64_t q = 0; q < nq; ++q) {
+        const int32_t* v = f + kFields * q;
+        for (int k = 0; k < kFields; ++k) {
+            const Table& tb = tabs[table_index(k, v[0])];
+            const int64_t i = (int64_t)v[k] - tb.min;
+            const uint32_t fr = (tb.A && i >= 0 && i < (int64_t)tb.A) ? tb.freq[(size_t)i] : 0u;
+            bits += (double)b - std::log2((double)(fr ? fr : 1u));
+        }
+    }
+    return bits;
+}
+
+// Tables (alphabets, counts, frequencies at 2^b) of the given fields.
+void build_tables(const int32_t* f, int64_t nvec, int b, int nthreads, Table* tabs) {
+    const Hist al = alphabet_of(f, nvec, nthreads);
+    count_fields(f, nvec, al, tabs, nthreads);
+    for (int t = 0; t < kTables; ++t) normalise(tabs[t], b);
+}
+
+// App. C.2 allocation: every candidate of every row quantised at rho_k s and
+// refitted, its distortion sum (w - sigma y)^2; admissible when its symbols lie
+// in the baseline alphabets.  A sweep prices the candidates under the current
+// tables, bisects log2 lambda on [-80, 80] (64 steps) for the smallest lambda
+// whose choices argmin D + lambda R (ties: lowest k) fit the baseline's ideal
+// code length, and rebuilds the tables from the choices.  `fields` holds the
+// ratio-1 fields on entry and the chosen ones on return; `scales` the chosen
+// row scales.  Sums run in the same order as the documented algorithm.
+void rdo_refine(const float* W, int64_t rows, int64_t cols, const std::vector<double>& norms, double s, int b, int K,
+                int sweeps, int nthreads, std::vector<int32_t>& fields, std::vector<float>& scales) {
+    const int64_t nq = cols / 8, nvec = rows * nq, rowf = kFields * nq;
+    if (K > 64) K = 64;
+    double rho[64];
+    rdo_ratios(K, rho);
+    std::vector<int32_t> cf((size_t)(K * rows * rowf));
+    std::vector<float> cs((size_t)(K * rows));
+    std::vector<double> cd((size_t)(K * rows)), cr((size_t)(K * rows)), rsel((size_t)rows);
+    std::vector<uint8_t> ok((size_t)(K * rows));
+    std::vector<int> sel((size_t)rows, 0);
+    Table base[kTables];
+    build_tables(fields.data(), nvec, b, nthreads, base);
+    parallel_for(rows, nthreads, [&](int64_t a, int64_t e) {
+        std::vector<double> y((size_t)cols);
+        double u[8];
+        for (int64_t r = a; r < e; ++r) {
+            const float* w = W + r * cols;
+            for (int k = 0; k < K; ++k) {
+                const double sk = rho[k] * s;
+                int32_t* f = cf.data() + (size_t)((k * rows + r) * rowf);
+                double num = 0.0, den = 0.0;
+                for (int64_t q = 0; q < nq; ++q) {
+                    for (int i = 0; i < 8; ++i) u[i] = ((double)w[8 * q + i] / norms[r]) / sk;
+                    e8_fields(u, f + kFields * q, y.data() + 8 * q);
+                }
+                for (int64_t j = 0; j < cols; ++j) {
+                    num += (double)w[j] * y[j];
+                    den += y[j] * y[j];
+                }
+                const float sg = den == 0.0 ? 0.0f : (float)(num / den);
+                double d = 0.0;
+                for (int64_t j = 0; j < cols; ++j) {
+                    const double er = (double)w[j] - (double)sg * y[j];
+                    d += er * er;
+                }
+                uint8_t in = 1;
+                for (int64_t q = 0; q < nq && in; ++q)
+                    for (int m = 0; m < kFields; ++m) {
+                        const Table& tb = base[table_index(m, f[kFields * q])];
+                        const int64_t i = (int64_t)f[kFields * q + m] - tb.min;
+                        if (!tb.A || i < 0 || i >= (int64_t)tb.A) in = 0;
+                    }
+                cs[(size_t)(k * rows + r)] = sg;
+                cd[(size_t)(k * rows + r)] = d;
+                ok[(size_t)(k * rows + r)] = in;
+            }
+        }
+    });
+    parallel_for(rows, nthreads, [&](int64_t a, int64_t e) {
+        for (int64_t r = a; r < e; ++r) rsel[(size_t)r] = row_bits(cf.data() + (size_t)(r * rowf), nq, base, b);
+    });
+    double budget = 0.0;
+    for (int64_t r = 0; r < rows; ++r) budget += rsel[(size_t)r];
+    Table next[kTables];
+    const Table* model = base;
+    for (int sw = 0; sw < sweeps; ++sw) {
+        parallel_for(rows, nthreads, [&](int64_t a, int64_t e) {
+            for (int64_t r = a; r < e; ++r)
+                for (int k = 0; k < K; ++k) {
+                    const size_t i = (size_t)(k * rows + r);
+                    cr[i] = ok[i] ? row_bits(cf.data() + (size_t)((k * rows + r) * rowf), nq, model, b) : INFINITY;
+                }
+        });
+        double lo = -80.0, hi = 80.0;
+        for (int it = 0; it <= 64; ++it) {
+            const double t = it < 64 ? 0.5 * (lo + hi) : hi;
+            const double lam = std::exp2(t);
+            parallel_for(rows, nthreads, [&](int64_t a, int64_t e) {
+                for (int64_t r = a; r < e; ++r) {
+                    int best = 0;
+                    double jbest = cd[(size_t)r] + lam * cr[(size_t)r];
+                    for (int k = 1; k < K; ++k) {
+                        const double j = cd[(size_t)(k * rows + r)] + lam * cr[(size_t)(k * rows + r)];
+                        if (j < jbest) {
+                            jbest = j;
+                            best = k;
+                        }
+                    }
+                    sel[(size_t)r] = best;
+                    rsel[(size_t)r] = cr[(size_t)(best * rows + r)];
+                }
+            });
+            double total = 0.0;
+            for (int64_t r = 0; r < rows; ++r) total += rsel[(size_t)r];
+            if (it < 64) {
+                if (total <= budget) hi = t;
+                else lo = t;
+            }
+        }
+        parallel_for(rows, nthreads, [&](int64_t a, int64_t e) {
+            for (int64_t r = a; r < e; ++r)
+                std::memcpy(fields.data() + (size_t)(r * rowf), cf.data() + (size_t)((sel[(size_t)r] * rows + r) * rowf),
+                            sizeof(int32_t) * (size_t)rowf);
+        });
+        build_tables(fields.data(), nvec, b, nthreads, next);
+        model = next;
+    }
+    for (int64_t r = 0; r < rows; ++r) scales[(size_t)r] = cs[(size_t)(sel[(size_t)r] * rows + r)];
+}
+
 // ------------------------------------------------------------------- rANS
 
 // Encode one tile (vectors [v0, v0 + vt)): steps in reverse, lanes in reverse
@@ -457,6 +619,11 @@ ep_status ep_encode_tensor(const float* W, int64_t rows, int64_t cols, double ta
         }
         std::vector<float> scales(rows);
         for (int64_t r = 0; r < rows; ++r) scales[r] = den[r] == 0.0 ? 0.0f : (float)(num[r] / den[r]);
+        if (o.rdo_candidates > 1) {
+            rdo_refine(W, rows, cols, enc.norms, s, b, o.rdo_candidates, o.rdo_sweeps > 0 ? o.rdo_sweeps : 1,
+                       nthreads, fields, scales);
+            al = alphabet_of(fields.data(), nvec, nthreads);
+        }
 
         Table tabs[kTables];
         count_fields(fields.data(), nvec, al, tabs, nthreads);

@@ -72,6 +72,9 @@ typedef struct {
     uint64_t seed;            /* sample seed; 0: derived from the shape */
     int has_container_scales; /* 1: count 4 bytes per row of FP8/INT8 container scales in the rate */
     int num_threads;          /* 0: all hardware threads */
+    int rdo_candidates;       /* per-row rate-distortion refinement (§3.5, App. C.2): K candidate
+                                 scales per row (0 or 1: off, the default, as in the paper's results) */
+    int rdo_sweeps;           /* its allocation sweeps; 0: 1 */
 } ep_encode_opts;
 
 /* The packer's output; host memory owned by the library, freed by ep_free_blob. */
@@ -97,7 +100,9 @@ typedef struct {
  * ep_encode_tensor -- compress W (host, row-major float32 [rows, cols], the
  * container's values) to about target_bpp stored bits per weight.
  * Follows §3.1: row normalisation, sampled-row scale search (§3.4, App. C.1),
- * E8 quantisation, row-scale refit (§3.5), seventeen tables and tiled
+ * E8 quantisation, row-scale refit (§3.5), optional per-row refinement (§3.5,
+ * App. C.2: K candidate scales per row, allocated under the baseline's code
+ * length; memory grows by K x 36 bytes per vector), seventeen tables and tiled
  * interleaved rANS (§3.6, App. C.3).  Runs on the host with num_threads threads.
  * opts may be NULL.  On EP_OK *out holds a new blob (free with ep_free_blob).
  * Errors: EP_EINVAL (null W/out, rows or cols <= 0, target_bpp <= 0, b out of

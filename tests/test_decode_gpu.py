@@ -90,6 +90,16 @@ def test_one_coset_and_wide_alphabet():
     _check(as_lib_blob(ob), ALL_DT, "one coset, A = 2^b")
 
 
+def test_rdo_stream():
+    """A stream from the per-row refinement (App. C.2): rows at different resolutions, same decoder."""
+    rng = np.random.default_rng(14)
+    W = np.empty((128, 512), np.float32)
+    for r in range(128):
+        W[r] = rng.standard_t([2.5, 4, 8, 30][r % 4], 512) * 0.02 * np.exp(rng.normal(0, 0.5))
+    ob = oracle.encode(W, 3.0, rdo_candidates=5, tile_vectors=200)
+    _check(as_lib_blob(ob), [ep.BF16, ep.FP32, ep.LATTICE_I32], "rdo K=5")
+
+
 def test_zero_rows_and_signed_zeros():
     rng = np.random.default_rng(3)
     W = (rng.standard_normal((64, 512)) * 0.05).astype(np.float32)
@@ -125,6 +135,32 @@ def test_repeat_on_side_stream():
         b = _gpu(blob, ep.BF16, stream=s)
     np.testing.assert_array_equal(a, b)
     assert_parity(a, oracle_decode(blob, ep.BF16), ep.BF16, "side stream")
+
+
+def test_cuda_graph_capture_and_replay():
+    """Two decodes of different streams captured in one CUDA graph (the library's first call on
+    the device happens before the capture) and replayed: the same bits as the oracle."""
+    import torch
+
+    b1 = ep.encode_tensor(synth.generate(synth.small_fp32(seed=12)), 4.0)
+    b2 = ep.encode_tensor(synth.generate(synth.small_fp32(seed=13)), 6.0, tile_vectors=100)
+    d1, d2 = ep.DeviceBlob(b1), ep.DeviceBlob(b2)
+    o1 = ep.decode_tensor(d1, ep.BF16)
+    o2 = ep.decode_tensor(d2, ep.FP16)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        ep.decode_tensor(d1, ep.BF16, out=o1)
+        ep.decode_tensor(d2, ep.FP16, out=o2)
+    o1.zero_()
+    o2.zero_()
+    for _ in range(3):
+        g.replay()
+    torch.cuda.synchronize()
+    assert ep.decode_status() == 0
+    assert_parity(to_raw(o1).reshape(-1), oracle_decode(b1, ep.BF16), ep.BF16, "graph 1")
+    assert_parity(to_raw(o2).reshape(-1), oracle_decode(b2, ep.FP16), ep.FP16, "graph 2")
+    del g
 
 
 # ------------------------------------------------------------ corrupt streams

@@ -26,6 +26,15 @@ def _same(ob, lb):
     assert lb.s == ob.s
 
 
+def _mixed_rows(seed, rows=160, cols=512):
+    """Rows with different tails and scales (where the per-row refinement changes choices)."""
+    rng = np.random.default_rng(seed)
+    W = np.empty((rows, cols), np.float32)
+    for r in range(rows):
+        W[r] = rng.standard_t([2.5, 4, 8, 30][r % 4], cols) * 0.02 * np.exp(rng.normal(0, 0.5))
+    return W
+
+
 CASES = [
     ("small fp32", lambda: synth.generate(synth.small_fp32()), 4.0, dict(prob_bits=12, tile_vectors=512)),
     ("t5 2bpp", lambda: (np.random.default_rng(1).standard_t(5, (300, 512)) * 0.02).astype(np.float32), 2.0, {}),
@@ -42,6 +51,9 @@ CASES = [
      dict(has_container_scales=True)),
     ("small sample", lambda: (np.random.default_rng(8).standard_normal((400, 256)) * 0.02).astype(np.float32), 4.0,
      dict(sample_vectors=500, seed=77, search_steps=9)),
+    ("rdo K=5", lambda: _mixed_rows(9), 3.0, dict(rdo_candidates=5)),
+    ("rdo K=7 two sweeps 8bpp", lambda: _mixed_rows(10), 8.0, dict(rdo_candidates=7, rdo_sweeps=2)),
+    ("rdo K=3 2bpp", lambda: _mixed_rows(11, rows=96), 2.0, dict(rdo_candidates=3)),
 ]
 
 
