@@ -203,7 +203,7 @@ def decode_fields(payload, tile_index, freq_tables, rows: int, cols: int, t0: in
     ntiles = (tile_index.size - 1) // 33
     t1 = ntiles if t1 is None else t1
     V = int(freq_tables[12:16].view(np.uint32)[0]) if V is None else V
-    nvec = rows * (cols // 8)
+    nvec = rows * -(-cols // 8)
     nv = min(t1 * V, nvec) - t0 * V
     out = np.zeros((max(nv, 0), 9), np.int32)
     rc = lib().epo_decode_fields(_p(payload), _p(tile_index), _p(freq_tables), rows, cols, t0, t1,
@@ -215,15 +215,18 @@ def decode_fields(payload, tile_index, freq_tables, rows: int, cols: int, t0: in
 
 def decode(payload, tile_index, freq_tables, row_scales, rows: int, cols: int, dtype: int,
            t0: int = 0, t1: int | None = None) -> np.ndarray:
-    """Decode tiles [t0, t1) to dtype; returns the tiles' weights flat (8 per vector)."""
+    """Decode tiles [t0, t1) to dtype; returns the tiles' weights flat: the contiguous range of
+    the row-major matrix their vectors cover (8 per vector, fewer at a padded row end)."""
     payload, tile_index, freq_tables = _bufs(payload, tile_index, freq_tables)
     row_scales = np.ascontiguousarray(row_scales, dtype=np.float32)
     ntiles = (tile_index.size - 1) // 33
     t1 = ntiles if t1 is None else t1
     V = int(freq_tables[12:16].view(np.uint32)[0])
-    nvec = rows * (cols // 8)
-    nv = min(t1 * V, nvec) - t0 * V
-    out = np.zeros(max(nv, 0) * 8, _NP_OUT[dtype])
+    nq = -(-cols // 8)  # vectors per row: rows are padded to whole vectors
+    nvec = rows * nq
+    v0, v1 = t0 * V, min(t1 * V, nvec)
+    elem = lambda v: (v // nq) * cols + 8 * (v % nq) if v < nvec else rows * cols  # noqa: E731
+    out = np.zeros(max(elem(v1) - elem(v0), 0) if v1 > v0 else 0, _NP_OUT[dtype])
     rc = lib().epo_decode(_p(payload), _p(tile_index), _p(freq_tables), _p(row_scales), rows, cols, dtype,
                           t0, t1, _p(out) if out.size else None)
     if rc:

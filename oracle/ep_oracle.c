@@ -106,13 +106,13 @@ uint64_t epo_shape_seed(int64_t rows, int64_t cols) {
 /*
  * Sampled rate evaluation (App. C.1): complete rows, nominal budget of
  * sample_vectors eight-dimensional vectors, fixed for the whole search.
- * READING: Rs = min(rows, ceil(sample_vectors / (cols/8))) rows drawn without
+ * READING: Rs = min(rows, ceil(sample_vectors / ceil(cols/8))) rows drawn without
  * replacement by a partial Fisher-Yates shuffle; r_i = i + (next mod (rows - i)).
  * Returns Rs; out_rows receives the chosen rows in draw order.
  */
 int64_t epo_sample_rows(int64_t rows, int64_t cols, int64_t sample_vectors, uint64_t seed,
                         int64_t* out_rows) {
-    int64_t nq = cols / 8;
+    int64_t nq = ceil_div(cols, 8);
     int64_t rs = ceil_div(sample_vectors, nq);
     if (rs > rows) rs = rows;
     if (rs < 1) rs = 1;
@@ -400,14 +400,16 @@ static int64_t header_bytes(int ntab) {
 
 /* ------------------------------------------------------------------------ */
 /* Quantisation of whole rows at scale s: u = (w / n_r) / s, y = Q_E8(u).   */
+/* READING (cols % 8 != 0): the row is padded with zeros to whole vectors;  */
+/* the padding is quantised with its vector and dropped by the decoder.     */
 /* ------------------------------------------------------------------------ */
 
 static void quantize_row(const float* w, int64_t cols, double norm, double s, int direct_z8,
                          int32_t* fields_out, double* y_out /* nullable, 8 per vector */) {
     double u[8], y[8];
     int64_t f[NFIELDS];
-    for (int64_t q = 0; q < cols / 8; ++q) {
-        for (int k = 0; k < 8; ++k) u[k] = ((double)w[8 * q + k] / norm) / s;
+    for (int64_t q = 0; q < ceil_div(cols, 8); ++q) {
+        for (int k = 0; k < 8; ++k) u[k] = 8 * q + k < cols ? ((double)w[8 * q + k] / norm) / s : 0.0;
         int c = epo_quantize_e8(u, y);
         epo_fields_from_point(y, c, direct_z8, f);
         for (int k = 0; k < NFIELDS; ++k) fields_out[NFIELDS * q + k] = (int32_t)f[k];
@@ -439,7 +441,7 @@ static int64_t side_bytes(const shape_t* sh, const table_t* tabs) {
 
 static double estimate_rate(const shape_t* sh, const float* W, const double* norms,
                             const int64_t* srows, int64_t rs, double s, int b, int32_t* scratch_fields) {
-    int64_t nq = sh->cols / 8;
+    int64_t nq = ceil_div(sh->cols, 8);
     for (int64_t i = 0; i < rs; ++i) {
         int64_t r = srows[i];
         quantize_row(W + r * sh->cols, sh->cols, norms[r], s, sh->direct_z8, scratch_fields + NFIELDS * nq * i, NULL);
@@ -458,7 +460,7 @@ static double estimate_rate(const shape_t* sh, const float* W, const double* nor
                 if (tabs[t].count[k]) bits += (double)tabs[t].count[k] * ((double)b - log2((double)tabs[t].freq[k]));
         double payload_bytes = bits / 8.0 * ((double)sh->nvec / (double)nsamp);
         double total = payload_bytes + (double)side_bytes(sh, tabs);
-        rate = 8.0 * total / (double)(sh->nvec * 8);
+        rate = 8.0 * total / (double)(sh->rows * sh->cols); /* per real weight */
     }
     for (int t = 0; t < sh->ntab; ++t) table_free(&tabs[t]);
     return rate;
@@ -579,7 +581,7 @@ static void write_tables(epo_blob* bl, const table_t* tabs) {
 }
 
 /*
- * Entropy-code given fields (rows x cols/8 vectors, 9 fields each) with given
+ * Entropy-code given fields (rows x ceil(cols/8) vectors, 9 fields each) with given
  * row scales: tables from the full-tensor counts (§3.6 "We recount the final
  * full-tensor fields"), tiles of V vectors, interleaved rANS per tile.
  * Returns 0, or a negative code when an alphabet exceeds 2^b.
@@ -619,11 +621,11 @@ static int code_fields(epo_blob* bl, int pooled) {
 int epo_encode_fields(const int32_t* fields, int64_t rows, int64_t cols, const float* row_scales, int b, int V,
                       int flags, epo_blob** out) {
     *out = NULL;
-    if (rows <= 0 || cols <= 0 || cols % 8 || b < 9 || b > 15 || V < 1) return -1;
+    if (rows <= 0 || cols <= 0 || b < 9 || b > 15 || V < 1) return -1;
     epo_blob* bl = (epo_blob*)calloc(1, sizeof(epo_blob));
     bl->rows = rows;
     bl->cols = cols;
-    bl->nvec = rows * (cols / 8);
+    bl->nvec = rows * ceil_div(cols, 8);
     bl->b = b;
     bl->V = V;
     bl->flags = flags;
@@ -727,7 +729,7 @@ static double row_bits(const int32_t* f, int64_t nq, const table_t* tabs, int b,
  */
 static void rdo_refine(const shape_t* sh, const float* W, const double* norms, double s, int b, int K, int sweeps,
                        int32_t* fields, float* scales) {
-    const int64_t rows = sh->rows, cols = sh->cols, nq = cols / 8, rowf = NFIELDS * nq;
+    const int64_t rows = sh->rows, cols = sh->cols, nq = ceil_div(cols, 8), rowf = NFIELDS * nq;
     double rho[64];
     if (K > 64) K = 64;
     epo_rdo_ratios(K, rho);
@@ -737,7 +739,7 @@ static void rdo_refine(const shape_t* sh, const float* W, const double* norms, d
     double* cr = (double*)malloc(sizeof(double) * (size_t)(K * rows));
     unsigned char* ok = (unsigned char*)malloc((size_t)(K * rows));
     int* sel = (int*)malloc(sizeof(int) * (size_t)rows);
-    double* y = (double*)malloc(sizeof(double) * (size_t)cols);
+    double* y = (double*)malloc(sizeof(double) * (size_t)(8 * nq));
     table_t base[MAX_TABLES], tabs[MAX_TABLES];
     count_tables(fields, sh->nvec, sh->pooled, sh->ntab, UINT64_MAX, base);
     build_freqs(base, sh->ntab, b);
@@ -811,20 +813,20 @@ static void rdo_refine(const shape_t* sh, const float* W, const double* norms, d
 
 int epo_encode(const float* W, int64_t rows, int64_t cols, const epo_opts* opts, epo_blob** out) {
     *out = NULL;
-    if (rows <= 0 || cols <= 0 || cols % 8) return -1;
+    if (rows <= 0 || cols <= 0) return -1;
     if (!(opts->target_bpp > 0.0)) return -1;
     int flags = (opts->direct_z8 ? 1 : 0) | (opts->pooled ? 2 : 0);
     shape_t sh;
     sh.rows = rows;
     sh.cols = cols;
-    sh.nvec = rows * (cols / 8);
+    sh.nvec = rows * ceil_div(cols, 8);
     sh.pooled = opts->pooled != 0;
     sh.direct_z8 = opts->direct_z8 != 0;
     sh.ntab = sh.pooled ? 9 : 17;
     sh.has_container_scales = opts->has_container_scales != 0;
     int64_t V = opts->tile_vectors > 0 ? opts->tile_vectors : epo_tile_vectors(epo_default_tile_symbols(opts->target_bpp));
     sh.ntiles = ceil_div(sh.nvec, V);
-    int64_t nq = cols / 8;
+    int64_t nq = ceil_div(cols, 8);
 
     double* norms = (double*)malloc(sizeof(double) * (size_t)rows);
     for (int64_t r = 0; r < rows; ++r) norms[r] = epo_row_norm(W + r * cols, cols);
@@ -844,7 +846,7 @@ int epo_encode(const float* W, int64_t rows, int64_t cols, const epo_opts* opts,
     bl->target_bpp = opts->target_bpp;
     bl->has_container_scales = sh.has_container_scales;
     bl->fields = (int32_t*)malloc(sizeof(int32_t) * (size_t)(NFIELDS * sh.nvec));
-    double* ys = (double*)malloc(sizeof(double) * (size_t)(rows * cols));
+    double* ys = (double*)malloc(sizeof(double) * (size_t)(rows * 8 * nq)); /* 8 per vector */
 
     int steps = opts->search_steps > 0 ? opts->search_steps : 12;
     int b = opts->prob_bits > 0 ? opts->prob_bits : (opts->target_bpp <= 7.0 ? 11 : 12);
@@ -864,7 +866,7 @@ int epo_encode(const float* W, int64_t rows, int64_t cols, const epo_opts* opts,
         }
         s = sqrt(lo * hi);
         for (int64_t r = 0; r < rows; ++r)
-            quantize_row(W + r * cols, cols, norms[r], s, sh.direct_z8, bl->fields + NFIELDS * nq * r, ys + r * cols);
+            quantize_row(W + r * cols, cols, norms[r], s, sh.direct_z8, bl->fields + NFIELDS * nq * r, ys + r * 8 * nq);
         table_t tabs[MAX_TABLES];
         uint64_t amax = count_tables(bl->fields, sh.nvec, sh.pooled, sh.ntab, 0, tabs);
         for (int t = 0; t < sh.ntab; ++t) table_free(&tabs[t]);
@@ -878,7 +880,7 @@ int epo_encode(const float* W, int64_t rows, int64_t cols, const epo_opts* opts,
             s = 1.05 * s * (double)amax / (double)(1u << b);
             for (int64_t r = 0; r < rows; ++r)
                 quantize_row(W + r * cols, cols, norms[r], s, sh.direct_z8, bl->fields + NFIELDS * nq * r,
-                             ys + r * cols);
+                             ys + r * 8 * nq);
             amax = count_tables(bl->fields, sh.nvec, sh.pooled, sh.ntab, 0, tabs);
             for (int t = 0; t < sh.ntab; ++t) table_free(&tabs[t]);
         }
@@ -887,7 +889,8 @@ int epo_encode(const float* W, int64_t rows, int64_t cols, const epo_opts* opts,
     bl->b = b;
     bl->s = s;
     bl->row_scales = (float*)malloc(sizeof(float) * (size_t)rows);
-    for (int64_t r = 0; r < rows; ++r) bl->row_scales[r] = epo_refit_row(W + r * cols, ys + r * cols, cols);
+    /* the refit runs over the row's real entries (the padding is not data) */
+    for (int64_t r = 0; r < rows; ++r) bl->row_scales[r] = epo_refit_row(W + r * cols, ys + r * 8 * nq, cols);
     if (opts->rdo_candidates > 1)
         rdo_refine(&sh, W, norms, s, b, opts->rdo_candidates, opts->rdo_sweeps > 0 ? opts->rdo_sweeps : 1,
                    bl->fields, bl->row_scales);
@@ -909,14 +912,14 @@ double epo_estimate_rate(const float* W, int64_t rows, int64_t cols, const epo_o
     shape_t sh;
     sh.rows = rows;
     sh.cols = cols;
-    sh.nvec = rows * (cols / 8);
+    sh.nvec = rows * ceil_div(cols, 8);
     sh.pooled = opts->pooled != 0;
     sh.direct_z8 = opts->direct_z8 != 0;
     sh.ntab = sh.pooled ? 9 : 17;
     sh.has_container_scales = opts->has_container_scales != 0;
     int64_t V = opts->tile_vectors > 0 ? opts->tile_vectors : epo_tile_vectors(epo_default_tile_symbols(opts->target_bpp));
     sh.ntiles = ceil_div(sh.nvec, V);
-    int64_t nq = cols / 8;
+    int64_t nq = ceil_div(cols, 8);
     double* norms = (double*)malloc(sizeof(double) * (size_t)rows);
     for (int64_t r = 0; r < rows; ++r) norms[r] = epo_row_norm(W + r * cols, cols);
     int64_t* srows = (int64_t*)malloc(sizeof(int64_t) * (size_t)rows);
@@ -1110,9 +1113,9 @@ static int dmodel_load(const uint8_t* ft, int64_t rows, int64_t cols, dmodel_t* 
     m->ntab = (int)get_u32(ft + 40);
     m->flags = (int)get_u32(ft + 44);
     if (m->b < 9 || m->b > 15 || m->V < 1) return -5;
-    if (m->rows != rows || m->cols != cols || cols % 8) return -5;
+    if (m->rows != rows || m->cols != cols) return -5;
     if (!((m->ntab == 17 && !(m->flags & 2)) || (m->ntab == 9 && (m->flags & 2)))) return -5;
-    m->nvec = rows * (cols / 8);
+    m->nvec = rows * ceil_div(cols, 8);
     if (m->ntiles != ceil_div(m->nvec, m->V)) return -5;
     uint32_t M = 1u << m->b;
     int64_t o = header_bytes(m->ntab);
@@ -1224,16 +1227,19 @@ int epo_decode(const uint16_t* payload, const uint32_t* tile_index, const uint8_
     int32_t* fields = (int32_t*)malloc(sizeof(int32_t) * (size_t)(NFIELDS * (nv > 0 ? nv : 1)));
     rc = decode_tiles_fields(&m, payload, tile_index, t0, t1, fields);
     int direct = (m.flags & 1) != 0;
-    int64_t nq = cols / 8;
+    /* vector v holds elements row * cols + 8q .. (row = v / nq, q = v % nq) up to the row's
+     * end; the vectors [v0, v1) cover the contiguous element range [E(v0), E(v1)) */
+    int64_t nq = ceil_div(cols, 8);
+    int64_t e0 = (v0 / nq) * cols + 8 * (v0 % nq);
     int sz = dtype_size(dtype);
     for (int64_t i = 0; !rc && i < nv; ++i) {
         int64_t f[NFIELDS], y2[8];
         for (int k = 0; k < NFIELDS; ++k) f[k] = fields[NFIELDS * i + k];
         epo_point_from_fields(f, direct, y2);
-        int64_t row = (v0 + i) / nq;
+        int64_t row = (v0 + i) / nq, q = (v0 + i) % nq;
         float sigma = row_scales[row];
-        uint8_t* o = (uint8_t*)out + (size_t)(8 * i) * (size_t)sz;
-        for (int k = 0; k < 8; ++k) {
+        uint8_t* o = (uint8_t*)out + (size_t)(row * cols + 8 * q - e0) * (size_t)sz;
+        for (int k = 0; k < 8 && 8 * q + k < cols; ++k) {
             if (dtype == EPO_LATTICE) {
                 ((int32_t*)o)[k] = (int32_t)y2[k];
                 continue;
