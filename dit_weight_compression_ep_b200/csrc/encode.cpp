@@ -101,16 +101,18 @@ inline void e8_fields(const double* u, int32_t* f, double* y) {
     for (int k = 0; k < 8; ++k) y[k] = z[k] + 0.5 * c;
 }
 
-// Quantise one row at scale s: u = (w / n) / s; fields into f (9 per vector);
-// optional refit sums <w, y> and <y, y> in index order.
+// Quantise one row at scale s: u = (w / n) / s, a partial last vector padded
+// with zeros; fields into f (9 per vector); optional refit sums <w, y> and
+// <y, y> over the real entries in index order.
 void quantize_row(const float* w, int64_t cols, double n, double s, int32_t* f, double* num, double* den) {
     double u[8], y[8];
     double sn = 0.0, sd = 0.0;
-    for (int64_t q = 0; q < cols / 8; ++q) {
-        for (int k = 0; k < 8; ++k) u[k] = ((double)w[8 * q + k] / n) / s;
+    for (int64_t q = 0; q < (cols + 7) / 8; ++q) {
+        const int real = (int)std::min<int64_t>(8, cols - 8 * q);
+        for (int k = 0; k < 8; ++k) u[k] = k < real ? ((double)w[8 * q + k] / n) / s : 0.0;
         e8_fields(u, f + kFields * q, y);
         if (num) {
-            for (int k = 0; k < 8; ++k) {
+            for (int k = 0; k < real; ++k) {
                 sn += (double)w[8 * q + k] * y[k];
                 sd += y[k] * y[k];
             }
@@ -331,7 +333,7 @@ void build_tables(const int32_t* f, int64_t nvec, int b, int nthreads, Table* ta
 // row scales.  Sums run in the same order as the documented algorithm.
 void rdo_refine(const float* W, int64_t rows, int64_t cols, const std::vector<double>& norms, double s, int b, int K,
                 int sweeps, int nthreads, std::vector<int32_t>& fields, std::vector<float>& scales) {
-    const int64_t nq = cols / 8, nvec = rows * nq, rowf = kFields * nq;
+    const int64_t nq = (cols + 7) / 8, nvec = rows * nq, rowf = kFields * nq;
     if (K > 64) K = 64;
     double rho[64];
     rdo_ratios(K, rho);
@@ -343,7 +345,7 @@ void rdo_refine(const float* W, int64_t rows, int64_t cols, const std::vector<do
     Table base[kTables];
     build_tables(fields.data(), nvec, b, nthreads, base);
     parallel_for(rows, nthreads, [&](int64_t a, int64_t e) {
-        std::vector<double> y((size_t)cols);
+        std::vector<double> y((size_t)(8 * nq));
         double u[8];
         for (int64_t r = a; r < e; ++r) {
             const float* w = W + r * cols;
@@ -352,7 +354,7 @@ void rdo_refine(const float* W, int64_t rows, int64_t cols, const std::vector<do
                 int32_t* f = cf.data() + (size_t)((k * rows + r) * rowf);
                 double num = 0.0, den = 0.0;
                 for (int64_t q = 0; q < nq; ++q) {
-                    for (int i = 0; i < 8; ++i) u[i] = ((double)w[8 * q + i] / norms[r]) / sk;
+                    for (int i = 0; i < 8; ++i) u[i] = 8 * q + i < cols ? ((double)w[8 * q + i] / norms[r]) / sk : 0.0;
                     e8_fields(u, f + kFields * q, y.data() + 8 * q);
                 }
                 for (int64_t j = 0; j < cols; ++j) {
@@ -513,7 +515,7 @@ struct Encoder {
         }
         const double payload = bits / 8.0 * ((double)nvec / (double)ns);
         const double total = payload + (double)side_bytes(al);
-        return 8.0 * total / (double)(nvec * 8);
+        return 8.0 * total / (double)(rows * cols);  // per real weight
     }
 };
 
@@ -528,12 +530,11 @@ ep_status ep_encode_tensor(const float* W, int64_t rows, int64_t cols, double ta
     if (!W || !out) return EP_EINVAL;
     *out = nullptr;
     if (rows <= 0 || cols <= 0 || !(target_bpp > 0.0)) return EP_EINVAL;
-    if (cols % 8) return EP_EUNSUPPORTED;
     ep_encode_opts o{};
     if (opts) o = *opts;
     int b = o.prob_bits > 0 ? o.prob_bits : (target_bpp <= 7.0 ? 11 : 12);
     if (b < kMinB || b > kMaxB) return EP_EINVAL;
-    const int64_t nq = cols / 8, nvec = rows * nq;
+    const int64_t nq = (cols + 7) / 8, nvec = rows * nq;  // rows padded to whole vectors
     if (nvec >= (1ll << 31)) return EP_EINVAL;
     const int64_t V = o.tile_vectors > 0 ? o.tile_vectors : std::max<int64_t>(32, tile_symbols_for(target_bpp) / 9);
     int nthreads = o.num_threads > 0 ? o.num_threads : (int)std::max(1u, std::thread::hardware_concurrency());

@@ -71,8 +71,9 @@ def test_decode_rejects_bad_arguments_on_host(lib):
 
 def test_encode_rejects_bad_arguments(lib):
     W = np.zeros((4, 16), np.float32)
+    assert ep.encode_tensor(np.ones((4, 12), np.float32), 4.0).cols == 12  # rows padded to whole vectors
     with pytest.raises(ep.EntroPackError):
-        ep.encode_tensor(np.zeros((4, 12), np.float32), 4.0)     # cols % 8
+        ep.encode_tensor(np.zeros((0, 16), np.float32), 4.0)      # no rows
     with pytest.raises(ep.EntroPackError):
         ep.encode_tensor(W, 0.0)
     with pytest.raises(ep.EntroPackError):

@@ -51,6 +51,11 @@ CASES = [
      dict(has_container_scales=True)),
     ("small sample", lambda: (np.random.default_rng(8).standard_normal((400, 256)) * 0.02).astype(np.float32), 4.0,
      dict(sample_vectors=500, seed=77, search_steps=9)),
+    ("ragged 1001", lambda: (np.random.default_rng(12).standard_t(5, (90, 1001)) * 0.02).astype(np.float32), 4.0, {}),
+    ("ragged 60", lambda: (np.random.default_rng(13).standard_normal((300, 60)) * 0.02).astype(np.float32), 6.0,
+     dict(tile_vectors=50)),
+    ("ragged 5", lambda: (np.random.default_rng(14).standard_normal((700, 5)) * 0.02).astype(np.float32), 3.0, {}),
+    ("rdo ragged 517", lambda: _mixed_rows(15, cols=517), 3.0, dict(rdo_candidates=5)),
     ("rdo K=5", lambda: _mixed_rows(9), 3.0, dict(rdo_candidates=5)),
     ("rdo K=7 two sweeps 8bpp", lambda: _mixed_rows(10), 8.0, dict(rdo_candidates=7, rdo_sweeps=2)),
     ("rdo K=3 2bpp", lambda: _mixed_rows(11, rows=96), 2.0, dict(rdo_candidates=3)),
