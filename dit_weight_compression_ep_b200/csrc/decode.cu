@@ -215,7 +215,7 @@ __device__ unsigned parse_header(const uint8_t* ft, int64_t rows, int64_t cols, 
     g.b = h[kHB];
     g.V = h[kHV];
     g.T = h[kHT];
-    g.nvec = rows * (cols / 8);
+    g.nvec = rows * ((cols + 7) / 8);  // rows padded to whole vectors
     const int64_t hrows = (int64_t)(((uint64_t)h[2 * kHRows64 + 1] << 32) | h[2 * kHRows64]);
     const int64_t hcols = (int64_t)(((uint64_t)h[2 * kHCols64 + 1] << 32) | h[2 * kHCols64]);
     bool ok = h[kHMagic] == kMagic && h[kHVersion] == kVersion && h[kHJ] == (uint32_t)kLanes &&
@@ -399,6 +399,24 @@ __device__ __forceinline__ bool build_lut_slice(const Geo& g, const uint16_t* fq
 
 template <int DT>
 struct Out;
+
+// One element of the output type (the element-wise path of rows padded to whole vectors).
+template <int DT>
+__device__ __forceinline__ void put_elem(void* out, int64_t i, float w) {
+    if constexpr (DT == EP_BF16) {
+        reinterpret_cast<__nv_bfloat16*>(out)[i] = __float2bfloat16_rn(w);
+    } else if constexpr (DT == EP_FP16) {
+        reinterpret_cast<__half*>(out)[i] = __float2half_rn(w);
+    } else if constexpr (DT == EP_FP8_E4M3) {
+        reinterpret_cast<__nv_fp8_storage_t*>(out)[i] = __nv_cvt_float_to_fp8(w, __NV_SATFINITE, __NV_E4M3);
+    } else if constexpr (DT == EP_INT8) {
+        reinterpret_cast<int8_t*>(out)[i] = (int8_t)__float2int_rn(fminf(fmaxf(w, -127.0f), 127.0f));
+    } else if constexpr (DT == EP_UINT8) {
+        reinterpret_cast<uint8_t*>(out)[i] = (uint8_t)(__float2int_rn(fminf(fmaxf(w, -128.0f), 127.0f)) + 128);
+    } else {
+        reinterpret_cast<float*>(out)[i] = w;
+    }
+}
 
 template <>
 struct Out<EP_BF16> {
@@ -631,6 +649,7 @@ struct TileCtx {
     // 2, 4, 2^16, -2^b, f1c - f0c, -f0c: run-time multipliers (integer multiply-adds run
     // beside the shift / logic / compare unit instead of on it)
     uint32_t two, four, k64, mneg, df, nf0;
+    int64_t cols;  // (a width that is not a multiple of 8 pads each row to whole vectors)
 };
 
 // One tile's bookkeeping: record, staging state and every lane's row.
@@ -710,7 +729,7 @@ __device__ __forceinline__ void renorm(uint32_t& x, uint32_t xn, bool act, uint3
     pb = __popc(bal) * tc.two + pb;
 }
 
-template <int DT, typename Lut, bool FULL>
+template <int DT, bool RAGGED, typename Lut, bool FULL>
 __device__ __forceinline__ void decode_round(void* out, const float sigma, const Lut& lut, const TileCtx& tc,
                                              Tile& tl, uint32_t& pb, uint32_t r, uint32_t lt, int lane,
                                              bool& corrupt) {
@@ -764,7 +783,22 @@ __device__ __forceinline__ void decode_round(void* out, const float sigma, const
     if (badsym && act) corrupt = true;
 
     if (act) {
-        if constexpr (DT == EP_LATTICE_I32) {
+        if constexpr (RAGGED) {
+            // vector g holds elements row * cols + 8q .. of a row padded to whole vectors
+            const uint32_t row = (uint32_t)(g / tc.nq), q = (uint32_t)g - row * tc.nq;
+            const int64_t e0 = (int64_t)row * tc.cols + 8 * (int64_t)q;
+            const int n = (int)min((int64_t)8, tc.cols - 8 * (int64_t)q);
+            if constexpr (DT == EP_LATTICE_I32) {
+#pragma unroll
+                for (int k = 0; k < 8; ++k)  // constant indices keep yb in registers
+                    if (k < n) reinterpret_cast<int*>(out)[e0 + k] = (int)(yb[k] - 0x4AC00000u);
+            } else {
+                wf[7] = sigma * (__uint_as_float(yb[7]) - 6291456.0f);
+#pragma unroll
+                for (int k = 0; k < 8; ++k)
+                    if (k < n) put_elem<DT>(out, e0 + k, wf[k]);
+            }
+        } else if constexpr (DT == EP_LATTICE_I32) {
             int4* o = reinterpret_cast<int4*>(out) + 2 * g;
             o[0] = make_int4((int)(yb[0] - 0x4AC00000u), (int)(yb[1] - 0x4AC00000u), (int)(yb[2] - 0x4AC00000u),
                              (int)(yb[3] - 0x4AC00000u));
@@ -778,7 +812,7 @@ __device__ __forceinline__ void decode_round(void* out, const float sigma, const
 }
 
 // Decode the tiles of this warp; the first one was begun in the prologue.
-template <int DT, typename Lut>
+template <int DT, bool RAGGED, typename Lut>
 __device__ void decode_tiles(const uint16_t* tiles, const uint32_t* tix, const float* scales, void* out,
                              const Lut& lut, const TileCtx& tc, Ring& rg, Tile& tl, uint32_t first_i) {
     const int lane = threadIdx.x & 31;
@@ -831,7 +865,7 @@ __device__ void decode_tiles(const uint16_t* tiles, const uint32_t* tix, const f
                     }
                 }
                 if (FULL) sig_next = ((r + 1) << 5) + lane < tl.vt ? __ldg(scales + tl.rowl) : 1.0f;
-                decode_round<DT, Lut, FULL>(out, sigma, lut, tc, tl, pb, r, lt, lane, corrupt);
+                decode_round<DT, RAGGED, Lut, FULL>(out, sigma, lut, tc, tl, pb, r, lt, lane, corrupt);
                 cur += (pb - p_start) >> 1;
             };
             for (uint32_t r = 0; r + 1 < tl.rounds; ++r) round(std::true_type{}, r);
@@ -869,7 +903,53 @@ struct Params {
     uint32_t one;  // 1, set by the host (see TileCtx)
 };
 
-template <int DT>
+// The decode loop for the stream's LUT format.  Rows padded to whole vectors (a width
+// that is not a multiple of 8) run a separate kernel (RAGGED: element-wise stores), so
+// the vector-store kernel is compiled without that path.
+template <int DT, bool R>
+__device__ __forceinline__ void run_decode(const Params& p, const Geo& g, uint32_t lut_s, const uint16_t* fq,
+                                           const int* s_min, const uint32_t* s_A, const uint32_t* s_off,
+                                           uint32_t desc2, const TileCtx& tc, Ring& rg, Tile& tl, uint32_t first_i) {
+#define EP_PACKED(BB, FF) \
+    decode_tiles<DT, R>(p.tiles, p.tix, p.scales, p.out,                                              \
+                     PackedLut<BB, FF>{lut_s, tc.four, 0u - (p.one << (BB + 2))},                      \
+                     tc, rg, tl, first_i)
+    switch (g.mode) {
+        case 9: EP_PACKED(9, false); break;
+        case 10: EP_PACKED(10, false); break;
+        case 11: EP_PACKED(11, false); break;
+        case kModeF + 9: EP_PACKED(9, true); break;
+        case kModeF + 10: EP_PACKED(10, true); break;
+        case kModeF + 11: EP_PACKED(11, true); break;
+        case kModeTwo:
+        case kModeTwoPair: {
+            const bool pair = g.mode == kModeTwoPair;
+            if (pair)
+                decode_tiles<DT, R>(p.tiles, p.tix, p.scales, p.out,
+                                 TwoLut<true>{lut_s, g.b, g.M - 1u, g.M, desc2, s_A}, tc, rg, tl, first_i);
+            else
+                decode_tiles<DT, R>(p.tiles, p.tix, p.scales, p.out,
+                                 TwoLut<false>{lut_s, g.b, g.M - 1u, 2u * g.M, desc2, s_A}, tc, rg, tl, first_i);
+            break;
+        }
+        default: {
+            CoarseLut cl;
+            cl.lut_s = lut_s;
+            cl.b = g.b;
+            cl.mmask = g.M - 1;
+            cl.sh = g.b - g.k;
+            cl.nb_shift = g.k;
+            cl.fq = fq;
+            cl.s_min = s_min;
+            cl.s_A = s_A;
+            cl.s_off = s_off;
+            decode_tiles<DT, R>(p.tiles, p.tix, p.scales, p.out, cl, tc, rg, tl, first_i);
+        }
+    }
+#undef EP_PACKED
+}
+
+template <int DT, bool RAGGED>
 __global__ void __launch_bounds__(kThreads, 1) decode_kernel(Params p) {
     extern __shared__ __align__(1024) uint8_t smem[];
     __shared__ int s_ok;
@@ -930,7 +1010,8 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(Params p) {
     tc.nvec = g.nvec;
     tc.V = g.V;
     tc.T = g.T;
-    tc.nq = (uint32_t)(p.cols / 8);
+    tc.nq = (uint32_t)((p.cols + 7) / 8);
+    tc.cols = p.cols;
     tc.b = g.b;
     tc.two = p.one << 1;
     tc.four = p.one << 2;
@@ -1024,44 +1105,8 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(Params p) {
     }
 
     const uint32_t lut_s = smem_u32(smem + kOffLut);
-#define EP_PACKED(BB, FF) \
-    decode_tiles<DT>(p.tiles, p.tix, p.scales, p.out,                                              \
-                     PackedLut<BB, FF>{lut_s, tc.four, 0u - (p.one << (BB + 2))},                      \
-                     tc, rg, tl, first_i)
-    switch (g.mode) {
-        case 9: EP_PACKED(9, false); break;
-        case 10: EP_PACKED(10, false); break;
-        case 11: EP_PACKED(11, false); break;
-        case kModeF + 9: EP_PACKED(9, true); break;
-        case kModeF + 10: EP_PACKED(10, true); break;
-        case kModeF + 11: EP_PACKED(11, true); break;
-        case kModeTwo:
-        case kModeTwoPair: {
-            const bool pair = g.mode == kModeTwoPair;
-            const uint32_t desc2 = smem_u32(smem + kOffDesc2);
-            if (pair)
-                decode_tiles<DT>(p.tiles, p.tix, p.scales, p.out,
-                                 TwoLut<true>{lut_s, g.b, g.M - 1u, g.M, desc2, s_A}, tc, rg, tl, first_i);
-            else
-                decode_tiles<DT>(p.tiles, p.tix, p.scales, p.out,
-                                 TwoLut<false>{lut_s, g.b, g.M - 1u, 2u * g.M, desc2, s_A}, tc, rg, tl, first_i);
-            break;
-        }
-        default: {
-            CoarseLut cl;
-            cl.lut_s = lut_s;
-            cl.b = g.b;
-            cl.mmask = g.M - 1;
-            cl.sh = g.b - g.k;
-            cl.nb_shift = g.k;
-            cl.fq = fq;
-            cl.s_min = s_min;
-            cl.s_A = s_A;
-            cl.s_off = s_off;
-            decode_tiles<DT>(p.tiles, p.tix, p.scales, p.out, cl, tc, rg, tl, first_i);
-        }
-    }
-#undef EP_PACKED
+    const uint32_t desc2 = smem_u32(smem + kOffDesc2);
+    run_decode<DT, RAGGED>(p, g, lut_s, fq, s_min, s_A, s_off, desc2, tc, rg, tl, first_i);
 }
 
 // ------------------------------------------------------------- host side
@@ -1077,7 +1122,11 @@ std::mutex g_mu;
 
 template <int DT>
 cudaError_t set_decode_attr() {
-    return cudaFuncSetAttribute(decode_kernel<DT>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+    cudaError_t e = cudaFuncSetAttribute(decode_kernel<DT, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         kSmemBytes);
+    if (e == cudaSuccess)
+        e = cudaFuncSetAttribute(decode_kernel<DT, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+    return e;
 }
 
 cudaError_t dev_setup(int dev, int dt, DevState*& ds) {
@@ -1127,7 +1176,8 @@ cudaError_t launch_decode(const Params& prm, cudaStream_t st, int num_sms) {
     attr[0].val.cooperative = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, decode_kernel<DT>, prm);
+    return (prm.cols & 7) ? cudaLaunchKernelEx(&cfg, decode_kernel<DT, true>, prm)
+                          : cudaLaunchKernelEx(&cfg, decode_kernel<DT, false>, prm);
 }
 
 }  // namespace
@@ -1141,9 +1191,8 @@ ep_status ep_decode_tensor(void* stream, const uint16_t* tiles, const uint32_t* 
     using namespace ep;
     if (!tiles || !tile_index || !freq_tables || !row_scales || !out) return EP_EINVAL;
     if (rows <= 0 || cols <= 0) return EP_EINVAL;
-    if (cols % 8) return EP_EUNSUPPORTED;
     if ((int)out_dtype < EP_BF16 || (int)out_dtype > EP_UINT8) return EP_EUNSUPPORTED;
-    const int64_t nvec = rows * (cols / 8);
+    const int64_t nvec = rows * ((cols + 7) / 8);
     if (nvec >= (1ll << 31) || rows >= (1ll << 31)) return EP_EINVAL;
     auto misaligned = [](const void* q, uintptr_t a) { return (reinterpret_cast<uintptr_t>(q) & (a - 1)) != 0; };
     if (misaligned(tiles, 16) || misaligned(freq_tables, 16) || misaligned(tile_index, 4) ||
@@ -1283,10 +1332,9 @@ extern "C" ep_status ep_decode_tensor_noalloc(void* stream, const uint16_t* tile
     using namespace ep;
     if (!tiles || !tile_index || !freq_tables || !row_scales || !out) return EP_EINVAL;
     if (rows <= 0 || cols <= 0) return EP_EINVAL;
-    if (cols % 8) return EP_EUNSUPPORTED;
     if ((int)out_dtype < EP_BF16 || (int)out_dtype > EP_UINT8) return EP_EUNSUPPORTED;
     // the largest tensor this entry point takes: fewer than 2^31 vectors of eight
-    const int64_t nvec = rows * (cols / 8);
+    const int64_t nvec = rows * ((cols + 7) / 8);
     if (nvec >= (1ll << 31) || rows >= (1ll << 31)) return EP_EINVAL;
     auto misaligned = [](const void* q, uintptr_t a) { return (reinterpret_cast<uintptr_t>(q) & (a - 1)) != 0; };
     if (misaligned(tiles, 16) || misaligned(freq_tables, 16) || misaligned(tile_index, 4) ||

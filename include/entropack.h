@@ -27,8 +27,9 @@
  *                Table 0 codes the coset bit c; table 1 + 2(k-1) + c codes field
  *                k (z1..z7, then m) of a vector in coset c (App. A.3).
  *   row_scales   float32[rows]: reconstruction scale of each row.
- * Vector g (8 consecutive weights of a row, g = row*cols/8 + col/8) lies in tile
- * g / V, on lane (g mod V) mod 32, round (g mod V) / 32 (the lane interleave).
+ * Vector g (8 consecutive weights of a row, g = row*nq + col/8, nq = ceil(cols/8):
+ * a partial last vector of a row is padded with zeros) lies in tile g / V, on
+ * lane (g mod V) mod 32, round (g mod V) / 32 (the lane interleave).
  */
 #ifndef ENTROPACK_H
 #define ENTROPACK_H
@@ -56,7 +57,7 @@ typedef enum {
 typedef enum {
     EP_OK = 0,
     EP_EINVAL = 1,        /* a null pointer, a bad size, a misaligned buffer */
-    EP_EUNSUPPORTED = 2,  /* cols % 8 != 0, an unknown dtype, a format variant the GPU does not decode */
+    EP_EUNSUPPORTED = 2,  /* an unknown dtype, a format variant the GPU does not decode */
     EP_EALPHABET = 3,     /* the packer could not fit the alphabets (should not happen) */
     EP_ECUDA = 4,         /* a CUDA runtime error at launch */
     EP_ECORRUPT = 5,      /* the device found an inconsistent stream or table header */
@@ -106,7 +107,9 @@ typedef struct {
  * interleaved rANS (§3.6, App. C.3).  Runs on the host with num_threads threads.
  * opts may be NULL.  On EP_OK *out holds a new blob (free with ep_free_blob).
  * Errors: EP_EINVAL (null W/out, rows or cols <= 0, target_bpp <= 0, b out of
- * [9, 15]), EP_EUNSUPPORTED (cols % 8 != 0), EP_EALPHABET, EP_ENOMEM.
+ * [9, 15]), EP_EALPHABET, EP_ENOMEM.  A width that is not a multiple of 8 pads every
+ * row with zeros to whole vectors (the normaliser, refit and rate use the real
+ * entries only); the decoder drops the padding.
  */
 ep_status ep_encode_tensor(const float* W, int64_t rows, int64_t cols, double target_bpp,
                            const ep_encode_opts* opts, ep_blob** out);
@@ -127,7 +130,9 @@ void ep_free_blob(ep_blob* blob);
  *   row_scales   device, float32[rows].
  *   rows, cols   the matrix shape; must match the header.
  *   out_dtype    one of ep_dtype.
- *   out          device, rows*cols elements of out_dtype, row-major, 16-byte aligned.
+ *   out          device, rows*cols elements of out_dtype, row-major, 16-byte aligned
+ *                (the padding of rows whose width is not a multiple of 8 is not
+ *                written; such rows are written element by element).
  * All buffers belong to the caller.  The library keeps one 128 KB workspace
  * per device (allocated with cudaMalloc and zeroed on the first call on that
  * device, so make the first call before any stream capture); every CTA writes

@@ -52,8 +52,8 @@ def test_decode_rejects_bad_arguments_on_host(lib):
         a[i] = None
         assert lib.ep_decode_tensor(*a) == EINVAL
     a = list(args)
-    a[6] = 60                   # cols % 8 != 0
-    assert lib.ep_decode_tensor(*a) == EUNSUP
+    a[6] = -8                   # cols <= 0
+    assert lib.ep_decode_tensor(*a) == EINVAL
     for dt in (7, 9, -1):       # unknown dtypes (EP_UINT8 = 6 is the last one)
         a = list(args)
         a[7] = dt

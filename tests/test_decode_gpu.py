@@ -74,6 +74,16 @@ def test_shapes(rows, cols, V):
     _check(as_lib_blob(ob), [ep.BF16, ep.FP32, ep.LATTICE_I32], f"{rows}x{cols} V={V}")
 
 
+@pytest.mark.parametrize("rows,cols,V", [(3, 5, 2), (40, 60, 32), (17, 1001, 100), (9, 4097, 455), (300, 1, 33),
+                                         (64, 1020, 1820)])
+def test_widths_not_a_multiple_of_8(rows, cols, V):
+    """Rows padded to whole vectors: the decoder writes the real entries element by element."""
+    rng = np.random.default_rng(rows * cols + V)
+    W = (rng.standard_t(5, (rows, cols)) * 0.02).astype(np.float32)
+    ob = oracle.encode(W, 5.0, tile_vectors=V)
+    _check(as_lib_blob(ob), ALL_DT, f"{rows}x{cols} V={V}")
+
+
 def test_one_coset_and_wide_alphabet():
     # every vector in D8 (the c = 1 tables are empty) and a coordinate alphabet of exactly 2^b
     b = 9
