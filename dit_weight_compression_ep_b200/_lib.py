@@ -89,6 +89,10 @@ def lib() -> C.CDLL:
         L.ep_decode_tensor.restype = C.c_int
         L.ep_decode_tensor_noalloc.argtypes = [P, P, P, P, P, C.c_int64, C.c_int64, C.c_int, P]
         L.ep_decode_tensor_noalloc.restype = C.c_int
+        L.ep_decode_prepare.argtypes = [P, P, C.c_int64, C.c_int64, P, C.c_size_t]
+        L.ep_decode_prepare.restype = C.c_int
+        L.ep_decode_tensor_prepared.argtypes = [P, P, P, P, P, P, C.c_size_t, C.c_int64, C.c_int64, C.c_int, P]
+        L.ep_decode_tensor_prepared.restype = C.c_int
         L.ep_decode_status.argtypes = [P]
         L.ep_decode_status.restype = C.c_int
         L.ep_status_string.argtypes = [C.c_int]
@@ -97,8 +101,10 @@ def lib() -> C.CDLL:
     return _lib
 
 
-EXPORTED = ("ep_encode_tensor", "ep_free_blob", "ep_decode_tensor", "ep_decode_tensor_noalloc", "ep_decode_status",
-            "ep_status_string")
+EXPORTED = ("ep_encode_tensor", "ep_free_blob", "ep_decode_tensor", "ep_decode_tensor_noalloc", "ep_decode_prepare",
+            "ep_decode_tensor_prepared", "ep_decode_status", "ep_status_string")
+
+LUT_BYTES = 131104  # EP_LUT_BYTES: a prepared decode table
 
 
 @dataclass
@@ -219,6 +225,37 @@ def decode_tensor_noalloc(db: DeviceBlob, out_dtype: int = BF16, out=None, strea
                                         int(out_dtype), out.data_ptr())
     if rc:
         raise EntroPackError(rc, "ep_decode_tensor_noalloc")
+    return out
+
+
+def prepare_lut(db: DeviceBlob, lut=None, stream=None):
+    """ep_decode_prepare: build the tensor's decode lookup table once into a LUT_BYTES uint8
+    device buffer (allocated here when `lut` is None); returns the buffer."""
+    import torch
+
+    if lut is None:
+        lut = torch.empty(LUT_BYTES, dtype=torch.uint8, device=db.payload.device)
+    st = stream if stream is not None else torch.cuda.current_stream(db.payload.device)
+    rc = lib().ep_decode_prepare(C.c_void_p(st.cuda_stream), db.freq_tables.data_ptr(), db.rows, db.cols,
+                                 lut.data_ptr(), lut.numel() * lut.element_size())
+    if rc:
+        raise EntroPackError(rc, "ep_decode_prepare")
+    return lut
+
+
+def decode_tensor_prepared(db: DeviceBlob, lut, out_dtype: int = BF16, out=None, stream=None):
+    """ep_decode_tensor_prepared: the decode with a table prepare_lut built from this tensor."""
+    import torch
+
+    if out is None:
+        out = torch.empty((db.rows, db.cols), dtype=_torch_dtype(out_dtype), device=db.payload.device)
+    st = stream if stream is not None else torch.cuda.current_stream(db.payload.device)
+    rc = lib().ep_decode_tensor_prepared(C.c_void_p(st.cuda_stream), db.payload.data_ptr(),
+                                         db.tile_index.data_ptr(), db.freq_tables.data_ptr(),
+                                         db.row_scales.data_ptr(), lut.data_ptr(), lut.numel() * lut.element_size(),
+                                         db.rows, db.cols, int(out_dtype), out.data_ptr())
+    if rc:
+        raise EntroPackError(rc, "ep_decode_tensor_prepared")
     return out
 
 

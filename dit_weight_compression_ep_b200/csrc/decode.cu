@@ -89,6 +89,13 @@ constexpr uint32_t kTwoRecMax = 32 * 1024;  // u16 records: sum over tables 1..1
 constexpr int kWsCountOffset = kLutBytes;
 constexpr int kWsBytes = kLutBytes + 32;
 constexpr uint32_t kGridSpins = 1u << 22;  // bound on the grid-barrier polls
+// A prepared table (ep_decode_prepare): the image, then a trailer at kLutBytes of
+// {magic, bad tables, fingerprint lo, fingerprint hi, image bytes}; same size as the workspace.
+constexpr uint32_t kLutMagic = 0x5450454Cu;
+static_assert(kWsBytes == EP_LUT_BYTES, "prepared table size");
+// ep_decode_prepare's kernel: the scan scratch (A + 1 <= 2^15 + 1 u16), then the descriptors
+constexpr int kPrepOffDesc = 65536 + 128;
+constexpr int kPrepSmemBytes = kPrepOffDesc + 3 * 32 * 4;
 
 // status bits
 constexpr unsigned kStCorrupt = 1u;      // payload / state / offset inconsistent
@@ -250,6 +257,21 @@ __device__ unsigned parse_header(const uint8_t* ft, int64_t rows, int64_t cols, 
     else
         g.image_bytes = packed ? 16u * g.M * 4u : 16u * (1u << g.k) * 8u;
     return 0;
+}
+
+// A fingerprint of what fixes the LUT image's layout: b, the LUT format and every table's
+// {min, A}.  Warp-uniform; a SplitMix64 finaliser per lane, summed in two 32-bit halves.
+__device__ __forceinline__ uint64_t mix64(uint64_t z) {
+    z = (z ^ (z >> 30)) * 0xBF58476D1CE4E5B9ull;
+    z = (z ^ (z >> 27)) * 0x94D049BB133111EBull;
+    return z ^ (z >> 31);
+}
+__device__ __forceinline__ uint2 table_fingerprint(const Geo& g, int mn, uint32_t A) {
+    const int lane = threadIdx.x & 31;
+    uint64_t v = 0;
+    if (lane < kTables) v = mix64(((uint64_t)lane << 56) ^ ((uint64_t)(uint32_t)mn << 20) ^ (uint64_t)A);
+    else if (lane == 31) v = mix64((0xE8ull << 56) ^ ((uint64_t)g.b << 8) ^ (uint64_t)(uint32_t)g.mode);
+    return make_uint2(__reduce_add_sync(kFull, (uint32_t)v), __reduce_add_sync(kFull, (uint32_t)(v >> 32)));
 }
 
 // ------------------------------------------------------- LUT image slice
@@ -898,9 +920,10 @@ struct Params {
     const uint8_t* ft;
     const float* scales;
     void* out;
-    uint8_t* ws;  // LUT image + grid-barrier state
+    uint8_t* ws;  // LUT image + grid-barrier state, or a prepared table (read only)
     int64_t rows, cols;
-    uint32_t one;  // 1, set by the host (see TileCtx)
+    uint32_t one;       // 1, set by the host (see TileCtx)
+    uint32_t prepared;  // ws holds a table ep_decode_prepare wrote: no build, no grid barrier
 };
 
 // The decode loop for the stream's LUT format.  Rows padded to whole vectors (a width
@@ -973,7 +996,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(Params p) {
     // in flight together.
     uint32_t fr[kPre];
     int t_pre = 0;
-    if (gridDim.x >= 16 && g.mode != kModeCoarse) {
+    if (gridDim.x >= 16 && g.mode != kModeCoarse && !p.prepared) {
         const int t = 1 + (int)(blockIdx.x * 16u / gridDim.x);
         const uint32_t At = __shfl_sync(kFull, lane_A, t);
         const uint32_t offt = __reduce_add_sync(kFull, lane < t ? lane_A : 0u);
@@ -1005,6 +1028,18 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(Params p) {
         if (t >= 1 && t < kTables)
             reinterpret_cast<uint2*>(smem + kOffDesc2)[t - 1] =
                 make_uint2(smem_u32(smem + kOffLut + kTwoRec) + 2u * (incl - A - A0 + (uint32_t)(t - 1)), (uint32_t)lane_mn);
+    }
+    // a prepared table: its trailer's loads go out now, with the prologue's other loads
+    uint2 fp = make_uint2(0u, 0u);
+    uint4 tr4 = make_uint4(0u, 0u, 0u, 0u);
+    uint32_t tr_ib = 0;
+    if (p.prepared && threadIdx.x < 32) {
+        fp = table_fingerprint(g, lane_mn, lane_A);
+        if (threadIdx.x == 0) {
+            const uint32_t* tr = reinterpret_cast<const uint32_t*>(p.ws + kLutBytes);
+            tr4 = __ldg(reinterpret_cast<const uint4*>(tr));
+            tr_ib = __ldg(tr + 4);
+        }
     }
     TileCtx tc;
     tc.nvec = g.nvec;
@@ -1046,6 +1081,14 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(Params p) {
         mbar_init(rg.bar_s + 8, 1);
         if (warp == 0) mbar_init(lut_bar, 1);
         fence_barrier_init();
+        // a prepared image comes straight into shared memory, ahead of the payload's first chunks
+        // (the copy stays inside the table buffer whatever its trailer holds; checked below)
+        if (warp == 0 && p.prepared && blockIdx.x < g.T) {
+            mbar_arrive_expect_tx(lut_bar, g.image_bytes);
+            for (uint32_t o = 0; o < g.image_bytes; o += 16384u)
+                bulk_g2s(smem_u32(smem + kOffLut) + o, p.ws + o,
+                         g.image_bytes - o < 16384u ? g.image_bytes - o : 16384u, lut_bar);
+        }
     }
     __syncthreads();  // barrier initialisation and descriptors visible to every warp
 
@@ -1054,46 +1097,56 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(Params p) {
     tc.df = tc.f1c - tc.f0c;
     tc.nf0 = 0u - tc.f0c;
 
-    // ---- a2: this CTA's slice of the LUT image, a grid-wide arrival, the image into shared memory
-    // A table that does not sum to 2^b gets zero entries (decoding with them stays in
-    // bounds) and raises the status word; the decode goes on, its output unspecified.
-    const bool bad = build_lut_slice(g, fq, s_min, s_A, s_off, p.ws, reinterpret_cast<uint16_t*>(smem + kOffLut),
-                                     t_pre, fr);
-    if (bad && threadIdx.x == 0) raise_status(kStHeader);
-    fence_proxy_async_shared();  // the scratch writes before the bulk copy overwrites them
-    __syncthreads();
-    if (threadIdx.x == 0) {
-        __threadfence();  // the CTA's image stores (ordered by the barrier above) before the arrival
-        // the counter grows by G per launch, so the arrival that returns `old` belongs to
-        // the launch that ends at the next multiple of G
-        unsigned long long* arrivals = reinterpret_cast<unsigned long long*>(p.ws + kWsCountOffset);
-        const unsigned long long old = atomicAdd(arrivals, 1ull);
-        // old / G without a 64-bit integer division: a double quotient (old < 2^53), corrected
-        const unsigned long long G = gridDim.x;
-        unsigned long long q = (unsigned long long)((double)old / (double)G);
-        q -= q * G > old ? 1ull : 0ull;
-        q += (q + 1ull) * G <= old ? 1ull : 0ull;
-        const unsigned long long target = (q + 1ull) * G;
-        uint32_t spins = 0;
-        // every CTA of the (cooperative, hence co-resident) grid arrives; bounded wait
-        while (ld_acquire_gpu(arrivals) < target && spins < kGridSpins) {
-            __nanosleep(32);
-            ++spins;
+    if (p.prepared) {
+        // ---- a2 from a prepared table (its copy is in flight): the trailer must carry this
+        // header's layout fingerprint
+        if (threadIdx.x == 0) {
+            s_ok = tr4.x == kLutMagic && tr4.z == fp.x && tr4.w == fp.y && tr_ib == g.image_bytes;
+            if (blockIdx.x == 0 && (!s_ok || tr4.y)) raise_status(kStHeader);
         }
-        s_ok = spins < kGridSpins;
-        if (!s_ok) raise_status(kStTimeout);
-        if (s_ok && blockIdx.x < g.T) {
-            fence_proxy_async_global();  // generic-proxy image stores before the bulk-copy reads
-            mbar_arrive_expect_tx(lut_bar, g.image_bytes);
-            for (uint32_t o = 0; o < g.image_bytes; o += 16384u)
-                bulk_g2s(smem_u32(smem + kOffLut) + o, p.ws + o,
-                         g.image_bytes - o < 16384u ? g.image_bytes - o : 16384u, lut_bar);
+    } else {
+        // ---- a2: this CTA's slice of the LUT image, a grid-wide arrival, the image into shared memory
+        // A table that does not sum to 2^b gets zero entries (decoding with them stays in
+        // bounds) and raises the status word; the decode goes on, its output unspecified.
+        const bool bad = build_lut_slice(g, fq, s_min, s_A, s_off, p.ws, reinterpret_cast<uint16_t*>(smem + kOffLut),
+                                         t_pre, fr);
+        if (bad && threadIdx.x == 0) raise_status(kStHeader);
+        fence_proxy_async_shared();  // the scratch writes before the bulk copy overwrites them
+        __syncthreads();
+        if (threadIdx.x == 0) {
+            __threadfence();  // the CTA's image stores (ordered by the barrier above) before the arrival
+            // the counter grows by G per launch, so the arrival that returns `old` belongs to
+            // the launch that ends at the next multiple of G
+            unsigned long long* arrivals = reinterpret_cast<unsigned long long*>(p.ws + kWsCountOffset);
+            const unsigned long long old = atomicAdd(arrivals, 1ull);
+            // old / G without a 64-bit integer division: a double quotient (old < 2^53), corrected
+            const unsigned long long G = gridDim.x;
+            unsigned long long q = (unsigned long long)((double)old / (double)G);
+            q -= q * G > old ? 1ull : 0ull;
+            q += (q + 1ull) * G <= old ? 1ull : 0ull;
+            const unsigned long long target = (q + 1ull) * G;
+            uint32_t spins = 0;
+            // every CTA of the (cooperative, hence co-resident) grid arrives; bounded wait
+            while (ld_acquire_gpu(arrivals) < target && spins < kGridSpins) {
+                __nanosleep(32);
+                ++spins;
+            }
+            s_ok = spins < kGridSpins;
+            if (!s_ok) raise_status(kStTimeout);
+            if (s_ok && blockIdx.x < g.T) {
+                fence_proxy_async_global();  // generic-proxy image stores before the bulk-copy reads
+                mbar_arrive_expect_tx(lut_bar, g.image_bytes);
+                for (uint32_t o = 0; o < g.image_bytes; o += 16384u)
+                    bulk_g2s(smem_u32(smem + kOffLut) + o, p.ws + o,
+                             g.image_bytes - o < 16384u ? g.image_bytes - o : 16384u, lut_bar);
+            }
         }
     }
     __syncthreads();
     if (blockIdx.x >= g.T) return;  // no tile for this CTA
     bool lut_ok = s_ok != 0;
-    if (lut_ok && !mbar_wait(lut_bar, 0)) {
+    // a prepared table's copy is in flight even when its trailer did not match
+    if ((lut_ok || p.prepared) && !mbar_wait(lut_bar, 0)) {
         lut_ok = false;
         raise_status(kStTimeout);
     }
@@ -1109,11 +1162,62 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(Params p) {
     run_decode<DT, RAGGED>(p, g, lut_s, fq, s_min, s_A, s_off, desc2, tc, rg, tl, first_i);
 }
 
+// ep_decode_prepare's kernel: a2 without the decode.  Every CTA builds its slice of the image
+// into the caller's table exactly as the decode kernel builds it into the workspace; CTA 0
+// writes the trailer's magic, fingerprint and image size (the host zeroed the trailer), a CTA
+// that finds a table not summing to 2^b sets its bad word.
+__global__ void __launch_bounds__(kThreads, 1) lut_prepare_kernel(const uint8_t* ft, int64_t rows, int64_t cols,
+                                                                   uint8_t* lut) {
+    extern __shared__ __align__(1024) uint8_t smem[];
+    int* s_min = reinterpret_cast<int*>(smem + kPrepOffDesc);
+    uint32_t* s_A = reinterpret_cast<uint32_t*>(smem + kPrepOffDesc + 128);
+    uint32_t* s_off = reinterpret_cast<uint32_t*>(smem + kPrepOffDesc + 256);
+    Geo g;
+    int lane_mn;
+    uint32_t lane_A;
+    const unsigned hs = parse_header(ft, rows, cols, g, lane_mn, lane_A);
+    if (hs) {
+        if (threadIdx.x == 0 && blockIdx.x == 0) raise_status(hs);
+        return;
+    }
+    const uint16_t* fq = reinterpret_cast<const uint16_t*>(ft + table_header_bytes(kTables));
+    if (threadIdx.x < 32) {
+        const int t = threadIdx.x;
+        uint32_t incl = lane_A;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const uint32_t v = __shfl_up_sync(kFull, incl, o);
+            if (t >= o) incl += v;
+        }
+        if (t < kTables) {
+            s_min[t] = lane_mn;
+            s_A[t] = lane_A;
+            s_off[t] = incl - lane_A;
+        }
+        const uint2 fp = table_fingerprint(g, lane_mn, lane_A);
+        if (t == 0 && blockIdx.x == 0) {
+            uint32_t* tr = reinterpret_cast<uint32_t*>(lut + kLutBytes);
+            tr[0] = kLutMagic;
+            tr[2] = fp.x;
+            tr[3] = fp.y;
+            tr[4] = g.image_bytes;
+        }
+    }
+    __syncthreads();
+    uint32_t fr[kPre] = {};
+    const bool bad = build_lut_slice(g, fq, s_min, s_A, s_off, lut, reinterpret_cast<uint16_t*>(smem), 0, fr);
+    if (bad && threadIdx.x == 0) {
+        raise_status(kStHeader);
+        atomicOr(reinterpret_cast<unsigned*>(lut + kLutBytes) + 1, 1u);
+    }
+}
+
 // ------------------------------------------------------------- host side
 
 struct DevState {
     int num_sms = 0;
     bool attr_done[8] = {};
+    bool prep_attr_done = false;
     uint8_t* ws = nullptr;         // the LUT workspace of this device
     cudaEvent_t ws_free = nullptr;  // recorded after every decode that used it
 };
@@ -1129,7 +1233,7 @@ cudaError_t set_decode_attr() {
     return e;
 }
 
-cudaError_t dev_setup(int dev, int dt, DevState*& ds) {
+cudaError_t dev_setup(int dev, int dt, DevState*& ds, bool need_ws = true) {
     std::lock_guard<std::mutex> lk(g_mu);
     ds = &g_dev[dev];
     cudaError_t e;
@@ -1137,7 +1241,7 @@ cudaError_t dev_setup(int dev, int dt, DevState*& ds) {
         e = cudaDeviceGetAttribute(&ds->num_sms, cudaDevAttrMultiProcessorCount, dev);
         if (e != cudaSuccess) return e;
     }
-    if (!ds->ws) {
+    if (need_ws && !ds->ws) {
         // one workspace per device, zeroed once; the grid barrier in it resets itself
         void* w = nullptr;
         e = cudaMalloc(&w, kWsBytes);
@@ -1167,7 +1271,7 @@ cudaError_t dev_setup(int dev, int dt, DevState*& ds) {
 template <int DT>
 cudaError_t launch_decode(const Params& prm, cudaStream_t st, int num_sms) {
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3((unsigned)num_sms);  // one CTA per SM; all co-resident (cooperative launch)
+    cfg.gridDim = dim3((unsigned)num_sms);  // one CTA per SM
     cfg.blockDim = dim3(kThreads);
     cfg.dynamicSmemBytes = kSmemBytes;
     cfg.stream = st;
@@ -1175,9 +1279,39 @@ cudaError_t launch_decode(const Params& prm, cudaStream_t st, int num_sms) {
     attr[0].id = cudaLaunchAttributeCooperative;
     attr[0].val.cooperative = 1;
     cfg.attrs = attr;
-    cfg.numAttrs = 1;
+    // the grid barrier needs every CTA co-resident (a cooperative launch); a prepared table needs none
+    cfg.numAttrs = prm.prepared ? 0 : 1;
     return (prm.cols & 7) ? cudaLaunchKernelEx(&cfg, decode_kernel<DT, true>, prm)
                           : cudaLaunchKernelEx(&cfg, decode_kernel<DT, false>, prm);
+}
+
+cudaError_t launch_any(ep_dtype dt, const Params& prm, cudaStream_t st, int num_sms) {
+    switch (dt) {
+        case EP_BF16: return launch_decode<EP_BF16>(prm, st, num_sms);
+        case EP_FP16: return launch_decode<EP_FP16>(prm, st, num_sms);
+        case EP_FP8_E4M3: return launch_decode<EP_FP8_E4M3>(prm, st, num_sms);
+        case EP_INT8: return launch_decode<EP_INT8>(prm, st, num_sms);
+        case EP_UINT8: return launch_decode<EP_UINT8>(prm, st, num_sms);
+        case EP_FP32: return launch_decode<EP_FP32>(prm, st, num_sms);
+        default: return launch_decode<EP_LATTICE_I32>(prm, st, num_sms);
+    }
+}
+
+bool misaligned(const void* q, uintptr_t a) { return (reinterpret_cast<uintptr_t>(q) & (a - 1)) != 0; }
+
+// the host checks every decode entry point shares
+ep_status check_decode_args(const uint16_t* tiles, const uint32_t* tile_index, const uint8_t* freq_tables,
+                            const float* row_scales, int64_t rows, int64_t cols, ep_dtype out_dtype, void* out) {
+    if (!tiles || !tile_index || !freq_tables || !row_scales || !out) return EP_EINVAL;
+    if (rows <= 0 || cols <= 0) return EP_EINVAL;
+    if ((int)out_dtype < EP_BF16 || (int)out_dtype > EP_UINT8) return EP_EUNSUPPORTED;
+    // the largest tensor: fewer than 2^31 vectors of eight
+    const int64_t nvec = rows * ((cols + 7) / 8);
+    if (nvec >= (1ll << 31) || rows >= (1ll << 31)) return EP_EINVAL;
+    if (misaligned(tiles, 16) || misaligned(freq_tables, 16) || misaligned(tile_index, 4) ||
+        misaligned(row_scales, 4) || misaligned(out, 16))
+        return EP_EINVAL;
+    return EP_OK;
 }
 
 }  // namespace
@@ -1189,15 +1323,8 @@ ep_status ep_decode_tensor(void* stream, const uint16_t* tiles, const uint32_t* 
                            const uint8_t* freq_tables, const float* row_scales, int64_t rows, int64_t cols,
                            ep_dtype out_dtype, void* out) {
     using namespace ep;
-    if (!tiles || !tile_index || !freq_tables || !row_scales || !out) return EP_EINVAL;
-    if (rows <= 0 || cols <= 0) return EP_EINVAL;
-    if ((int)out_dtype < EP_BF16 || (int)out_dtype > EP_UINT8) return EP_EUNSUPPORTED;
-    const int64_t nvec = rows * ((cols + 7) / 8);
-    if (nvec >= (1ll << 31) || rows >= (1ll << 31)) return EP_EINVAL;
-    auto misaligned = [](const void* q, uintptr_t a) { return (reinterpret_cast<uintptr_t>(q) & (a - 1)) != 0; };
-    if (misaligned(tiles, 16) || misaligned(freq_tables, 16) || misaligned(tile_index, 4) ||
-        misaligned(row_scales, 4) || misaligned(out, 16))
-        return EP_EINVAL;
+    const ep_status as = check_decode_args(tiles, tile_index, freq_tables, row_scales, rows, cols, out_dtype, out);
+    if (as != EP_OK) return as;
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return EP_ECUDA;
     DevState* ds = nullptr;
@@ -1211,19 +1338,58 @@ ep_status ep_decode_tensor(void* stream, const uint16_t* tiles, const uint32_t* 
     const bool capturing = e == cudaSuccess && cap != cudaStreamCaptureStatusNone;
     if (e == cudaSuccess && !capturing) e = cudaStreamWaitEvent(st, ds->ws_free, 0);
     if (e == cudaSuccess) {
-        Params prm{tiles, tile_index, freq_tables, row_scales, out, ds->ws, rows, cols, 1u};
-        switch (out_dtype) {
-            case EP_BF16: e = launch_decode<EP_BF16>(prm, st, ds->num_sms); break;
-            case EP_FP16: e = launch_decode<EP_FP16>(prm, st, ds->num_sms); break;
-            case EP_FP8_E4M3: e = launch_decode<EP_FP8_E4M3>(prm, st, ds->num_sms); break;
-            case EP_INT8: e = launch_decode<EP_INT8>(prm, st, ds->num_sms); break;
-            case EP_UINT8: e = launch_decode<EP_UINT8>(prm, st, ds->num_sms); break;
-            case EP_FP32: e = launch_decode<EP_FP32>(prm, st, ds->num_sms); break;
-            default: e = launch_decode<EP_LATTICE_I32>(prm, st, ds->num_sms); break;
-        }
+        const Params prm{tiles, tile_index, freq_tables, row_scales, out, ds->ws, rows, cols, 1u, 0u};
+        e = launch_any(out_dtype, prm, st, ds->num_sms);
     }
     if (e == cudaSuccess && !capturing) e = cudaEventRecord(ds->ws_free, st);
     return e == cudaSuccess ? EP_OK : EP_ECUDA;
+}
+
+ep_status ep_decode_prepare(void* stream, const uint8_t* freq_tables, int64_t rows, int64_t cols, void* lut,
+                            size_t lut_bytes) {
+    using namespace ep;
+    if (!freq_tables || !lut || lut_bytes < (size_t)EP_LUT_BYTES || rows <= 0 || cols <= 0) return EP_EINVAL;
+    if (misaligned(freq_tables, 16) || misaligned(lut, 16)) return EP_EINVAL;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return EP_ECUDA;
+    DevState* ds = nullptr;
+    if (dev_setup(dev, EP_BF16, ds, false) != cudaSuccess) return EP_ECUDA;
+    {
+        std::lock_guard<std::mutex> lk(g_mu);
+        if (!ds->prep_attr_done) {
+            if (cudaFuncSetAttribute(lut_prepare_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     kPrepSmemBytes) != cudaSuccess)
+                return EP_ECUDA;
+            ds->prep_attr_done = true;
+        }
+    }
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    uint8_t* l = static_cast<uint8_t*>(lut);
+    cudaError_t e = cudaMemsetAsync(l + kLutBytes, 0, EP_LUT_BYTES - kLutBytes, st);
+    if (e == cudaSuccess) {
+        lut_prepare_kernel<<<ds->num_sms, kThreads, kPrepSmemBytes, st>>>(freq_tables, rows, cols, l);
+        e = cudaGetLastError();
+    }
+    return e == cudaSuccess ? EP_OK : EP_ECUDA;
+}
+
+ep_status ep_decode_tensor_prepared(void* stream, const uint16_t* tiles, const uint32_t* tile_index,
+                                    const uint8_t* freq_tables, const float* row_scales, const void* lut,
+                                    size_t lut_bytes, int64_t rows, int64_t cols, ep_dtype out_dtype,
+                                    void* out) {
+    using namespace ep;
+    const ep_status as = check_decode_args(tiles, tile_index, freq_tables, row_scales, rows, cols, out_dtype, out);
+    if (as != EP_OK) return as;
+    if (!lut || lut_bytes < (size_t)EP_LUT_BYTES || misaligned(lut, 16)) return EP_EINVAL;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return EP_ECUDA;
+    DevState* ds = nullptr;
+    if (dev_setup(dev, (int)out_dtype, ds, false) != cudaSuccess) return EP_ECUDA;
+    // the table is only read: no workspace, nothing to order against other decodes
+    const Params prm{tiles, tile_index, freq_tables, row_scales, out,
+                     const_cast<uint8_t*>(static_cast<const uint8_t*>(lut)), rows, cols, 1u, 1u};
+    return launch_any(out_dtype, prm, static_cast<cudaStream_t>(stream), ds->num_sms) == cudaSuccess ? EP_OK
+                                                                                                     : EP_ECUDA;
 }
 
 ep_status ep_decode_status(void* stream) {
@@ -1330,16 +1496,9 @@ extern "C" ep_status ep_decode_tensor_noalloc(void* stream, const uint16_t* tile
                                               const uint8_t* freq_tables, const float* row_scales, int64_t rows,
                                               int64_t cols, ep_dtype out_dtype, void* out) {
     using namespace ep;
-    if (!tiles || !tile_index || !freq_tables || !row_scales || !out) return EP_EINVAL;
-    if (rows <= 0 || cols <= 0) return EP_EINVAL;
-    if ((int)out_dtype < EP_BF16 || (int)out_dtype > EP_UINT8) return EP_EUNSUPPORTED;
     // the largest tensor this entry point takes: fewer than 2^31 vectors of eight
-    const int64_t nvec = rows * ((cols + 7) / 8);
-    if (nvec >= (1ll << 31) || rows >= (1ll << 31)) return EP_EINVAL;
-    auto misaligned = [](const void* q, uintptr_t a) { return (reinterpret_cast<uintptr_t>(q) & (a - 1)) != 0; };
-    if (misaligned(tiles, 16) || misaligned(freq_tables, 16) || misaligned(tile_index, 4) ||
-        misaligned(row_scales, 4) || misaligned(out, 16))
-        return EP_EINVAL;
+    const ep_status as = check_decode_args(tiles, tile_index, freq_tables, row_scales, rows, cols, out_dtype, out);
+    if (as != EP_OK) return as;
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return EP_ECUDA;
     NoAllocState* ns = nullptr;
@@ -1348,16 +1507,8 @@ extern "C" ep_status ep_decode_tensor_noalloc(void* stream, const uint16_t* tile
     // the barrier words must start at zero; the array keeps whatever the last call left
     cudaError_t e = cudaMemsetAsync(ns->scratch + kWsCountOffset, 0, kNoAllocScratchBytes - kWsCountOffset, st);
     if (e == cudaSuccess) {
-        Params prm{tiles, tile_index, freq_tables, row_scales, out, ns->scratch, rows, cols, 1u};
-        switch (out_dtype) {
-            case EP_BF16: e = launch_decode<EP_BF16>(prm, st, ns->num_sms); break;
-            case EP_FP16: e = launch_decode<EP_FP16>(prm, st, ns->num_sms); break;
-            case EP_FP8_E4M3: e = launch_decode<EP_FP8_E4M3>(prm, st, ns->num_sms); break;
-            case EP_INT8: e = launch_decode<EP_INT8>(prm, st, ns->num_sms); break;
-            case EP_UINT8: e = launch_decode<EP_UINT8>(prm, st, ns->num_sms); break;
-            case EP_FP32: e = launch_decode<EP_FP32>(prm, st, ns->num_sms); break;
-            default: e = launch_decode<EP_LATTICE_I32>(prm, st, ns->num_sms); break;
-        }
+        const Params prm{tiles, tile_index, freq_tables, row_scales, out, ns->scratch, rows, cols, 1u, 0u};
+        e = launch_any(out_dtype, prm, st, ns->num_sms);
     }
     return e == cudaSuccess ? EP_OK : EP_ECUDA;
 }

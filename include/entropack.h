@@ -177,6 +177,53 @@ ep_status ep_decode_tensor_noalloc(void* stream, const uint16_t* tiles, const ui
                                    int64_t cols, ep_dtype out_dtype, void* out);
 
 /*
+ * Size in bytes of a prepared decode table: the lookup-table image (128 KiB,
+ * enough for any stream with b <= 15) and a 32-byte trailer.
+ */
+#define EP_LUT_BYTES 131104
+
+/*
+ * ep_decode_prepare -- build a tensor's decode lookup table once, into a
+ * caller buffer that later decodes of the same tensor read instead of building
+ * it again.  The tables map the low b bits of a rANS state to a symbol and its
+ * frequency interval (App. C.3, "Decoder lookup tables": the tables sit in
+ * shared memory or in packed global memory); they depend only on freq_tables,
+ * so a weight that is decoded many times (every denoising step, every prefill)
+ * can keep them beside its compressed bytes.
+ *   stream       cudaStream_t to launch on.
+ *   freq_tables  device, the tensor's table header and frequencies (16-byte aligned).
+ *   rows, cols   the matrix shape; must match the header.
+ *   lut          device, lut_bytes >= EP_LUT_BYTES, 16-byte aligned, owned by the
+ *                caller; written by this call (one memset of the trailer and one
+ *                launch on `stream`), read by ep_decode_tensor_prepared.
+ * Argument errors return at once (EP_EINVAL); launch errors as EP_ECUDA.  An
+ * invalid header or tables that do not sum to 2^b raise the device status word
+ * (ep_decode_status); a decode with that table raises it again.
+ */
+ep_status ep_decode_prepare(void* stream, const uint8_t* freq_tables, int64_t rows, int64_t cols, void* lut,
+                            size_t lut_bytes);
+
+/*
+ * ep_decode_tensor_prepared -- ep_decode_tensor with the lookup table that
+ * ep_decode_prepare built from the same freq_tables.  The arguments, alignment
+ * rules, output and status reporting are those of ep_decode_tensor, plus
+ *   lut, lut_bytes  the prepared table (device, >= EP_LUT_BYTES, 16-byte aligned;
+ *                   read only, so any number of decodes may share it at once).
+ * The call uses no library workspace and no grid-wide barrier: it makes one
+ * ordinary launch on the stream (one CTA per SM), so decodes on different
+ * streams may run at the same time and nothing orders them but their streams.
+ * A table whose layout does not match this tensor's header (b, LUT format, or
+ * any table's minimum or alphabet size), or a buffer ep_decode_prepare did not
+ * write, raises EP_ECORRUPT in the status word and nothing is decoded.  A table
+ * prepared from tables with the same layout but other frequencies is not
+ * detected: the output is then unspecified, and every access stays in bounds.
+ */
+ep_status ep_decode_tensor_prepared(void* stream, const uint16_t* tiles, const uint32_t* tile_index,
+                                    const uint8_t* freq_tables, const float* row_scales, const void* lut,
+                                    size_t lut_bytes, int64_t rows, int64_t cols, ep_dtype out_dtype,
+                                    void* out);
+
+/*
  * ep_decode_status -- synchronise `stream`, read and clear the status word of
  * the current device: EP_OK, EP_ECORRUPT (an inconsistent stream or header),
  * or EP_EUNSUPPORTED (a header variant the GPU decoder does not handle).

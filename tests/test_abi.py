@@ -69,6 +69,34 @@ def test_decode_rejects_bad_arguments_on_host(lib):
     assert lib.ep_decode_tensor(*a) == EINVAL
 
 
+def test_prepared_decode_rejects_bad_arguments_on_host(lib):
+    """Every case below is refused by the host checks, before any CUDA call."""
+    good = C.c_void_p(0x10000)
+    EINVAL, EUNSUP = ep._lib.STATUS_CODES["EP_EINVAL"], ep._lib.STATUS_CODES["EP_EUNSUPPORTED"]
+    n = ep.LUT_BYTES
+    prep = [None, good, 64, 64, good, n]
+    for i, bad in ((1, None), (4, None), (4, C.c_void_p(0x10008)), (1, C.c_void_p(0x10004)), (5, n - 1), (5, 0),
+                   (2, 0), (3, -8)):
+        a = list(prep)
+        a[i] = bad
+        assert lib.ep_decode_prepare(*a) == EINVAL, (i, bad)
+    dec = [None, good, good, good, good, good, n, 64, 64, ep.BF16, good]
+    for i, bad in ((1, None), (2, None), (3, None), (4, None), (5, None), (10, None), (5, C.c_void_p(0x10008)),
+                   (6, n - 1), (7, 0), (8, -8), (10, C.c_void_p(0x10004)), (1, C.c_void_p(0x10008))):
+        a = list(dec)
+        a[i] = bad
+        assert lib.ep_decode_tensor_prepared(*a) == EINVAL, (i, bad)
+    a = list(dec)
+    a[9] = 7
+    assert lib.ep_decode_tensor_prepared(*a) == EUNSUP
+
+
+def test_lut_bytes_matches_the_header():
+    src = open(os.path.join(ROOT, "include", "entropack.h")).read()
+    m = re.search(r"#define\s+EP_LUT_BYTES\s+(\d+)", src)
+    assert m and int(m.group(1)) == ep.LUT_BYTES == 128 * 1024 + 32
+
+
 def test_encode_rejects_bad_arguments(lib):
     W = np.zeros((4, 16), np.float32)
     assert ep.encode_tensor(np.ones((4, 12), np.float32), 4.0).cols == 12  # rows padded to whole vectors
