@@ -602,6 +602,118 @@ def run_sweep(args):
           f"= {100 * tot['decode_over_matmul']:.1f} %; oracle: {oc}; HBM peak {peak} GB/s ({peak_kind})")
 
 
+def run_dit(args):
+    """The whole 30-block DiT linear stack (150 layers at the per-layer rate allocation) decoded to
+    bf16 three ways: one ep_decode_tensor per layer, one ep_decode_tensor_prepared per layer, and
+    one ep_decode_batch per block (the block's five tensors in one launch); then the block-by-block
+    sequence a denoising step runs (decode the block's weights, then its five bf16 matmuls with
+    4096 tokens) against the matmuls alone.  Decode speed depends on a layer's shape and rate, not
+    on its seed, so the 25 (kind, rate) streams are encoded once and every block uses its own
+    combination of them.  Each figure: min and median of 5 timed passes of the whole stack (CUDA
+    events around the pass, one stream, eager launches), after a warm-up pass."""
+    import torch
+
+    import dit_weight_compression_ep_b200 as ep
+    from dit_weight_compression_ep_b200 import build, synth
+
+    build.build()
+    peak, peak_kind = _peaks()
+    dev = torch.device("cuda", 0)
+    alloc = synth.dit_stack_bpp()
+    kinds = list(synth.DIT_KINDS)
+    nblocks = 1 + max(b for b, _ in alloc)
+    streams = {}
+    for kind in kinds:
+        Wk = synth.generate(synth.dit_stack_layer(0, kind))
+        for bpp in sorted({alloc[(b, kind)] for b in range(nblocks)}):
+            blob = ep.encode_tensor(Wk, bpp)
+            db = ep.DeviceBlob(blob, dev)
+            streams[(kind, bpp)] = (blob, db, ep.prepare_lut(db))
+        del Wk
+    outs = {k: torch.empty(synth.DIT_KINDS[k], dtype=torch.bfloat16, device=dev) for k in kinds}
+    blocks = [[(k, alloc[(b, k)]) for k in kinds] for b in range(nblocks)]
+    batches = [ep.DecodeBatch([(streams[kb][1], streams[kb][2], outs[kb[0]]) for kb in blk], ep.BF16)
+               for blk in blocks]
+    numel = sum(streams[kb][0].rows * streams[kb][0].cols for blk in blocks for kb in blk)
+    nbytes = sum(streams[kb][0].stored_device_bytes() + 2 * streams[kb][0].rows * streams[kb][0].cols
+                 for blk in blocks for kb in blk)
+    st = torch.cuda.current_stream(dev)
+    X = {c: torch.randn(4096, c, dtype=torch.bfloat16, device=dev) for c in {synth.DIT_KINDS[k][1] for k in kinds}}
+
+    def per_call():
+        for blk in blocks:
+            for kb in blk:
+                ep.decode_tensor(streams[kb][1], ep.BF16, out=outs[kb[0]], stream=st)
+
+    def prepared():
+        for blk in blocks:
+            for kb in blk:
+                ep.decode_tensor_prepared(streams[kb][1], streams[kb][2], ep.BF16, out=outs[kb[0]], stream=st)
+
+    def batched():
+        for bt in batches:
+            bt.run(stream=st)
+
+    def matmuls_of(blk):
+        for k, _ in blk:
+            torch.matmul(X[synth.DIT_KINDS[k][1]], outs[k].t())
+
+    def matmuls_only():
+        for blk in blocks:
+            matmuls_of(blk)
+
+    def step_batched():
+        for bt, blk in zip(batches, blocks):
+            bt.run(stream=st)
+            matmuls_of(blk)
+
+    def step_per_call():
+        for blk in blocks:
+            for kb in blk:
+                ep.decode_tensor(streams[kb][1], ep.BF16, out=outs[kb[0]], stream=st)
+            matmuls_of(blk)
+
+    def timed(fn, passes=5):
+        fn()
+        torch.cuda.synchronize(dev)
+        ts = []
+        for _ in range(passes):
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(st)
+            fn()
+            b.record(st)
+            torch.cuda.synchronize(dev)
+            ts.append(a.elapsed_time(b))
+        if ep.decode_status(st) != 0:
+            raise RuntimeError("decode reported a corrupt stream")
+        return round(min(ts), 3), round(statistics.median(ts), 3)
+
+    # the three decodes give the same bits
+    batched()
+    ref = {k: o.clone() for k, o in outs.items()}
+    prepared()
+    torch.cuda.synchronize(dev)
+    if ep.decode_status(st) != 0 or not all(torch.equal(ref[k].view(torch.int16), outs[k].view(torch.int16))
+                                            for k in kinds):
+        raise RuntimeError("batched and prepared decodes differ")
+    res = {"case": f"DiT linear stack, {nblocks} blocks x {len(kinds)} layers, per-layer rates {synth.DIT_BPP_CHOICES}",
+           "weights": numel, "algorithmic_bytes": nbytes, "hbm_peak_gbs": peak, "peak_kind": peak_kind}
+    for name, fn in (("per_layer_decode", per_call), ("per_layer_prepared", prepared), ("block_batches", batched),
+                     ("matmuls_only_4096", matmuls_only), ("step_block_batches_then_matmuls", step_batched),
+                     ("step_per_layer_decode_then_matmuls", step_per_call)):
+        tmin, tmed = timed(fn)
+        res[name + "_ms"] = [tmin, tmed]
+        print(json.dumps({name: [tmin, tmed]}), flush=True)
+    for name in ("per_layer_decode", "per_layer_prepared", "block_batches"):
+        t = res[name + "_ms"][0] * 1e-3
+        res[name + "_gweights_s"] = round(numel / t / 1e9, 1)
+        res[name + "_hbm_frac"] = round(nbytes / t / 1e9 / peak, 4)
+    mm = res["matmuls_only_4096_ms"][0]
+    res["step_overhead_block_batches"] = round(res["step_block_batches_then_matmuls_ms"][0] / mm - 1, 4)
+    res["step_overhead_per_layer"] = round(res["step_per_layer_decode_then_matmuls_ms"][0] / mm - 1, 4)
+    print(json.dumps(res), flush=True)
+
+
 def run_linear(args):
     """A linear layer whose weight is stored compressed: decode it with the library, then the
     library GEMM (cuBLAS through torch), against the same GEMM with the weight resident
@@ -694,6 +806,7 @@ def main():
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--sweep", action="store_true", help="every workload's decode throughput (one GPU)")
     ap.add_argument("--linear", action="store_true", help="decode-then-GEMM against a resident weight (one GPU)")
+    ap.add_argument("--dit", action="store_true", help="the whole DiT stack: per layer, prepared, block batches")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
@@ -706,6 +819,9 @@ def main():
         return
     if args.linear:
         run_linear(args)
+        return
+    if args.dit:
+        run_dit(args)
         return
     if args.impl == "reference":
         if rank != 0:

@@ -7,5 +7,5 @@ Importing the package does not load the library; the first call does, and it
 raises if the library has not been built.
 """
 from ._lib import (BF16, FP16, FP8_E4M3, INT8, FP32, LATTICE_I32, UINT8, Blob, DeviceBlob, EntroPackError,  # noqa: F401
-                   LUT_BYTES, check_status, decode_status, decode_tensor, decode_tensor_prepared, encode_tensor, lib,
-                   prepare_lut)
+                   LUT_BYTES, DecodeBatch, batch_apportion, check_status, decode_status, decode_tensor,
+                   decode_tensor_prepared, encode_tensor, lib, prepare_lut)

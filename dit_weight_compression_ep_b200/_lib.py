@@ -48,6 +48,22 @@ class _Opts(C.Structure):
     ]
 
 
+class _BatchItem(C.Structure):
+    _fields_ = [
+        ("tiles", C.c_void_p),
+        ("tile_index", C.c_void_p),
+        ("freq_tables", C.c_void_p),
+        ("row_scales", C.c_void_p),
+        ("lut", C.c_void_p),
+        ("rows", C.c_int64),
+        ("cols", C.c_int64),
+        ("ntiles", C.c_int64),
+        ("tile_vectors", C.c_int64),
+        ("prob_bits", C.c_int),
+        ("out", C.c_void_p),
+    ]
+
+
 class _Blob(C.Structure):
     _fields_ = [
         ("rows", C.c_int64),
@@ -93,6 +109,15 @@ def lib() -> C.CDLL:
         L.ep_decode_prepare.restype = C.c_int
         L.ep_decode_tensor_prepared.argtypes = [P, P, P, P, P, P, C.c_size_t, C.c_int64, C.c_int64, C.c_int, P]
         L.ep_decode_tensor_prepared.restype = C.c_int
+        L.ep_batch_create.argtypes = [C.POINTER(_BatchItem), C.c_int, C.c_int, C.POINTER(C.c_void_p)]
+        L.ep_batch_create.restype = C.c_int
+        L.ep_decode_batch.argtypes = [P, P]
+        L.ep_decode_batch.restype = C.c_int
+        L.ep_batch_free.argtypes = [P]
+        L.ep_batch_free.restype = None
+        L.ep_batch_apportion.argtypes = [C.c_int, C.POINTER(C.c_int64), C.POINTER(C.c_int64), C.POINTER(C.c_int),
+                                         C.c_int, C.POINTER(C.c_int)]
+        L.ep_batch_apportion.restype = C.c_int
         L.ep_decode_status.argtypes = [P]
         L.ep_decode_status.restype = C.c_int
         L.ep_status_string.argtypes = [C.c_int]
@@ -102,7 +127,8 @@ def lib() -> C.CDLL:
 
 
 EXPORTED = ("ep_encode_tensor", "ep_free_blob", "ep_decode_tensor", "ep_decode_tensor_noalloc", "ep_decode_prepare",
-            "ep_decode_tensor_prepared", "ep_decode_status", "ep_status_string")
+            "ep_decode_tensor_prepared", "ep_batch_create", "ep_decode_batch", "ep_batch_free", "ep_batch_apportion",
+            "ep_decode_status", "ep_status_string")
 
 LUT_BYTES = 131104  # EP_LUT_BYTES: a prepared decode table
 
@@ -257,6 +283,62 @@ def decode_tensor_prepared(db: DeviceBlob, lut, out_dtype: int = BF16, out=None,
     if rc:
         raise EntroPackError(rc, "ep_decode_tensor_prepared")
     return out
+
+
+def batch_apportion(ntiles, tile_vectors, prob_bits, num_ctas: int):
+    """ep_batch_apportion (host only): SMs per tensor when a batch shares num_ctas of them out."""
+    n = len(ntiles)
+    counts = (C.c_int * max(n, 1))()
+    rc = lib().ep_batch_apportion(n, (C.c_int64 * max(n, 1))(*ntiles), (C.c_int64 * max(n, 1))(*tile_vectors),
+                                  (C.c_int * max(n, 1))(*prob_bits), num_ctas, counts)
+    if rc:
+        raise EntroPackError(rc, "ep_batch_apportion")
+    return list(counts)[:n]
+
+
+class DecodeBatch:
+    """ep_batch_create / ep_decode_batch: decode several tensors in one launch.
+
+    items: (DeviceBlob, prepared table, output tensor or None) triples; the outputs are allocated
+    here when None.  The blobs, tables and outputs are kept alive with the handle."""
+
+    def __init__(self, items, out_dtype: int = BF16):
+        import torch
+
+        self.out_dtype = out_dtype
+        self.items = []
+        arr = (_BatchItem * len(items))()
+        for k, (db, lut, out) in enumerate(items):
+            if out is None:
+                out = torch.empty((db.rows, db.cols), dtype=_torch_dtype(out_dtype), device=db.payload.device)
+            self.items.append((db, lut, out))
+            arr[k] = _BatchItem(db.payload.data_ptr(), db.tile_index.data_ptr(), db.freq_tables.data_ptr(),
+                                db.row_scales.data_ptr(), lut.data_ptr(), db.rows, db.cols, db.ntiles, db.V, db.b,
+                                out.data_ptr())
+        h = C.c_void_p()
+        rc = lib().ep_batch_create(arr, len(items), int(out_dtype), C.byref(h))
+        if rc:
+            raise EntroPackError(rc, "ep_batch_create")
+        self._h = h
+
+    @property
+    def outputs(self):
+        return [o for _, _, o in self.items]
+
+    def run(self, stream=None):
+        import torch
+
+        st = stream if stream is not None else torch.cuda.current_stream(self.items[0][0].payload.device)
+        rc = lib().ep_decode_batch(C.c_void_p(st.cuda_stream), self._h)
+        if rc:
+            raise EntroPackError(rc, "ep_decode_batch")
+        return self.outputs
+
+    def __del__(self):
+        h = getattr(self, "_h", None)
+        if h is not None and h.value:
+            lib().ep_batch_free(h)
+            self._h = None
 
 
 def decode_status(stream=None) -> int:

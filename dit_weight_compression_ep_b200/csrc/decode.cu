@@ -55,6 +55,8 @@
 #include <stdint.h>
 
 #include <mutex>
+#include <new>
+#include <vector>
 #include <type_traits>
 
 #include "entropack.h"
@@ -672,6 +674,7 @@ struct TileCtx {
     // beside the shift / logic / compare unit instead of on it)
     uint32_t two, four, k64, mneg, df, nf0;
     int64_t cols;  // (a width that is not a multiple of 8 pads each row to whole vectors)
+    uint32_t cta, G;  // this CTA's rank among the G CTAs that share the tensor: its tiles are cta + i G
 };
 
 // One tile's bookkeeping: record, staging state and every lane's row.
@@ -839,7 +842,7 @@ __device__ void decode_tiles(const uint16_t* tiles, const uint32_t* tix, const f
                              const Lut& lut, const TileCtx& tc, Ring& rg, Tile& tl, uint32_t first_i) {
     const int lane = threadIdx.x & 31;
     const uint32_t lt = lanemask_lt();
-    const uint32_t G = gridDim.x;
+    const uint32_t G = tc.G;
     bool corrupt = false;
     bool have = tl.t != 0xFFFFFFFFu;
 
@@ -899,7 +902,7 @@ __device__ void decode_tiles(const uint16_t* tiles, const uint32_t* tix, const f
         while (rg.waited < rg.seq && !rg.timed_out) ring_wait_one(rg);
         if (rg.timed_out) break;
         i += kWarps;
-        const uint64_t t64 = (uint64_t)blockIdx.x + (uint64_t)i * G;
+        const uint64_t t64 = (uint64_t)tc.cta + (uint64_t)i * G;
         have = t64 < tc.T;
         if (have) tile_begin(tc, tiles, tix, rg, tl, (uint32_t)t64, lane);
     }
@@ -972,8 +975,10 @@ __device__ __forceinline__ void run_decode(const Params& p, const Geo& g, uint32
 #undef EP_PACKED
 }
 
-template <int DT, bool RAGGED>
-__global__ void __launch_bounds__(kThreads, 1) decode_kernel(Params p) {
+// The decode of one tensor by G CTAs, this one of rank cta (the tensor's tiles cta + i G).
+// BATCH: a batch launch, always with a prepared table.
+template <int DT, bool RAGGED, bool BATCH>
+__device__ __forceinline__ void decode_body(const Params& p, const uint32_t cta, const uint32_t G) {
     extern __shared__ __align__(1024) uint8_t smem[];
     __shared__ int s_ok;
     int* s_min = reinterpret_cast<int*>(smem + kOffDesc);
@@ -987,17 +992,18 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(Params p) {
     uint32_t lane_A;
     const unsigned hs = parse_header(p.ft, p.rows, p.cols, g, lane_mn, lane_A);
     if (hs) {  // every CTA reads the same header, so every CTA leaves here
-        if (threadIdx.x == 0 && blockIdx.x == 0) raise_status(hs);
+        if (threadIdx.x == 0 && cta == 0) raise_status(hs);
         return;
     }
+    const bool prep = BATCH || p.prepared != 0;
     const uint16_t* fq = reinterpret_cast<const uint16_t*>(p.ft + table_header_bytes(kTables));
     // This CTA's table (one per CTA when G >= 16): its frequencies into registers now, so
     // that these loads, the coset table's, the tile records and the first payload chunks are
     // in flight together.
     uint32_t fr[kPre];
     int t_pre = 0;
-    if (gridDim.x >= 16 && g.mode != kModeCoarse && !p.prepared) {
-        const int t = 1 + (int)(blockIdx.x * 16u / gridDim.x);
+    if (G >= 16 && g.mode != kModeCoarse && !prep) {
+        const int t = 1 + (int)(cta * 16u / G);
         const uint32_t At = __shfl_sync(kFull, lane_A, t);
         const uint32_t offt = __reduce_add_sync(kFull, lane < t ? lane_A : 0u);
         if (At <= (uint32_t)(kPre * kThreads)) {
@@ -1033,7 +1039,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(Params p) {
     uint2 fp = make_uint2(0u, 0u);
     uint4 tr4 = make_uint4(0u, 0u, 0u, 0u);
     uint32_t tr_ib = 0;
-    if (p.prepared && threadIdx.x < 32) {
+    if (prep && threadIdx.x < 32) {
         fp = table_fingerprint(g, lane_mn, lane_A);
         if (threadIdx.x == 0) {
             const uint32_t* tr = reinterpret_cast<const uint32_t*>(p.ws + kLutBytes);
@@ -1052,11 +1058,13 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(Params p) {
     tc.four = p.one << 2;
     tc.k64 = p.one << 16;
     tc.mneg = 0u - (p.one << g.b);
+    tc.cta = cta;
+    tc.G = G;
     // the first tile's record, in flight with the loads above and below
     Tile tl;
     tl.t = 0xFFFFFFFFu;
     const uint32_t first_i = (uint32_t)warp;
-    const uint64_t t_first = (uint64_t)blockIdx.x + (uint64_t)first_i * gridDim.x;
+    const uint64_t t_first = (uint64_t)cta + (uint64_t)first_i * G;
     if (t_first < g.T) tile_load(tc, p.tix, tl, (uint32_t)t_first, lane);
     tc.total = p.tix[(size_t)kTileWords * g.T];
     tc.cmin = (uint32_t)__shfl_sync(kFull, lane_mn, 0);
@@ -1083,7 +1091,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(Params p) {
         fence_barrier_init();
         // a prepared image comes straight into shared memory, ahead of the payload's first chunks
         // (the copy stays inside the table buffer whatever its trailer holds; checked below)
-        if (warp == 0 && p.prepared && blockIdx.x < g.T) {
+        if (warp == 0 && prep && cta < g.T) {
             mbar_arrive_expect_tx(lut_bar, g.image_bytes);
             for (uint32_t o = 0; o < g.image_bytes; o += 16384u)
                 bulk_g2s(smem_u32(smem + kOffLut) + o, p.ws + o,
@@ -1097,12 +1105,12 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(Params p) {
     tc.df = tc.f1c - tc.f0c;
     tc.nf0 = 0u - tc.f0c;
 
-    if (p.prepared) {
+    if (prep) {
         // ---- a2 from a prepared table (its copy is in flight): the trailer must carry this
         // header's layout fingerprint
         if (threadIdx.x == 0) {
             s_ok = tr4.x == kLutMagic && tr4.z == fp.x && tr4.w == fp.y && tr_ib == g.image_bytes;
-            if (blockIdx.x == 0 && (!s_ok || tr4.y)) raise_status(kStHeader);
+            if (cta == 0 && (!s_ok || tr4.y)) raise_status(kStHeader);
         }
     } else {
         // ---- a2: this CTA's slice of the LUT image, a grid-wide arrival, the image into shared memory
@@ -1120,11 +1128,11 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(Params p) {
             unsigned long long* arrivals = reinterpret_cast<unsigned long long*>(p.ws + kWsCountOffset);
             const unsigned long long old = atomicAdd(arrivals, 1ull);
             // old / G without a 64-bit integer division: a double quotient (old < 2^53), corrected
-            const unsigned long long G = gridDim.x;
-            unsigned long long q = (unsigned long long)((double)old / (double)G);
-            q -= q * G > old ? 1ull : 0ull;
-            q += (q + 1ull) * G <= old ? 1ull : 0ull;
-            const unsigned long long target = (q + 1ull) * G;
+            const unsigned long long Gg = gridDim.x;  // the whole grid (here every CTA shares the tensor)
+            unsigned long long q = (unsigned long long)((double)old / (double)Gg);
+            q -= q * Gg > old ? 1ull : 0ull;
+            q += (q + 1ull) * Gg <= old ? 1ull : 0ull;
+            const unsigned long long target = (q + 1ull) * Gg;
             uint32_t spins = 0;
             // every CTA of the (cooperative, hence co-resident) grid arrives; bounded wait
             while (ld_acquire_gpu(arrivals) < target && spins < kGridSpins) {
@@ -1133,7 +1141,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(Params p) {
             }
             s_ok = spins < kGridSpins;
             if (!s_ok) raise_status(kStTimeout);
-            if (s_ok && blockIdx.x < g.T) {
+            if (s_ok && cta < g.T) {
                 fence_proxy_async_global();  // generic-proxy image stores before the bulk-copy reads
                 mbar_arrive_expect_tx(lut_bar, g.image_bytes);
                 for (uint32_t o = 0; o < g.image_bytes; o += 16384u)
@@ -1143,16 +1151,16 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(Params p) {
         }
     }
     __syncthreads();
-    if (blockIdx.x >= g.T) return;  // no tile for this CTA
+    if (cta >= g.T) return;  // no tile for this CTA
     bool lut_ok = s_ok != 0;
     // a prepared table's copy is in flight even when its trailer did not match
-    if ((lut_ok || p.prepared) && !mbar_wait(lut_bar, 0)) {
+    if ((lut_ok || prep) && !mbar_wait(lut_bar, 0)) {
         lut_ok = false;
         raise_status(kStTimeout);
     }
     lut_ok = __syncthreads_and(lut_ok) != 0;  // one decision for the whole CTA
     if (!lut_ok || bad_c) {
-        if (bad_c && threadIdx.x == 0 && blockIdx.x == 0) raise_status(kStHeader);
+        if (bad_c && threadIdx.x == 0 && cta == 0) raise_status(kStHeader);
         while (rg.waited < rg.seq && !rg.timed_out) ring_wait_one(rg);  // drain the prologue's copies
         return;
     }
@@ -1160,6 +1168,25 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(Params p) {
     const uint32_t lut_s = smem_u32(smem + kOffLut);
     const uint32_t desc2 = smem_u32(smem + kOffDesc2);
     run_decode<DT, RAGGED>(p, g, lut_s, fq, s_min, s_A, s_off, desc2, tc, rg, tl, first_i);
+}
+
+template <int DT, bool RAGGED>
+__global__ void __launch_bounds__(kThreads, 1) decode_kernel(Params p) {
+    decode_body<DT, RAGGED, false>(p, blockIdx.x, gridDim.x);
+}
+
+// One CTA of a batch launch: which tensor (its arguments, a prepared table) and which share of
+// its tiles.  count = 0: no work.
+struct alignas(16) BatchCta {
+    Params p;
+    uint32_t rank, count;
+};
+
+template <int DT, bool RAGGED>
+__global__ void __launch_bounds__(kThreads, 1) decode_batch_kernel(const BatchCta* plan) {
+    const BatchCta c = plan[blockIdx.x];
+    if (c.count == 0) return;
+    decode_body<DT, RAGGED, true>(c.p, c.rank, c.count);
 }
 
 // ep_decode_prepare's kernel: a2 without the decode.  Every CTA builds its slice of the image
@@ -1230,6 +1257,12 @@ cudaError_t set_decode_attr() {
                                          kSmemBytes);
     if (e == cudaSuccess)
         e = cudaFuncSetAttribute(decode_kernel<DT, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+    if (e == cudaSuccess)
+        e = cudaFuncSetAttribute(decode_batch_kernel<DT, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 kSmemBytes);
+    if (e == cudaSuccess)
+        e = cudaFuncSetAttribute(decode_batch_kernel<DT, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 kSmemBytes);
     return e;
 }
 
@@ -1295,6 +1328,43 @@ cudaError_t launch_any(ep_dtype dt, const Params& prm, cudaStream_t st, int num_
         case EP_FP32: return launch_decode<EP_FP32>(prm, st, num_sms);
         default: return launch_decode<EP_LATTICE_I32>(prm, st, num_sms);
     }
+}
+
+template <int DT>
+cudaError_t launch_batch(const BatchCta* plan, int ctas, bool ragged, cudaStream_t st) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)ctas);  // one CTA per SM; an ordinary launch (no grid barrier)
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = kSmemBytes;
+    cfg.stream = st;
+    return ragged ? cudaLaunchKernelEx(&cfg, decode_batch_kernel<DT, true>, plan)
+                  : cudaLaunchKernelEx(&cfg, decode_batch_kernel<DT, false>, plan);
+}
+
+cudaError_t launch_batch_any(ep_dtype dt, const BatchCta* plan, int ctas, bool ragged, cudaStream_t st) {
+    switch (dt) {
+        case EP_BF16: return launch_batch<EP_BF16>(plan, ctas, ragged, st);
+        case EP_FP16: return launch_batch<EP_FP16>(plan, ctas, ragged, st);
+        case EP_FP8_E4M3: return launch_batch<EP_FP8_E4M3>(plan, ctas, ragged, st);
+        case EP_INT8: return launch_batch<EP_INT8>(plan, ctas, ragged, st);
+        case EP_UINT8: return launch_batch<EP_UINT8>(plan, ctas, ragged, st);
+        case EP_FP32: return launch_batch<EP_FP32>(plan, ctas, ragged, st);
+        default: return launch_batch<EP_LATTICE_I32>(plan, ctas, ragged, st);
+    }
+}
+
+// A model of one tensor's decode time on c CTAs (arbitrary units), for sharing out the SMs:
+// a sub-partition either issues its share of the steps (about 31 instructions a step with a
+// packed table, more with the two-level or bucketed ones at b >= 12) or, with few tiles a warp,
+// waits on their chains (about 158 cycles a step, at least one tile a warp).  Continuous in c,
+// so that every further CTA lowers it.
+double batch_time(int64_t T, int64_t V, int b, int64_t c) {
+    const double steps = (double)((V + 31) / 32) * 9.0;
+    const double per_cta = (double)T / (double)c;
+    const double per_warp = per_cta / kWarps > 1.0 ? per_cta / kWarps : 1.0;
+    const double issue = per_cta / 4.0 * steps * (b >= 12 ? 48.0 : 31.4);
+    const double chain = per_warp * steps * 158.0;
+    return issue > chain ? issue : chain;
 }
 
 bool misaligned(const void* q, uintptr_t a) { return (reinterpret_cast<uintptr_t>(q) & (a - 1)) != 0; }
@@ -1390,6 +1460,116 @@ ep_status ep_decode_tensor_prepared(void* stream, const uint16_t* tiles, const u
                      const_cast<uint8_t*>(static_cast<const uint8_t*>(lut)), rows, cols, 1u, 1u};
     return launch_any(out_dtype, prm, static_cast<cudaStream_t>(stream), ds->num_sms) == cudaSuccess ? EP_OK
                                                                                                      : EP_ECUDA;
+}
+
+ep_status ep_batch_apportion(int n, const int64_t* ntiles, const int64_t* tile_vectors, const int* prob_bits,
+                             int num_ctas, int* counts) {
+    using namespace ep;
+    if (n <= 0 || !ntiles || !tile_vectors || !prob_bits || !counts || num_ctas < n) return EP_EINVAL;
+    for (int k = 0; k < n; ++k) {
+        if (ntiles[k] < 1 || tile_vectors[k] < 1) return EP_EINVAL;
+        counts[k] = 1;
+    }
+    // each further CTA goes to the tensor that would finish last, while it has a tile for it
+    for (int c = n; c < num_ctas; ++c) {
+        int best = -1;
+        double bt = -1.0;
+        for (int k = 0; k < n; ++k) {
+            if (counts[k] >= ntiles[k]) continue;
+            const double t = batch_time(ntiles[k], tile_vectors[k], prob_bits[k], counts[k]);
+            if (t > bt) {
+                bt = t;
+                best = k;
+            }
+        }
+        if (best < 0) break;
+        ++counts[best];
+    }
+    return EP_OK;
+}
+
+}  // extern "C"
+
+struct ep_batch {
+    int dev;
+    int ctas;
+    ep_dtype dt;
+    bool ragged;
+    ep::BatchCta* plan;  // device, one entry per CTA
+};
+
+extern "C" {
+
+ep_status ep_batch_create(const ep_batch_item* items, int n_items, ep_dtype out_dtype, ep_batch** out) {
+    using namespace ep;
+    if (!items || !out || n_items <= 0) return EP_EINVAL;
+    *out = nullptr;
+    if ((int)out_dtype < EP_BF16 || (int)out_dtype > EP_UINT8) return EP_EUNSUPPORTED;
+    bool ragged = false;
+    for (int k = 0; k < n_items; ++k) {
+        const ep_batch_item& it = items[k];
+        const ep_status as = check_decode_args(it.tiles, it.tile_index, it.freq_tables, it.row_scales, it.rows,
+                                               it.cols, out_dtype, it.out);
+        if (as != EP_OK) return as;
+        if (!it.lut || misaligned(it.lut, 16) || it.ntiles < 1 || it.tile_vectors < 1) return EP_EINVAL;
+        ragged |= (it.cols & 7) != 0;
+    }
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return EP_ECUDA;
+    DevState* ds = nullptr;
+    if (dev_setup(dev, (int)out_dtype, ds, false) != cudaSuccess) return EP_ECUDA;
+    if (n_items > ds->num_sms) return EP_EINVAL;  // at most one tensor per SM
+    std::vector<int64_t> T(n_items), V(n_items);
+    std::vector<int> b(n_items), counts(n_items);
+    for (int k = 0; k < n_items; ++k) {
+        T[k] = items[k].ntiles;
+        V[k] = items[k].tile_vectors;
+        b[k] = items[k].prob_bits;
+    }
+    if (ep_batch_apportion(n_items, T.data(), V.data(), b.data(), ds->num_sms, counts.data()) != EP_OK)
+        return EP_EINVAL;
+    std::vector<BatchCta> plan((size_t)ds->num_sms);
+    size_t c = 0;
+    for (int k = 0; k < n_items; ++k) {
+        const ep_batch_item& it = items[k];
+        const Params prm{it.tiles, it.tile_index, it.freq_tables, it.row_scales, it.out,
+                         const_cast<uint8_t*>(static_cast<const uint8_t*>(it.lut)), it.rows, it.cols, 1u, 1u};
+        for (int r = 0; r < counts[k]; ++r, ++c) plan[c] = BatchCta{prm, (uint32_t)r, (uint32_t)counts[k]};
+    }
+    for (; c < plan.size(); ++c) plan[c] = BatchCta{};  // count 0: no work
+    ep_batch* h = new (std::nothrow) ep_batch{dev, ds->num_sms, out_dtype, ragged, nullptr};
+    if (!h) return EP_ENOMEM;
+    void* d = nullptr;
+    if (cudaMalloc(&d, plan.size() * sizeof(BatchCta)) != cudaSuccess) {
+        delete h;
+        return EP_ECUDA;
+    }
+    if (cudaMemcpy(d, plan.data(), plan.size() * sizeof(BatchCta), cudaMemcpyHostToDevice) != cudaSuccess) {
+        cudaFree(d);
+        delete h;
+        return EP_ECUDA;
+    }
+    h->plan = static_cast<BatchCta*>(d);
+    *out = h;
+    return EP_OK;
+}
+
+ep_status ep_decode_batch(void* stream, const ep_batch* batch) {
+    using namespace ep;
+    if (!batch || !batch->plan) return EP_EINVAL;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return EP_ECUDA;
+    if (dev != batch->dev) return EP_EINVAL;
+    return launch_batch_any(batch->dt, batch->plan, batch->ctas, batch->ragged, static_cast<cudaStream_t>(stream)) ==
+                   cudaSuccess
+               ? EP_OK
+               : EP_ECUDA;
+}
+
+void ep_batch_free(ep_batch* batch) {
+    if (!batch) return;
+    if (batch->plan) cudaFree(batch->plan);
+    delete batch;
 }
 
 ep_status ep_decode_status(void* stream) {

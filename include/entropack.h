@@ -224,6 +224,73 @@ ep_status ep_decode_tensor_prepared(void* stream, const uint16_t* tiles, const u
                                     void* out);
 
 /*
+ * Batched decode: several tensors in one launch.  A layer-by-layer decode leaves
+ * most of the GPU idle on small tensors and on low rates (few tiles, each a long
+ * sequential chain: at the pages' tile sizes a 3840x3840 weight has under two
+ * tiles per warp scheduler); a batch shares the SMs out among its tensors, so
+ * the tiles of all of them run side by side.  There is no counterpart in the
+ * EntroPack paper; each tensor is decoded exactly as by ep_decode_tensor (one
+ * warp per tile, the same tables and arithmetic), only the assignment of tiles
+ * to SMs differs.
+ *
+ * ep_batch_item: one tensor of a batch; the pointers, shapes and alignment rules
+ * of ep_decode_tensor_prepared, plus
+ *   lut             its prepared table (ep_decode_prepare), EP_LUT_BYTES;
+ *   ntiles, tile_vectors, prob_bits
+ *                   T, V and b of its stream (the packer's blob fields).  They
+ *                   only weigh the tensor when the SMs are shared out; the
+ *                   decode itself takes T, V and b from the table header.
+ */
+typedef struct {
+    const uint16_t* tiles;
+    const uint32_t* tile_index;
+    const uint8_t* freq_tables;
+    const float* row_scales;
+    const void* lut;
+    int64_t rows, cols;
+    int64_t ntiles, tile_vectors;
+    int prob_bits;
+    void* out;
+} ep_batch_item;
+
+typedef struct ep_batch ep_batch;
+
+/*
+ * ep_batch_create -- plan one launch that decodes items[0..n_items) into
+ * out_dtype.  Every SM runs one CTA, which decodes a share of one tensor's
+ * tiles; each tensor gets at least one SM and at most one per tile, the rest
+ * going one by one to the tensor a simple cost model says finishes last
+ * (ep_batch_apportion).  At most one tensor per SM (n_items <= the SM count,
+ * else EP_EINVAL).  The plan (the items' pointers and shares, 80 bytes per SM)
+ * is copied to a device buffer the handle owns (cudaMalloc + a synchronous
+ * copy: create batches before any stream capture).  The items' buffers stay
+ * the caller's and must outlive the handle.  Argument errors: EP_EINVAL,
+ * EP_EUNSUPPORTED; CUDA errors: EP_ECUDA.  On success *out holds the handle.
+ */
+ep_status ep_batch_create(const ep_batch_item* items, int n_items, ep_dtype out_dtype, ep_batch** out);
+
+/*
+ * ep_decode_batch -- one launch on `stream` (an ordinary launch, one CTA per
+ * SM) that decodes every tensor of the batch into its `out`.  Outputs, status
+ * reporting and the checks of each tensor's header and table are those of
+ * ep_decode_tensor_prepared.  The current device must be the one the batch was
+ * created on (else EP_EINVAL).  Capturable in a CUDA graph.
+ */
+ep_status ep_decode_batch(void* stream, const ep_batch* batch);
+
+/* Free a batch handle (NULL is allowed); synchronises the device (cudaFree). */
+void ep_batch_free(ep_batch* batch);
+
+/*
+ * ep_batch_apportion -- the host-only share-out ep_batch_create uses: counts[k]
+ * SMs for tensor k, each in [1, ntiles[k]], together at most num_ctas (fewer
+ * when the tensors have fewer tiles than that).  EP_EINVAL when n <= 0,
+ * num_ctas < n, a pointer is NULL or a tensor has no tile.
+ */
+ep_status ep_batch_apportion(int n, const int64_t* ntiles, const int64_t* tile_vectors, const int* prob_bits,
+                             int num_ctas, int* counts);
+
+/*
  * ep_decode_status -- synchronise `stream`, read and clear the status word of
  * the current device: EP_OK, EP_ECORRUPT (an inconsistent stream or header),
  * or EP_EUNSUPPORTED (a header variant the GPU decoder does not handle).
