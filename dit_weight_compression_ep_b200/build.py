@@ -17,7 +17,7 @@ BUILD = os.path.join(ROOT, "_build")
 
 CU_SOURCES = ["decode.cu"]
 CPP_SOURCES = ["encode.cpp"]
-HEADERS = ["ep_format.h"]
+HEADERS = ["ep_format.h", "encode_host.h"]
 
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]

@@ -24,9 +24,15 @@
 
 #include "entropack.h"
 #include "ep_format.h"
+#include "encode_host.h"
 
 namespace ep {
 namespace {
+
+using host::Hist;
+using host::normalise;
+using host::Table;
+using host::tile_symbols_for;
 
 // ------------------------------------------------------------------ threads
 
@@ -126,46 +132,6 @@ void quantize_row(const float* w, int64_t cols, double n, double s, int32_t* f, 
 
 // --------------------------------------------------------------- the model
 
-struct Hist {
-    int64_t lo[kTables], hi[kTables];
-    void reset() {
-        for (int t = 0; t < kTables; ++t) {
-            lo[t] = INT64_MAX;
-            hi[t] = INT64_MIN;
-        }
-    }
-    void add_range(const int32_t* f, int64_t n) {
-        for (int64_t g = 0; g < n; ++g) {
-            const int32_t* v = f + kFields * g;
-            for (int k = 0; k < kFields; ++k) {
-                const int t = table_index(k, v[0]);
-                lo[t] = std::min<int64_t>(lo[t], v[k]);
-                hi[t] = std::max<int64_t>(hi[t], v[k]);
-            }
-        }
-    }
-    void merge(const Hist& o) {
-        for (int t = 0; t < kTables; ++t) {
-            lo[t] = std::min(lo[t], o.lo[t]);
-            hi[t] = std::max(hi[t], o.hi[t]);
-        }
-    }
-    uint64_t alpha(int t) const { return hi[t] >= lo[t] ? (uint64_t)(hi[t] - lo[t] + 1) : 0; }
-    uint64_t amax_coord() const {
-        uint64_t m = 0;
-        for (int t = 1; t < kTables; ++t) m = std::max(m, alpha(t));
-        return m;
-    }
-};
-
-struct Table {
-    int32_t min = 0;
-    uint32_t A = 0;
-    uint64_t total = 0;
-    std::vector<uint64_t> count;
-    std::vector<uint32_t> freq, cum;
-};
-
 // alphabets ([min, max] per table) of vectors [0, nvec): contiguous parts per thread, then merged
 Hist alphabet_of(const int32_t* f, int64_t nvec, int nthreads) {
     const int nt = std::max(1, (int)std::min<int64_t>(nthreads, (nvec + 65535) / 65536));
@@ -226,48 +192,6 @@ void count_fields(const int32_t* f, int64_t nvec, const Hist& al, Table* tabs, i
             tabs[t].count[s] = v;
             tabs[t].total += v;
         }
-}
-
-// Frequencies at M = 2^b: f = max(1, floor(count*M/total + 1/2)) for present
-// symbols; the excess comes off the largest f > 1 one unit at a time (lowest
-// symbol on ties), a shortfall goes to the most frequent symbol (lowest on ties).
-void normalise(Table& tb, int b) {
-    const uint32_t M = 1u << b;
-    tb.freq.assign(std::max<uint32_t>(tb.A, 1), 0);
-    tb.cum.assign(std::max<uint32_t>(tb.A, 1) + 1, 0);
-    if (tb.A == 0) return;
-    uint64_t sum = 0;
-    for (uint32_t s = 0; s < tb.A; ++s) {
-        if (tb.count[s]) {
-            const double q = (double)tb.count[s] * (double)M / (double)tb.total;
-            const double r = std::floor(q + 0.5);
-            tb.freq[s] = r < 1.0 ? 1u : (uint32_t)r;
-        }
-        sum += tb.freq[s];
-    }
-    if (sum > M) {
-        // max-heap on (f, -s): the same choice as a scan for the largest f > 1, lowest s
-        auto cmp = [&](uint32_t x, uint32_t y) {
-            return tb.freq[x] != tb.freq[y] ? tb.freq[x] < tb.freq[y] : x > y;
-        };
-        std::priority_queue<uint32_t, std::vector<uint32_t>, decltype(cmp)> pq(cmp);
-        for (uint32_t s = 0; s < tb.A; ++s)
-            if (tb.freq[s] > 1) pq.push(s);
-        while (sum > M && !pq.empty()) {
-            const uint32_t s = pq.top();
-            pq.pop();
-            tb.freq[s] -= 1;
-            sum -= 1;
-            if (tb.freq[s] > 1) pq.push(s);
-        }
-    }
-    if (sum < M) {
-        uint32_t best = 0;
-        for (uint32_t s = 1; s < tb.A; ++s)
-            if (tb.count[s] > tb.count[best]) best = s;
-        tb.freq[best] += (uint32_t)(M - sum);
-    }
-    for (uint32_t s = 0; s < tb.A; ++s) tb.cum[s + 1] = tb.cum[s] + tb.freq[s];
 }
 
 // ------------------------------------------------- per-row refinement (RDO)
@@ -467,16 +391,6 @@ void encode_tile(const int32_t* fields, int64_t v0, int64_t vt, const Table* tab
 
 // ---------------------------------------------------------------- the blob
 
-int64_t tile_symbols_for(double target) {
-    if (target <= 2.5) return 32768;
-    if (target <= 5.0) return 16384;
-    if (target <= 7.0) return 8192;
-    return 4096;
-}
-
-void put32(uint8_t* p, uint32_t v) { std::memcpy(p, &v, 4); }  // little-endian hosts only
-void put64(uint8_t* p, uint64_t v) { std::memcpy(p, &v, 8); }
-
 struct Encoder {
     const float* W;
     int64_t rows, cols, nq, nvec;
@@ -485,14 +399,6 @@ struct Encoder {
     bool container;
     int64_t ntiles;
     std::vector<double> norms;
-
-    int64_t side_bytes(const Hist& al) const {
-        int64_t tb = table_header_bytes(kTables);
-        for (int t = 0; t < kTables; ++t) tb += 2 * (int64_t)al.alpha(t);
-        int64_t side = tb + ntiles * (4 * kLanes + 4) + 4 + 4 * rows;
-        if (container) side += 4 * rows;
-        return side;
-    }
 
     // Stored-size estimate from the sampled rows at (s, b); +inf when an alphabet exceeds 2^b.
     double estimate(const std::vector<int64_t>& srows, double s, int b, std::vector<int32_t>& sf) const {
@@ -507,19 +413,166 @@ struct Encoder {
         if (al.amax_coord() > (1ull << b)) return INFINITY;
         Table tabs[kTables];
         count_fields(sf.data(), ns, al, tabs, nthreads);
-        double bits = 0.0;
-        for (int t = 0; t < kTables; ++t) {
-            normalise(tabs[t], b);
-            for (uint32_t k = 0; k < tabs[t].A; ++k)
-                if (tabs[t].count[k]) bits += (double)tabs[t].count[k] * ((double)b - std::log2((double)tabs[t].freq[k]));
-        }
-        const double payload = bits / 8.0 * ((double)nvec / (double)ns);
-        const double total = payload + (double)side_bytes(al);
-        return 8.0 * total / (double)(rows * cols);  // per real weight
+        return host::estimate_bpp(tabs, al, b, nvec, ns, ntiles, rows, cols, container);
     }
 };
 
 }  // namespace
+
+// ------------------------------------------------ shared with the GPU encoder
+
+namespace host {
+
+// Frequencies at M = 2^b: f = max(1, floor(count*M/total + 1/2)) for present
+// symbols; the excess comes off the largest f > 1 one unit at a time (lowest
+// symbol on ties), a shortfall goes to the most frequent symbol (lowest on ties).
+void normalise(Table& tb, int b) {
+    const uint32_t M = 1u << b;
+    tb.freq.assign(std::max<uint32_t>(tb.A, 1), 0);
+    tb.cum.assign(std::max<uint32_t>(tb.A, 1) + 1, 0);
+    if (tb.A == 0) return;
+    uint64_t sum = 0;
+    for (uint32_t s = 0; s < tb.A; ++s) {
+        if (tb.count[s]) {
+            const double q = (double)tb.count[s] * (double)M / (double)tb.total;
+            const double r = std::floor(q + 0.5);
+            tb.freq[s] = r < 1.0 ? 1u : (uint32_t)r;
+        }
+        sum += tb.freq[s];
+    }
+    if (sum > M) {
+        // max-heap on (f, -s): the same choice as a scan for the largest f > 1, lowest s
+        auto cmp = [&](uint32_t x, uint32_t y) {
+            return tb.freq[x] != tb.freq[y] ? tb.freq[x] < tb.freq[y] : x > y;
+        };
+        std::priority_queue<uint32_t, std::vector<uint32_t>, decltype(cmp)> pq(cmp);
+        for (uint32_t s = 0; s < tb.A; ++s)
+            if (tb.freq[s] > 1) pq.push(s);
+        while (sum > M && !pq.empty()) {
+            const uint32_t s = pq.top();
+            pq.pop();
+            tb.freq[s] -= 1;
+            sum -= 1;
+            if (tb.freq[s] > 1) pq.push(s);
+        }
+    }
+    if (sum < M) {
+        uint32_t best = 0;
+        for (uint32_t s = 1; s < tb.A; ++s)
+            if (tb.count[s] > tb.count[best]) best = s;
+        tb.freq[best] += (uint32_t)(M - sum);
+    }
+    for (uint32_t s = 0; s < tb.A; ++s) tb.cum[s + 1] = tb.cum[s] + tb.freq[s];
+}
+
+int64_t tile_symbols_for(double target) {
+    if (target <= 2.5) return 32768;
+    if (target <= 5.0) return 16384;
+    if (target <= 7.0) return 8192;
+    return 4096;
+}
+
+void put32(uint8_t* p, uint32_t v) { std::memcpy(p, &v, 4); }  // little-endian hosts only
+void put64(uint8_t* p, uint64_t v) { std::memcpy(p, &v, 8); }
+
+std::vector<int64_t> sample_rows(int64_t rows, int64_t cols, const ep_encode_opts& o) {
+    // sampled rows: partial Fisher-Yates driven by splitmix64 (Steele, Lea & Flood)
+    const int64_t nq = (cols + 7) / 8;
+    const int64_t sv = o.sample_vectors > 0 ? o.sample_vectors : (int64_t)1 << 18;
+    const int64_t rs = std::max<int64_t>(1, std::min<int64_t>(rows, (sv + nq - 1) / nq));
+    std::vector<int64_t> perm(rows);
+    for (int64_t i = 0; i < rows; ++i) perm[i] = i;
+    uint64_t st = o.seed ? o.seed : (((uint64_t)rows << 32) ^ (uint64_t)cols);
+    std::vector<int64_t> srows(rs);
+    for (int64_t i = 0; i < rs; ++i) {
+        st += 0x9E3779B97F4A7C15ull;
+        uint64_t z = st;
+        z = (z ^ (z >> 30)) * 0xBF58476D1CE4E5B9ull;
+        z = (z ^ (z >> 27)) * 0x94D049BB133111EBull;
+        z ^= z >> 31;
+        const int64_t j = i + (int64_t)(z % (uint64_t)(rows - i));
+        std::swap(perm[i], perm[j]);
+        srows[i] = perm[i];
+    }
+    return srows;
+}
+
+int64_t side_bytes(const Hist& al, int64_t ntiles, int64_t rows, bool container) {
+    int64_t tb = table_header_bytes(kTables);
+    for (int t = 0; t < kTables; ++t) tb += 2 * (int64_t)al.alpha(t);
+    int64_t side = tb + ntiles * (4 * kLanes + 4) + 4 + 4 * rows;
+    if (container) side += 4 * rows;
+    return side;
+}
+
+double estimate_bpp(Table* tabs, const Hist& al, int b, int64_t nvec, int64_t ns, int64_t ntiles, int64_t rows,
+                    int64_t cols, bool container) {
+    double bits = 0.0;
+    for (int t = 0; t < kTables; ++t) {
+        normalise(tabs[t], b);
+        for (uint32_t k = 0; k < tabs[t].A; ++k)
+            if (tabs[t].count[k]) bits += (double)tabs[t].count[k] * ((double)b - std::log2((double)tabs[t].freq[k]));
+    }
+    const double payload = bits / 8.0 * ((double)nvec / (double)ns);
+    const double total = payload + (double)side_bytes(al, ntiles, rows, container);
+    return 8.0 * total / (double)(rows * cols);  // per real weight
+}
+
+ep_blob* new_blob(int64_t rows, int64_t cols, int b, int64_t V, int64_t T, uint64_t words, const Table* tabs) {
+    ep_blob* bl = (ep_blob*)std::calloc(1, sizeof(ep_blob));
+    if (!bl) return nullptr;
+    bl->rows = rows;
+    bl->cols = cols;
+    bl->b = b;
+    bl->V = (int)V;
+    bl->J = kLanes;
+    bl->ntiles = (int)T;
+    bl->payload_words = words;
+    bl->payload_alloc_words = (words + 7) / 8 * 8;
+    bl->payload = (uint16_t*)std::calloc(std::max<size_t>(bl->payload_alloc_words, 8), sizeof(uint16_t));
+    bl->tile_index = (uint32_t*)std::malloc(sizeof(uint32_t) * (size_t)(kTileWords * T + 1));
+    int64_t nf = 0;
+    for (int t = 0; t < kTables; ++t) nf += tabs[t].A;
+    bl->freq_bytes = (size_t)(table_header_bytes(kTables) + 2 * nf);
+    bl->freq_tables = (uint8_t*)std::calloc(bl->freq_bytes, 1);
+    bl->row_scales = (float*)std::malloc(sizeof(float) * (size_t)rows);
+    if (!bl->payload || !bl->tile_index || !bl->freq_tables || !bl->row_scales) {
+        ep_free_blob(bl);
+        return nullptr;
+    }
+    uint8_t* h = bl->freq_tables;
+    put32(h + 0, kMagic);
+    put32(h + 4, kVersion);
+    put32(h + 8, (uint32_t)b);
+    put32(h + 12, (uint32_t)V);
+    put32(h + 16, (uint32_t)kLanes);
+    put32(h + 20, (uint32_t)T);
+    put64(h + 24, (uint64_t)rows);
+    put64(h + 32, (uint64_t)cols);
+    put32(h + 40, (uint32_t)kTables);
+    put32(h + 44, 0u);
+    int64_t fo = table_header_bytes(kTables);
+    for (int t = 0; t < kTables; ++t) {
+        put32(h + kHeaderFixedBytes + 8 * t, (uint32_t)tabs[t].min);
+        put32(h + kHeaderFixedBytes + 8 * t + 4, tabs[t].A);
+        for (uint32_t k = 0; k < tabs[t].A; ++k) {
+            const uint16_t v = (uint16_t)tabs[t].freq[k];
+            std::memcpy(h + fo, &v, 2);
+            fo += 2;
+        }
+    }
+    return bl;
+}
+
+void finish_blob(ep_blob* bl, double s, bool container) {
+    const int64_t rows = bl->rows;
+    bl->s = s;
+    bl->stored_bytes = (int64_t)(2 * bl->payload_words) + (int64_t)(4 * ((size_t)kTileWords * bl->ntiles + 1)) +
+                       (int64_t)bl->freq_bytes + 4 * rows + (container ? 4 * rows : 0);
+    bl->stored_bpp = 8.0 * (double)bl->stored_bytes / (double)(rows * bl->cols);
+}
+
+}  // namespace host
 }  // namespace ep
 
 extern "C" {
@@ -564,23 +617,8 @@ ep_status ep_encode_tensor(const float* W, int64_t rows, int64_t cols, double ta
             }
         });
 
-        // sampled rows: partial Fisher-Yates driven by splitmix64 (Steele, Lea & Flood)
-        const int64_t sv = o.sample_vectors > 0 ? o.sample_vectors : (int64_t)1 << 18;
-        int64_t rs = std::max<int64_t>(1, std::min<int64_t>(rows, (sv + nq - 1) / nq));
-        std::vector<int64_t> perm(rows);
-        for (int64_t i = 0; i < rows; ++i) perm[i] = i;
-        uint64_t st = o.seed ? o.seed : (((uint64_t)rows << 32) ^ (uint64_t)cols);
-        std::vector<int64_t> srows(rs);
-        for (int64_t i = 0; i < rs; ++i) {
-            st += 0x9E3779B97F4A7C15ull;
-            uint64_t z = st;
-            z = (z ^ (z >> 30)) * 0xBF58476D1CE4E5B9ull;
-            z = (z ^ (z >> 27)) * 0x94D049BB133111EBull;
-            z ^= z >> 31;
-            const int64_t j = i + (int64_t)(z % (uint64_t)(rows - i));
-            std::swap(perm[i], perm[j]);
-            srows[i] = perm[i];
-        }
+        const std::vector<int64_t> srows = host::sample_rows(rows, cols, o);
+        const int64_t rs = (int64_t)srows.size();
         std::vector<int32_t> sf((size_t)(kFields * nq * rs));
         std::vector<int32_t> fields((size_t)(kFields * nvec));
         std::vector<double> num(rows), den(rows);
@@ -653,27 +691,8 @@ ep_status ep_encode_tensor(const float* W, int64_t rows, int64_t cols, double ta
         if (words > 0xFFFFFFFFull) return EP_EINVAL;
         tix[kTileWords * T] = (uint32_t)words;
 
-        ep_blob* bl = (ep_blob*)std::calloc(1, sizeof(ep_blob));
+        ep_blob* bl = host::new_blob(rows, cols, b, V, T, words, tabs);
         if (!bl) return EP_ENOMEM;
-        bl->rows = rows;
-        bl->cols = cols;
-        bl->b = b;
-        bl->V = (int)V;
-        bl->J = kLanes;
-        bl->ntiles = (int)T;
-        bl->payload_words = words;
-        bl->payload_alloc_words = (words + 7) / 8 * 8;
-        bl->payload = (uint16_t*)std::calloc(std::max<size_t>(bl->payload_alloc_words, 8), sizeof(uint16_t));
-        bl->tile_index = (uint32_t*)std::malloc(sizeof(uint32_t) * tix.size());
-        int64_t nf = 0;
-        for (int t = 0; t < kTables; ++t) nf += tabs[t].A;
-        bl->freq_bytes = (size_t)(table_header_bytes(kTables) + 2 * nf);
-        bl->freq_tables = (uint8_t*)std::calloc(bl->freq_bytes, 1);
-        bl->row_scales = (float*)std::malloc(sizeof(float) * (size_t)rows);
-        if (!bl->payload || !bl->tile_index || !bl->freq_tables || !bl->row_scales) {
-            ep_free_blob(bl);
-            return EP_ENOMEM;
-        }
         size_t o16 = 0;
         for (int64_t t = 0; t < T; ++t) {
             if (!tile_words[t].empty())
@@ -682,31 +701,7 @@ ep_status ep_encode_tensor(const float* W, int64_t rows, int64_t cols, double ta
         }
         std::memcpy(bl->tile_index, tix.data(), sizeof(uint32_t) * tix.size());
         std::memcpy(bl->row_scales, scales.data(), sizeof(float) * (size_t)rows);
-        uint8_t* h = bl->freq_tables;
-        put32(h + 0, kMagic);
-        put32(h + 4, kVersion);
-        put32(h + 8, (uint32_t)b);
-        put32(h + 12, (uint32_t)V);
-        put32(h + 16, (uint32_t)kLanes);
-        put32(h + 20, (uint32_t)T);
-        put64(h + 24, (uint64_t)rows);
-        put64(h + 32, (uint64_t)cols);
-        put32(h + 40, (uint32_t)kTables);
-        put32(h + 44, 0u);
-        int64_t fo = table_header_bytes(kTables);
-        for (int t = 0; t < kTables; ++t) {
-            put32(h + kHeaderFixedBytes + 8 * t, (uint32_t)tabs[t].min);
-            put32(h + kHeaderFixedBytes + 8 * t + 4, tabs[t].A);
-            for (uint32_t k = 0; k < tabs[t].A; ++k) {
-                const uint16_t v = (uint16_t)tabs[t].freq[k];
-                std::memcpy(h + fo, &v, 2);
-                fo += 2;
-            }
-        }
-        bl->s = s;
-        bl->stored_bytes = (int64_t)(2 * words) + (int64_t)(4 * tix.size()) + (int64_t)bl->freq_bytes + 4 * rows +
-                           (enc.container ? 4 * rows : 0);
-        bl->stored_bpp = 8.0 * (double)bl->stored_bytes / (double)(rows * cols);
+        host::finish_blob(bl, s, enc.container);
         *out = bl;
         return EP_OK;
     } catch (const std::bad_alloc&) {
