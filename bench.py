@@ -714,6 +714,61 @@ def run_dit(args):
     print(json.dumps(res), flush=True)
 
 
+def run_encode(args):
+    """Conversion speed: the 3840x10240 headline at 4 bpp through the CPU packer (all host
+    threads) and the GPU encoder (weights already on the GPU, blob returned in host memory; the
+    two blobs are checked identical), then the whole DiT stack (150 layers at the per-layer
+    rates) through the GPU encoder, each layer's float32 weights copied from pinned host memory
+    inside the timed loop.  Wall-clock times (the encoder synchronises its stream)."""
+    import torch
+
+    import dit_weight_compression_ep_b200 as ep
+    from dit_weight_compression_ep_b200 import build, synth
+
+    build.build()
+    W = synth.generate(synth.headline())
+    Wd = torch.from_numpy(W).cuda()
+    cpu_t, gpu_t = [], []
+    for _ in range(3):
+        t0 = time.time()
+        cb = ep.encode_tensor(W, 4.0)
+        cpu_t.append(time.time() - t0)
+    ep.encode_tensor_gpu(Wd, 4.0)  # warm-up (module load, first allocations)
+    for _ in range(5):
+        torch.cuda.synchronize()
+        t0 = time.time()
+        gb = ep.encode_tensor_gpu(Wd, 4.0)
+        gpu_t.append(time.time() - t0)
+    same = (np.array_equal(gb.payload, cb.payload) and np.array_equal(gb.tile_index, cb.tile_index) and
+            np.array_equal(gb.freq_tables, cb.freq_tables) and
+            np.array_equal(gb.row_scales.view(np.uint32), cb.row_scales.view(np.uint32)))
+    res = {"case": "encode 3840x10240 at 4 bpp", "cpu_packer_s": round(min(cpu_t), 4),
+           "cpu_threads": os.cpu_count(), "gpu_encoder_s": round(min(gpu_t), 4), "identical_blobs": same,
+           "pages_gpu_ms_per_39m_layer": "11-36 (their GPU, context)"}
+    print(json.dumps(res), flush=True)
+    del Wd
+    alloc = synth.dit_stack_bpp()
+    kinds = list(synth.DIT_KINDS)
+    host = {k: torch.from_numpy(synth.generate(synth.dit_stack_layer(0, k))).pin_memory() for k in kinds}
+    dev = {k: torch.empty(host[k].shape, dtype=torch.float32, device="cuda") for k in kinds}
+    order = sorted(alloc.items())
+    for k in kinds:  # warm-up
+        dev[k].copy_(host[k])
+    torch.cuda.synchronize()
+    t0 = time.time()
+    nweights, nbytes = 0, 0
+    for (_, k), bpp in order:
+        dev[k].copy_(host[k], non_blocking=True)
+        b = ep.encode_tensor_gpu(dev[k], bpp)
+        nweights += b.rows * b.cols
+        nbytes += b.stored_bytes
+    tot = time.time() - t0
+    res2 = {"case": "encode the DiT stack (150 layers, per-layer rates) on the GPU", "seconds": round(tot, 3),
+            "layers": len(order), "weights": nweights, "stored_bytes": nbytes,
+            "stored_bpp": round(8.0 * nbytes / nweights, 4), "pages_whole_model_s": "3.5 (their GPU, context)"}
+    print(json.dumps(res2), flush=True)
+
+
 def run_linear(args):
     """A linear layer whose weight is stored compressed: decode it with the library, then the
     library GEMM (cuBLAS through torch), against the same GEMM with the weight resident
@@ -807,6 +862,7 @@ def main():
     ap.add_argument("--sweep", action="store_true", help="every workload's decode throughput (one GPU)")
     ap.add_argument("--linear", action="store_true", help="decode-then-GEMM against a resident weight (one GPU)")
     ap.add_argument("--dit", action="store_true", help="the whole DiT stack: per layer, prepared, block batches")
+    ap.add_argument("--encode", action="store_true", help="conversion speed: CPU packer and GPU encoder")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
@@ -822,6 +878,9 @@ def main():
         return
     if args.dit:
         run_dit(args)
+        return
+    if args.encode:
+        run_encode(args)
         return
     if args.impl == "reference":
         if rank != 0:

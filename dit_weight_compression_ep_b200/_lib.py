@@ -99,6 +99,9 @@ def lib() -> C.CDLL:
         L.ep_encode_tensor.argtypes = [P, C.c_int64, C.c_int64, C.c_double, C.POINTER(_Opts),
                                        C.POINTER(C.POINTER(_Blob))]
         L.ep_encode_tensor.restype = C.c_int
+        L.ep_encode_tensor_gpu.argtypes = [P, P, C.c_int64, C.c_int64, C.c_double, C.POINTER(_Opts),
+                                           C.POINTER(C.POINTER(_Blob))]
+        L.ep_encode_tensor_gpu.restype = C.c_int
         L.ep_free_blob.argtypes = [C.POINTER(_Blob)]
         L.ep_free_blob.restype = None
         L.ep_decode_tensor.argtypes = [P, P, P, P, P, C.c_int64, C.c_int64, C.c_int, P]
@@ -126,7 +129,7 @@ def lib() -> C.CDLL:
     return _lib
 
 
-EXPORTED = ("ep_encode_tensor", "ep_free_blob", "ep_decode_tensor", "ep_decode_tensor_noalloc", "ep_decode_prepare",
+EXPORTED = ("ep_encode_tensor", "ep_encode_tensor_gpu", "ep_free_blob", "ep_decode_tensor", "ep_decode_tensor_noalloc", "ep_decode_prepare",
             "ep_decode_tensor_prepared", "ep_batch_create", "ep_decode_batch", "ep_batch_free", "ep_batch_apportion",
             "ep_decode_status", "ep_status_string")
 
@@ -187,6 +190,33 @@ def encode_tensor(W: np.ndarray, target_bpp: float, *, prob_bits: int = 0, tile_
     rc = lib().ep_encode_tensor(W.ctypes.data, W.shape[0], W.shape[1], float(target_bpp), C.byref(o), C.byref(out))
     if rc:
         raise EntroPackError(rc, "ep_encode_tensor")
+    return _take_blob(out)
+
+
+def encode_tensor_gpu(W, target_bpp: float, *, prob_bits: int = 0, tile_vectors: int = 0, sample_vectors: int = 0,
+                      search_steps: int = 0, seed: int = 0, has_container_scales: bool = False,
+                      rdo_candidates: int = 0, stream=None) -> Blob:
+    """Compress a float32 CUDA matrix with ep_encode_tensor_gpu: the same blob as encode_tensor, its
+    full-tensor stages on the GPU (launched on `stream`, default torch's current stream).  The
+    per-row refinement (rdo_candidates > 1) is not on this path: EP_EUNSUPPORTED."""
+    import torch
+
+    if not (isinstance(W, torch.Tensor) and W.is_cuda and W.dtype == torch.float32 and W.dim() == 2):
+        raise ValueError("W must be a 2-D float32 CUDA tensor")
+    W = W.contiguous()
+    o = _Opts(prob_bits, tile_vectors, sample_vectors, search_steps, seed, int(has_container_scales), 0,
+              int(rdo_candidates), 0)
+    st = stream if stream is not None else torch.cuda.current_stream(W.device)
+    out = C.POINTER(_Blob)()
+    rc = lib().ep_encode_tensor_gpu(C.c_void_p(st.cuda_stream), W.data_ptr(), W.shape[0], W.shape[1],
+                                    float(target_bpp), C.byref(o), C.byref(out))
+    if rc:
+        raise EntroPackError(rc, "ep_encode_tensor_gpu")
+    return _take_blob(out)
+
+
+def _take_blob(out) -> Blob:
+    """Copy a library blob into numpy arrays and free it."""
     try:
         b = out.contents
         T = b.ntiles

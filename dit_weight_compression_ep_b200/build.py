@@ -15,7 +15,9 @@ INCLUDE = os.path.join(ROOT, "include")
 SO = os.path.join(HERE, "libentropack.so")
 BUILD = os.path.join(ROOT, "_build")
 
-CU_SOURCES = ["decode.cu"]
+CU_SOURCES = ["decode.cu", "encode_gpu.cu"]
+# the GPU encoder rounds every product and sum as the CPU packer does: no multiply-add contraction
+CU_FLAGS = {"encode_gpu.cu": ["-fmad=false", "-Xcompiler", "-ffp-contract=off"]}
 CPP_SOURCES = ["encode.cpp"]
 HEADERS = ["ep_format.h", "encode_host.h"]
 
@@ -44,7 +46,7 @@ def build(force: bool = False, verbose: bool = False) -> str:
     for src in CU_SOURCES:
         obj = os.path.join(BUILD, src + ".o")
         cmd = [NVCC, *ARCH, "-lineinfo", "-O3", "-std=c++17", "-Xcompiler", "-fPIC", "-I", INCLUDE, "-I", CSRC,
-               "-c", os.path.join(CSRC, src), "-o", obj]
+               *CU_FLAGS.get(src, []), "-c", os.path.join(CSRC, src), "-o", obj]
         if verbose:
             cmd.insert(1, "-Xptxas=-v")
         subprocess.check_call(cmd)

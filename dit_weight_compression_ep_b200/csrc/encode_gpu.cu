@@ -1,0 +1,530 @@
+// encode_gpu.cu -- ep_encode_tensor_gpu: the packer with its full-tensor stages on the GPU.
+//
+// EntroPack paper §3.1 pipeline, as in encode.cpp: row normalisation, the sampled-row scale
+// search (§3.4, App. C.1), full-tensor E8 quantisation (§1, Conway & Sloane 1982), the row-scale
+// refit (§3.5), the seventeen coset-conditioned tables (§3.6, App. A.3) and tiled interleaved
+// rANS (§3.6, App. C.3).  The result is byte for byte the CPU packer's blob:
+//   - every floating-point step is the host's operation in the host's order (one thread per
+//     row for the row sums, taken in index order), and this file is compiled without
+//     multiply-add contraction (-fmad=false), so each product and sum rounds as on the host;
+//     division, square root and rint are IEEE round-to-nearest on both sides;
+//   - the search's estimates come from exact integer counts made here and turned into bits on
+//     the host by the same code as the CPU packer (normalisation and log2 stay on the host);
+//   - the rANS step is integer arithmetic; a warp encodes a tile, lane j holding the tile's
+//     lane j, and each step's words are placed in the order the host emits them.
+// What runs on the host: the sample choice, the search's decisions, the b escalation, table
+// normalisation and the blob header.  The per-row refinement (App. C.2) is not on this path.
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include <algorithm>
+#include <climits>
+#include <cmath>
+#include <new>
+#include <vector>
+
+#include "encode_host.h"
+#include "entropack.h"
+#include "ep_format.h"
+
+namespace ep {
+namespace {
+
+using host::Hist;
+using host::Table;
+
+constexpr int kQThreads = 256;
+
+// ------------------------------------------------------------ the quantiser
+
+// Nearest point of D8: round to nearest (ties to even); an odd sum moves the coordinate
+// furthest from its rounding (the first such) one step the other way (up when u - a >= 0).
+__device__ __forceinline__ void d8_nearest(const double (&u)[8], double (&a)[8]) {
+    long long par = 0;
+    int far_k = 0;
+    double far_d = -1.0;
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+        a[k] = rint(u[k]);
+        par += (long long)a[k];
+        const double d = fabs(u[k] - a[k]);
+        if (d > far_d) {
+            far_d = d;
+            far_k = k;
+        }
+    }
+    if (par & 1LL) {
+#pragma unroll
+        for (int k = 0; k < 8; ++k)
+            if (k == far_k) a[k] += (u[k] - a[k] >= 0.0) ? 1.0 : -1.0;
+    }
+}
+
+// E8 = D8 u (D8 + 1/2), the nearer coset (ties to D8); the fields (c, z1..z7, m) into f.
+__device__ __forceinline__ void e8_fields(const double (&u)[8], int32_t* f) {
+    double a[8], h[8], v[8];
+    d8_nearest(u, a);
+#pragma unroll
+    for (int k = 0; k < 8; ++k) v[k] = u[k] - 0.5;
+    d8_nearest(v, h);
+    double da = 0.0, dh = 0.0;
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+        const double ea = u[k] - a[k];
+        const double eh = u[k] - (h[k] + 0.5);
+        da += ea * ea;
+        dh += eh * eh;
+    }
+    const int c = dh < da ? 1 : 0;
+    long long s7 = 0;
+    f[0] = c;
+#pragma unroll
+    for (int k = 0; k < 7; ++k) {
+        const double z = c ? h[k] : a[k];
+        f[1 + k] = (int32_t)z;
+        s7 += (long long)z;
+    }
+    const long long z8 = (long long)(c ? h[7] : a[7]);
+    f[8] = (int32_t)((z8 - (s7 & 1LL)) / 2);
+}
+
+// ----------------------------------------------------------------- kernels
+
+// Row normaliser: the RMS of the row (a sum of squares in index order), 1 for a zero row.
+__global__ void k_norms(const float* W, int64_t rows, int64_t cols, double* norms) {
+    const int64_t r = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (r >= rows) return;
+    const float* w = W + r * cols;
+    double acc = 0.0;
+    for (int64_t j = 0; j < cols; ++j) acc += (double)w[j] * (double)w[j];
+    const double n = sqrt(acc / (double)cols);
+    norms[r] = n > 0.0 ? n : 1.0;
+}
+
+// Fields of vectors [0, nrows * nq) at scale s: vector (i, q) is vector q of row rowlist[i]
+// (row i without a list); a partial last vector is padded with zeros.
+__global__ void k_quantize(const float* W, int64_t cols, int64_t nq, const double* norms, const int64_t* rowlist,
+                           int64_t nrows, double s, int32_t* fields) {
+    const int64_t g = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (g >= nrows * nq) return;
+    const int64_t i = g / nq, q = g - i * nq;
+    const int64_t r = rowlist ? rowlist[i] : i;
+    const float* w = W + r * cols + 8 * q;
+    const double n = norms[r];
+    const int64_t real = cols - 8 * q < 8 ? cols - 8 * q : 8;
+    double u[8];
+#pragma unroll
+    for (int k = 0; k < 8; ++k) u[k] = k < real ? ((double)w[k] / n) / s : 0.0;
+    e8_fields(u, fields + kFields * g);
+}
+
+// [min, max] of every table's symbols over vectors [0, nvec) (lohi: 17 minima, then 17 maxima).
+__global__ void k_alphabet(const int32_t* fields, int64_t nvec, int* lohi) {
+    int lo[kTables], hi[kTables];
+#pragma unroll
+    for (int t = 0; t < kTables; ++t) {
+        lo[t] = INT_MAX;
+        hi[t] = INT_MIN;
+    }
+    for (int64_t g = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; g < nvec; g += (int64_t)gridDim.x * blockDim.x) {
+        const int32_t* v = fields + kFields * g;
+        const int c = v[0];
+        lo[0] = min(lo[0], c);
+        hi[0] = max(hi[0], c);
+#pragma unroll
+        for (int k = 1; k < kFields; ++k) {
+            const int x = v[k];
+            // table 1 + 2(k - 1) + c, written without a dynamic index
+            if (c) {
+                lo[2 * k] = min(lo[2 * k], x);
+                hi[2 * k] = max(hi[2 * k], x);
+            } else {
+                lo[2 * k - 1] = min(lo[2 * k - 1], x);
+                hi[2 * k - 1] = max(hi[2 * k - 1], x);
+            }
+        }
+    }
+#pragma unroll
+    for (int t = 0; t < kTables; ++t) {
+        int a = lo[t], b = hi[t];
+        for (int o = 16; o > 0; o >>= 1) {
+            a = min(a, __shfl_xor_sync(0xFFFFFFFFu, a, o));
+            b = max(b, __shfl_xor_sync(0xFFFFFFFFu, b, o));
+        }
+        if ((threadIdx.x & 31) == 0) {
+            if (a != INT_MAX) atomicMin(lohi + t, a);
+            if (b != INT_MIN) atomicMax(lohi + kTables + t, b);
+        }
+    }
+}
+
+// Counts of every table's symbols over vectors [0, nvec): per-CTA shared histograms when the
+// tables' bins fit (nbins <= kSmemBins), global atomics otherwise.
+constexpr int kSmemBins = 12288;
+struct CountArgs {
+    int tmin[kTables];
+    uint32_t tbase[kTables];
+};
+__global__ void k_count(const int32_t* fields, int64_t nvec, CountArgs ca, uint32_t nbins, unsigned long long* counts) {
+    __shared__ uint32_t sh[kSmemBins];
+    const bool in_smem = nbins <= (uint32_t)kSmemBins;
+    if (in_smem)
+        for (uint32_t i = threadIdx.x; i < nbins; i += blockDim.x) sh[i] = 0;
+    __syncthreads();
+    for (int64_t g = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; g < nvec; g += (int64_t)gridDim.x * blockDim.x) {
+        const int32_t* v = fields + kFields * g;
+        const int c = v[0];
+#pragma unroll
+        for (int k = 0; k < kFields; ++k) {
+            const int t = table_index(k, c);
+            const uint32_t bin = ca.tbase[t] + (uint32_t)(v[k] - ca.tmin[t]);
+            if (in_smem) atomicAdd(sh + bin, 1u);
+            else atomicAdd(counts + bin, 1ull);
+        }
+    }
+    if (in_smem) {
+        __syncthreads();
+        for (uint32_t i = threadIdx.x; i < nbins; i += blockDim.x)
+            if (sh[i]) atomicAdd(counts + i, (unsigned long long)sh[i]);
+    }
+}
+
+// Row scales: the least-squares scale <w, y> / <y, y> over the real entries, sums in index
+// order (y = z + c/2 rebuilt from the fields), 0 for a zero denominator.
+__global__ void k_refit(const float* W, int64_t rows, int64_t cols, int64_t nq, const int32_t* fields, float* scales) {
+    const int64_t r = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (r >= rows) return;
+    const float* w = W + r * cols;
+    double sn = 0.0, sd = 0.0;
+    for (int64_t q = 0; q < nq; ++q) {
+        const int32_t* f = fields + kFields * (r * nq + q);
+        const int c = f[0];
+        double y[8];
+        long long s7 = 0;
+#pragma unroll
+        for (int k = 0; k < 7; ++k) {
+            y[k] = (double)f[1 + k] + 0.5 * c;
+            s7 += f[1 + k];
+        }
+        y[7] = (double)(2LL * f[8] + (s7 & 1LL)) + 0.5 * c;
+        const int64_t real = cols - 8 * q < 8 ? cols - 8 * q : 8;
+#pragma unroll
+        for (int k = 0; k < 8; ++k)
+            if (k < real) {
+                sn += (double)w[8 * q + k] * y[k];
+                sd += y[k] * y[k];
+            }
+    }
+    scales[r] = sd == 0.0 ? 0.0f : (float)(sn / sd);
+}
+
+// rANS, one warp per tile: lane j encodes the tile's lane j (vectors 32 r + j), steps in
+// reverse.  The host emits a step's words in descending lane order and reverses the whole
+// tile at the end; here lane j's word of a step goes to position n + (emitting lanes above j)
+// of the reversed stream, n the words emitted before the step (the copy-out reverses).
+struct RansArgs {
+    const uint32_t* freq;  // every table's frequencies, back to back from tbase
+    const uint32_t* cum;
+    int tmin[kTables];
+    uint32_t tbase[kTables];
+};
+__global__ void k_rans(const int32_t* fields, int64_t nvec, int64_t V, int64_t T, int b, RansArgs ra,
+                       uint16_t* scratch, uint32_t* nwords, uint32_t* states) {
+    const int64_t t = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+    if (t >= T) return;
+    const int j = threadIdx.x & 31;
+    const uint32_t above = j == 31 ? 0u : (0xFFFFFFFFu << (j + 1));
+    const int64_t v0 = t * V;
+    const int64_t vt = nvec - v0 < V ? nvec - v0 : V;
+    const int64_t rounds = (vt + kLanes - 1) / kLanes;
+    uint16_t* out = scratch + (size_t)t * (size_t)(kFields * V);
+    const uint32_t M = 1u << b;
+    uint32_t x = kStateLow, n = 0;
+    for (int64_t st = kFields * rounds - 1; st >= 0; --st) {
+        const int64_t r = st / kFields;
+        const int k = (int)(st - r * kFields);
+        const int64_t v = kLanes * r + j;
+        const bool act = v < vt;
+        bool emit = false;
+        uint32_t word = 0;
+        if (act) {
+            const int32_t* f = fields + kFields * (v0 + v);
+            const int tb = table_index(k, f[0]);
+            const uint32_t idx = ra.tbase[tb] + (uint32_t)(f[k] - ra.tmin[tb]);
+            const uint32_t fr = ra.freq[idx], cm = ra.cum[idx];
+            if (x >= (fr << (31 - b))) {
+                emit = true;
+                word = x & 0xFFFFu;
+                x >>= 16;
+            }
+            x = (x / fr) * M + (x % fr) + cm;
+        }
+        const uint32_t em = __ballot_sync(0xFFFFFFFFu, emit);
+        if (emit) out[n + __popc(em & above)] = (uint16_t)word;
+        n += __popc(em);
+    }
+    states[(size_t)t * kLanes + j] = x;
+    if (j == 0) nwords[t] = n;
+}
+
+// Tile t's words, reversed, to payload[off[t] ..).
+__global__ void k_copy_out(const uint16_t* scratch, int64_t V, const uint32_t* nwords, const uint32_t* off,
+                           uint16_t* payload) {
+    const int64_t t = blockIdx.x;
+    const uint32_t n = nwords[t];
+    const uint16_t* src = scratch + (size_t)t * (size_t)(kFields * V);
+    uint16_t* dst = payload + off[t];
+    for (uint32_t i = threadIdx.x; i < n; i += blockDim.x) dst[i] = src[n - 1 - i];
+}
+
+// ------------------------------------------------------------- host side
+
+// Device buffers freed on every exit path.
+struct DevBuf {
+    void* p = nullptr;
+    ~DevBuf() {
+        if (p) cudaFree(p);
+    }
+    template <typename T>
+    T* as() const {
+        return static_cast<T*>(p);
+    }
+    cudaError_t alloc(size_t bytes) { return cudaMalloc(&p, bytes > 0 ? bytes : 16); }
+};
+
+int grid_for(int64_t n, int threads) { return (int)std::max<int64_t>(1, (n + threads - 1) / threads); }
+
+struct GpuEncoder {
+    cudaStream_t st;
+    int nsm = 148;
+    const float* W;
+    int64_t rows, cols, nq, nvec;
+    DevBuf d_lohi, d_counts;
+
+    cudaError_t alphabet(const int32_t* f, int64_t n, Hist& al) {
+        int init[2 * kTables];
+        for (int t = 0; t < kTables; ++t) {
+            init[t] = INT_MAX;
+            init[kTables + t] = INT_MIN;
+        }
+        cudaError_t e = cudaMemcpyAsync(d_lohi.p, init, sizeof(init), cudaMemcpyHostToDevice, st);
+        if (e != cudaSuccess) return e;
+        k_alphabet<<<std::min(grid_for(n, 256), 8 * nsm), 256, 0, st>>>(f, n, d_lohi.as<int>());
+        int got[2 * kTables];
+        e = cudaMemcpyAsync(got, d_lohi.p, sizeof(got), cudaMemcpyDeviceToHost, st);
+        if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+        if (e != cudaSuccess) return e;
+        al.reset();
+        for (int t = 0; t < kTables; ++t) {
+            if (got[t] == INT_MAX) continue;  // an empty table
+            al.lo[t] = got[t];
+            al.hi[t] = got[kTables + t];
+        }
+        return cudaSuccess;
+    }
+
+    // counts of vectors [0, n) into tables laid out like the CPU packer's count_fields
+    cudaError_t count(const int32_t* f, int64_t n, const Hist& al, Table* tabs) {
+        CountArgs ca;
+        uint32_t nb = 0;
+        for (int t = 0; t < kTables; ++t) {
+            tabs[t].A = (uint32_t)al.alpha(t);
+            tabs[t].min = tabs[t].A ? (int32_t)al.lo[t] : 0;
+            tabs[t].total = 0;
+            tabs[t].count.assign(std::max<uint32_t>(tabs[t].A, 1), 0);
+            ca.tmin[t] = tabs[t].min;
+            ca.tbase[t] = nb;
+            nb += (uint32_t)tabs[t].count.size();
+        }
+        DevBuf d;
+        cudaError_t e = d.alloc(sizeof(unsigned long long) * nb);
+        if (e == cudaSuccess) e = cudaMemsetAsync(d.p, 0, sizeof(unsigned long long) * nb, st);
+        if (e != cudaSuccess) return e;
+        k_count<<<std::min(grid_for(n, 256), 4 * nsm), 256, 0, st>>>(f, n, ca, nb, d.as<unsigned long long>());
+        std::vector<unsigned long long> h(nb);
+        e = cudaMemcpyAsync(h.data(), d.p, sizeof(unsigned long long) * nb, cudaMemcpyDeviceToHost, st);
+        if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+        if (e != cudaSuccess) return e;
+        for (int t = 0; t < kTables; ++t) {
+            for (size_t s = 0; s < tabs[t].count.size(); ++s) {
+                tabs[t].count[s] = h[ca.tbase[t] + s];
+                tabs[t].total += h[ca.tbase[t] + s];
+            }
+        }
+        return cudaSuccess;
+    }
+
+    cudaError_t quantize(const double* norms, const int64_t* rowlist, int64_t nr, double s, int32_t* f) {
+        k_quantize<<<grid_for(nr * nq, kQThreads), kQThreads, 0, st>>>(W, cols, nq, norms, rowlist, nr, s, f);
+        return cudaGetLastError();
+    }
+};
+
+}  // namespace
+}  // namespace ep
+
+extern "C" ep_status ep_encode_tensor_gpu(void* stream, const float* W, int64_t rows, int64_t cols,
+                                          double target_bpp, const ep_encode_opts* opts, ep_blob** out) {
+    using namespace ep;
+    if (!W || !out) return EP_EINVAL;
+    *out = nullptr;
+    if (rows <= 0 || cols <= 0 || !(target_bpp > 0.0)) return EP_EINVAL;
+    if ((reinterpret_cast<uintptr_t>(W) & 3u) != 0) return EP_EINVAL;
+    ep_encode_opts o{};
+    if (opts) o = *opts;
+    if (o.rdo_candidates > 1) return EP_EUNSUPPORTED;  // the per-row refinement stays on the CPU packer
+    int b = o.prob_bits > 0 ? o.prob_bits : (target_bpp <= 7.0 ? 11 : 12);
+    if (b < kMinB || b > kMaxB) return EP_EINVAL;
+    const int64_t nq = (cols + 7) / 8, nvec = rows * nq;
+    if (nvec >= (1ll << 31)) return EP_EINVAL;
+    const int64_t V = o.tile_vectors > 0 ? o.tile_vectors : std::max<int64_t>(32, host::tile_symbols_for(target_bpp) / 9);
+    const int64_t T = (nvec + V - 1) / V;
+    if (T >= (1ll << 31) / kTileWords) return EP_EINVAL;
+    const bool container = o.has_container_scales != 0;
+
+    try {
+        GpuEncoder g;
+        g.st = static_cast<cudaStream_t>(stream);
+        g.W = W;
+        g.rows = rows;
+        g.cols = cols;
+        g.nq = nq;
+        g.nvec = nvec;
+        int dev = 0;
+        if (cudaGetDevice(&dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&g.nsm, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+            return EP_ECUDA;
+        const cudaStream_t st = g.st;
+        DevBuf d_norms, d_srows, d_sf, d_fields, d_scales;
+        if (g.d_lohi.alloc(sizeof(int) * 2 * kTables) != cudaSuccess || d_norms.alloc(sizeof(double) * rows) ||
+            d_fields.alloc(sizeof(int32_t) * kFields * (size_t)nvec) || d_scales.alloc(sizeof(float) * rows))
+            return EP_ECUDA;
+        k_norms<<<grid_for(rows, 128), 128, 0, st>>>(W, rows, cols, d_norms.as<double>());
+
+        const std::vector<int64_t> srows = host::sample_rows(rows, cols, o);
+        const int64_t rs = (int64_t)srows.size(), ns = rs * nq;
+        if (d_srows.alloc(sizeof(int64_t) * rs) || d_sf.alloc(sizeof(int32_t) * kFields * (size_t)ns)) return EP_ECUDA;
+        if (cudaMemcpyAsync(d_srows.p, srows.data(), sizeof(int64_t) * rs, cudaMemcpyHostToDevice, st) != cudaSuccess)
+            return EP_ECUDA;
+
+        auto estimate = [&](double s, double& est) -> cudaError_t {
+            cudaError_t e = g.quantize(d_norms.as<double>(), d_srows.as<int64_t>(), rs, s, d_sf.as<int32_t>());
+            Hist al;
+            if (e == cudaSuccess) e = g.alphabet(d_sf.as<int32_t>(), ns, al);
+            if (e != cudaSuccess) return e;
+            if (al.amax_coord() > (1ull << b)) {
+                est = INFINITY;
+                return cudaSuccess;
+            }
+            Table tabs[kTables];
+            e = g.count(d_sf.as<int32_t>(), ns, al, tabs);
+            if (e == cudaSuccess) est = host::estimate_bpp(tabs, al, b, nvec, ns, T, rows, cols, container);
+            return e;
+        };
+        auto quantize_all = [&](double s, Hist& al) -> cudaError_t {
+            cudaError_t e = g.quantize(d_norms.as<double>(), nullptr, rows, s, d_fields.as<int32_t>());
+            return e == cudaSuccess ? g.alphabet(d_fields.as<int32_t>(), nvec, al) : e;
+        };
+
+        // the scale search and the b escalation, decided on the host as in the CPU packer
+        const int steps = o.search_steps > 0 ? o.search_steps : 12;
+        double s = 1.0;
+        Hist al;
+        for (;;) {
+            double lo = 1e-3, hi = 8.0;
+            for (int it = 0; it < steps; ++it) {
+                s = std::sqrt(lo * hi);
+                double est = 0.0;
+                if (estimate(s, est) != cudaSuccess) return EP_ECUDA;
+                if (est > target_bpp) lo = s;
+                else hi = s;
+            }
+            s = std::sqrt(lo * hi);
+            if (quantize_all(s, al) != cudaSuccess) return EP_ECUDA;
+            if (al.amax_coord() <= (1ull << b)) break;
+            if (b < kMaxB) {
+                ++b;
+                continue;
+            }
+            while (al.amax_coord() > (1ull << b)) {
+                s = 1.05 * s * (double)al.amax_coord() / (double)(1u << b);
+                if (quantize_all(s, al) != cudaSuccess) return EP_ECUDA;
+            }
+            break;
+        }
+        k_refit<<<grid_for(rows, 128), 128, 0, st>>>(W, rows, cols, nq, d_fields.as<int32_t>(), d_scales.as<float>());
+
+        Table tabs[kTables];
+        if (g.count(d_fields.as<int32_t>(), nvec, al, tabs) != cudaSuccess) return EP_ECUDA;
+        for (int t = 0; t < kTables; ++t) {
+            if (tabs[t].A > (1u << b)) return EP_EALPHABET;
+            host::normalise(tabs[t], b);
+        }
+
+        // rANS: the tables to the device, a warp per tile into scratch, then the words in order
+        RansArgs ra;
+        std::vector<uint32_t> hf, hc;
+        for (int t = 0; t < kTables; ++t) {
+            ra.tmin[t] = tabs[t].min;
+            ra.tbase[t] = (uint32_t)hf.size();
+            for (size_t k = 0; k < tabs[t].freq.size(); ++k) {
+                hf.push_back(tabs[t].freq[k]);
+                hc.push_back(tabs[t].cum[k]);
+            }
+        }
+        DevBuf d_freq, d_cum, d_scratch, d_nwords, d_states, d_off, d_payload;
+        if (d_freq.alloc(4 * hf.size()) || d_cum.alloc(4 * hc.size()) ||
+            d_scratch.alloc(sizeof(uint16_t) * (size_t)kFields * (size_t)V * (size_t)T) || d_nwords.alloc(4 * T) ||
+            d_states.alloc(sizeof(uint32_t) * kLanes * (size_t)T) || d_off.alloc(4 * T))
+            return EP_ECUDA;
+        if (cudaMemcpyAsync(d_freq.p, hf.data(), 4 * hf.size(), cudaMemcpyHostToDevice, st) ||
+            cudaMemcpyAsync(d_cum.p, hc.data(), 4 * hc.size(), cudaMemcpyHostToDevice, st))
+            return EP_ECUDA;
+        ra.freq = d_freq.as<uint32_t>();
+        ra.cum = d_cum.as<uint32_t>();
+        k_rans<<<grid_for(T * 32, 128), 128, 0, st>>>(d_fields.as<int32_t>(), nvec, V, T, b, ra,
+                                                      d_scratch.as<uint16_t>(), d_nwords.as<uint32_t>(),
+                                                      d_states.as<uint32_t>());
+        std::vector<uint32_t> nw((size_t)T), off((size_t)T);
+        if (cudaMemcpyAsync(nw.data(), d_nwords.p, 4 * T, cudaMemcpyDeviceToHost, st) ||
+            cudaStreamSynchronize(st))
+            return EP_ECUDA;
+        uint64_t words = 0;
+        for (int64_t t = 0; t < T; ++t) {
+            if (words >= 0xFFFFFFFFull) return EP_EINVAL;
+            off[t] = (uint32_t)words;
+            words += nw[t];
+        }
+        if (words > 0xFFFFFFFFull) return EP_EINVAL;
+        if (d_payload.alloc(sizeof(uint16_t) * std::max<uint64_t>(words, 1)) ||
+            cudaMemcpyAsync(d_off.p, off.data(), 4 * T, cudaMemcpyHostToDevice, st))
+            return EP_ECUDA;
+        k_copy_out<<<(unsigned)T, 256, 0, st>>>(d_scratch.as<uint16_t>(), V, d_nwords.as<uint32_t>(),
+                                                d_off.as<uint32_t>(), d_payload.as<uint16_t>());
+
+        ep_blob* bl = host::new_blob(rows, cols, b, V, T, words, tabs);
+        if (!bl) return EP_ENOMEM;
+        std::vector<uint32_t> states((size_t)kLanes * T);
+        cudaError_t e = cudaMemcpyAsync(bl->payload, d_payload.p, 2 * words, cudaMemcpyDeviceToHost, st);
+        if (e == cudaSuccess)
+            e = cudaMemcpyAsync(states.data(), d_states.p, 4 * states.size(), cudaMemcpyDeviceToHost, st);
+        if (e == cudaSuccess)
+            e = cudaMemcpyAsync(bl->row_scales, d_scales.p, sizeof(float) * rows, cudaMemcpyDeviceToHost, st);
+        if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+        if (e != cudaSuccess) {
+            ep_free_blob(bl);
+            return EP_ECUDA;
+        }
+        for (int64_t t = 0; t < T; ++t) {
+            bl->tile_index[kTileWords * t] = off[t];
+            for (int j = 0; j < kLanes; ++j) bl->tile_index[kTileWords * t + 1 + j] = states[(size_t)kLanes * t + j];
+        }
+        bl->tile_index[kTileWords * T] = (uint32_t)words;
+        host::finish_blob(bl, s, container);
+        *out = bl;
+        return EP_OK;
+    } catch (const std::bad_alloc&) {
+        return EP_ENOMEM;
+    }
+}

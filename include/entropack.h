@@ -114,7 +114,29 @@ typedef struct {
 ep_status ep_encode_tensor(const float* W, int64_t rows, int64_t cols, double target_bpp,
                            const ep_encode_opts* opts, ep_blob** out);
 
-/* Free a blob returned by ep_encode_tensor (NULL is allowed). */
+/*
+ * ep_encode_tensor_gpu -- the packer of ep_encode_tensor with its full-tensor
+ * stages on the GPU: row normalisation, the quantisation of the sampled rows
+ * for every step of the scale search and of the whole tensor, the symbol
+ * counts, the row-scale refit and the tiled rANS (one warp per tile).  The
+ * search's decisions, the table normalisation and the header stay on the host.
+ * The blob is byte for byte the one ep_encode_tensor returns for the same
+ * matrix and options: every floating-point step is the host's operation in the
+ * host's order, without multiply-add contraction, and the estimates' bits come
+ * from exact counts (paper §3.1 pipeline; §3.4, §3.5, §3.6, App. C.1, C.3).
+ *   stream  cudaStream_t to launch on (the call synchronises it several times).
+ *   W       device, float32 [rows, cols] row-major, 4-byte aligned; not modified.
+ *   opts    as ep_encode_tensor; num_threads is ignored and rdo_candidates > 1
+ *           (the per-row refinement) returns EP_EUNSUPPORTED.
+ * Scratch is allocated with cudaMalloc and freed before the call returns (about
+ * 36 + 18 bytes per vector of eight weights).  On EP_OK *out holds a host blob
+ * (free with ep_free_blob).  Errors: EP_EINVAL, EP_EUNSUPPORTED, EP_EALPHABET,
+ * EP_ENOMEM, EP_ECUDA.
+ */
+ep_status ep_encode_tensor_gpu(void* stream, const float* W, int64_t rows, int64_t cols, double target_bpp,
+                               const ep_encode_opts* opts, ep_blob** out);
+
+/* Free a blob returned by ep_encode_tensor or ep_encode_tensor_gpu (NULL is allowed). */
 void ep_free_blob(ep_blob* blob);
 
 /*

@@ -108,3 +108,24 @@ def test_encode_rejects_bad_arguments(lib):
         ep.encode_tensor(W, 4.0, prob_bits=16)
     with pytest.raises(ep.EntroPackError):
         ep.encode_tensor(W, 4.0, prob_bits=8)
+
+
+def test_gpu_encoder_refuses_bad_arguments_on_host(lib):
+    """Every case is refused before any CUDA call (a fake device pointer never reaches a kernel)."""
+    EINVAL, EUNSUP = ep._lib.STATUS_CODES["EP_EINVAL"], ep._lib.STATUS_CODES["EP_EUNSUPPORTED"]
+    good = C.c_void_p(0x10000)
+    out = C.POINTER(ep._lib._Blob)()
+
+    def call(W=good, rows=64, cols=64, bpp=4.0, **kw):
+        o = ep._lib._Opts(kw.get("prob_bits", 0), 0, 0, 0, 0, 0, 0, kw.get("rdo", 0), 0)
+        return lib.ep_encode_tensor_gpu(None, W, rows, cols, bpp, C.byref(o), C.byref(out))
+
+    assert call(W=None) == EINVAL
+    assert call(rows=0) == EINVAL
+    assert call(cols=-1) == EINVAL
+    assert call(bpp=0.0) == EINVAL
+    assert call(W=C.c_void_p(0x10002)) == EINVAL      # not 4-byte aligned
+    assert call(prob_bits=16) == EINVAL
+    assert call(prob_bits=8) == EINVAL
+    assert call(rdo=4) == EUNSUP                        # the per-row refinement stays on the CPU packer
+    assert call(rows=1 << 20, cols=1 << 14) == EINVAL  # 2^31 vectors
