@@ -4,8 +4,8 @@
 // search (§3.4, App. C.1), full-tensor E8 quantisation (§1, Conway & Sloane 1982), the row-scale
 // refit (§3.5), the seventeen coset-conditioned tables (§3.6, App. A.3) and tiled interleaved
 // rANS (§3.6, App. C.3).  The result is byte for byte the CPU packer's blob:
-//   - every floating-point step is the host's operation in the host's order (one thread per
-//     row for the row sums, taken in index order), and this file is compiled without
+//   - every floating-point step is the host's operation in the host's order (each row's sums
+//     are taken in column order), and this file is compiled without
 //     multiply-add contraction (-fmad=false), so each product and sum rounds as on the host;
 //     division, square root and rint are IEEE round-to-nearest on both sides;
 //   - the search's estimates come from exact integer counts made here and turned into bits on
@@ -20,6 +20,7 @@
 
 #include <algorithm>
 #include <climits>
+#include <mutex>
 #include <cmath>
 #include <new>
 #include <vector>
@@ -91,15 +92,56 @@ __device__ __forceinline__ void e8_fields(const double (&u)[8], int32_t* f) {
 
 // ----------------------------------------------------------------- kernels
 
+// Per-row sums in column order: a warp owns 32 rows (lane i adds row r0 + i, so every row's sum
+// is the host's sequential sum).  Columns go in chunks of 32, copied (lane = column, coalesced)
+// by cp.async into a ring of shared-memory slots kept kDepth chunks ahead, so the loads stay in
+// flight without holding registers while each lane adds its row's 32 entries from the slot.
+__device__ __forceinline__ void cp_async4(void* dst, const void* src) {
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"((uint32_t)__cvta_generic_to_shared(dst)),
+                 "l"(src)
+                 : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+    asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+
 // Row normaliser: the RMS of the row (a sum of squares in index order), 1 for a zero row.
-__global__ void k_norms(const float* W, int64_t rows, int64_t cols, double* norms) {
-    const int64_t r = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-    if (r >= rows) return;
-    const float* w = W + r * cols;
+constexpr int kNormDepth = 8;
+__global__ void __launch_bounds__(32) k_norms(const float* W, int64_t rows, int64_t cols, double* norms) {
+    __shared__ float ring[kNormDepth][32][33];
+    const int lane = threadIdx.x & 31;
+    const int64_t r0 = (int64_t)blockIdx.x * 32;
+    const int nr = rows - r0 < 32 ? (int)(rows - r0) : 32;
+    const int64_t nch = (cols + 31) / 32;
+    auto issue = [&](int64_t c) {
+        if (c < nch) {
+            const int64_t col = 32 * c + lane;
+            if (col < cols)
+                for (int rr = 0; rr < nr; ++rr) cp_async4(&ring[c % kNormDepth][rr][lane], W + (r0 + rr) * cols + col);
+        }
+        cp_async_commit();  // an empty group past the end keeps the group count in step
+    };
+    for (int64_t c = 0; c < kNormDepth - 1; ++c) issue(c);
     double acc = 0.0;
-    for (int64_t j = 0; j < cols; ++j) acc += (double)w[j] * (double)w[j];
-    const double n = sqrt(acc / (double)cols);
-    norms[r] = n > 0.0 ? n : 1.0;
+    for (int64_t c = 0; c < nch; ++c) {
+        issue(c + kNormDepth - 1);
+        cp_async_wait<kNormDepth - 1>();  // chunk c has landed (this lane's copies)
+        __syncwarp();                     // and every lane's
+        const int n = cols - 32 * c < 32 ? (int)(cols - 32 * c) : 32;
+        const float* src = &ring[c % kNormDepth][lane][0];
+        for (int k = 0; k < n; ++k) {
+            const double w = (double)src[k];
+            acc += w * w;
+        }
+        __syncwarp();  // the slot is refilled by the next iteration's copies
+    }
+    cp_async_wait<0>();
+    if (lane < nr) {
+        const double n = sqrt(acc / (double)cols);
+        norms[r0 + lane] = n > 0.0 ? n : 1.0;
+    }
 }
 
 // Fields of vectors [0, nrows * nq) at scale s: vector (i, q) is vector q of row rowlist[i]
@@ -191,32 +233,58 @@ __global__ void k_count(const int32_t* fields, int64_t nvec, CountArgs ca, uint3
 }
 
 // Row scales: the least-squares scale <w, y> / <y, y> over the real entries, sums in index
-// order (y = z + c/2 rebuilt from the fields), 0 for a zero denominator.
-__global__ void k_refit(const float* W, int64_t rows, int64_t cols, int64_t nq, const int32_t* fields, float* scales) {
-    const int64_t r = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-    if (r >= rows) return;
-    const float* w = W + r * cols;
-    double sn = 0.0, sd = 0.0;
-    for (int64_t q = 0; q < nq; ++q) {
-        const int32_t* f = fields + kFields * (r * nq + q);
-        const int c = f[0];
-        double y[8];
-        long long s7 = 0;
-#pragma unroll
-        for (int k = 0; k < 7; ++k) {
-            y[k] = (double)f[1 + k] + 0.5 * c;
-            s7 += f[1 + k];
-        }
-        y[7] = (double)(2LL * f[8] + (s7 & 1LL)) + 0.5 * c;
-        const int64_t real = cols - 8 * q < 8 ? cols - 8 * q : 8;
-#pragma unroll
-        for (int k = 0; k < 8; ++k)
-            if (k < real) {
-                sn += (double)w[8 * q + k] * y[k];
-                sd += y[k] * y[k];
+// order (y = z + c/2 rebuilt from the fields), 0 for a zero denominator.  Same ring as k_norms,
+// with the fields of the chunk's four vectors (36 words a row) beside its 32 weights.
+constexpr int kRefitDepth = 4;
+__global__ void __launch_bounds__(32) k_refit(const float* W, int64_t rows, int64_t cols, int64_t nq,
+                                               const int32_t* fields, float* scales) {
+    __shared__ float rw[kRefitDepth][32][33];
+    __shared__ int32_t rf[kRefitDepth][32][37];
+    const int lane = threadIdx.x & 31;
+    const int64_t r0 = (int64_t)blockIdx.x * 32;
+    const int nr = rows - r0 < 32 ? (int)(rows - r0) : 32;
+    const int64_t nch = (cols + 31) / 32;
+    auto issue = [&](int64_t c) {
+        if (c < nch) {
+            const int slot = (int)(c % kRefitDepth);
+            const int64_t col = 32 * c + lane;
+            const int64_t nv = nq - 4 * c < 4 ? nq - 4 * c : 4;  // vectors of this chunk
+            for (int rr = 0; rr < nr; ++rr) {
+                if (col < cols) cp_async4(&rw[slot][rr][lane], W + (r0 + rr) * cols + col);
+                const int32_t* f = fields + kFields * ((r0 + rr) * nq + 4 * c);
+                if (lane < kFields * nv) cp_async4(&rf[slot][rr][lane], f + lane);
+                if (lane + 32 < kFields * nv) cp_async4(&rf[slot][rr][lane + 32], f + lane + 32);
             }
+        }
+        cp_async_commit();
+    };
+    for (int64_t c = 0; c < kRefitDepth - 1; ++c) issue(c);
+    double sn = 0.0, sd = 0.0;
+    for (int64_t c = 0; c < nch; ++c) {
+        issue(c + kRefitDepth - 1);
+        cp_async_wait<kRefitDepth - 1>();
+        __syncwarp();
+        const int slot = (int)(c % kRefitDepth);
+        const int n = cols - 32 * c < 32 ? (int)(cols - 32 * c) : 32;
+        const float* w = &rw[slot][lane][0];
+        const int32_t* f = &rf[slot][lane][0];
+        for (int k0 = 0; k0 < n; k0 += 8) {
+            const int32_t* v = f + kFields * (k0 >> 3);
+            const double half_c = 0.5 * v[0];
+            long long s7 = 0;
+            for (int k = 0; k < 7; ++k) s7 += v[1 + k];
+            const int m = n - k0 < 8 ? n - k0 : 8;
+            for (int k = 0; k < m; ++k) {
+                const long long z = k < 7 ? (long long)v[1 + k] : 2LL * v[8] + (s7 & 1LL);
+                const double y = (double)z + half_c;
+                sn += (double)w[k0 + k] * y;
+                sd += y * y;
+            }
+        }
+        __syncwarp();
     }
-    scales[r] = sd == 0.0 ? 0.0f : (float)(sn / sd);
+    cp_async_wait<0>();
+    if (lane < nr) scales[r0 + lane] = sd == 0.0 ? 0.0f : (float)(sn / sd);
 }
 
 // rANS, one warp per tile: lane j encodes the tile's lane j (vectors 32 r + j), steps in
@@ -280,36 +348,71 @@ __global__ void k_copy_out(const uint16_t* scratch, int64_t V, const uint32_t* n
 
 // ------------------------------------------------------------- host side
 
-// Device buffers freed on every exit path.
+// The encoder's scratch comes from a memory pool of the library's own, stream-ordered, which
+// keeps up to kPoolKeep bytes between calls (no device-wide synchronisation per allocation).
+constexpr uint64_t kPoolKeep = 1ull << 30;
+std::mutex g_pool_mu;
+cudaMemPool_t g_pool[64] = {};
+
+cudaError_t pool_of(int dev, cudaMemPool_t& out) {
+    std::lock_guard<std::mutex> lk(g_pool_mu);
+    if (!g_pool[dev]) {
+        cudaMemPoolProps pp = {};
+        pp.allocType = cudaMemAllocationTypePinned;
+        pp.location.type = cudaMemLocationTypeDevice;
+        pp.location.id = dev;
+        cudaError_t e = cudaMemPoolCreate(&g_pool[dev], &pp);
+        if (e != cudaSuccess) return e;
+        uint64_t keep = kPoolKeep;
+        e = cudaMemPoolSetAttribute(g_pool[dev], cudaMemPoolAttrReleaseThreshold, &keep);
+        if (e != cudaSuccess) return e;
+    }
+    out = g_pool[dev];
+    return cudaSuccess;
+}
+
+// A device buffer from the pool, released in stream order on every exit path.
 struct DevBuf {
     void* p = nullptr;
+    cudaStream_t st = nullptr;
+    static thread_local cudaMemPool_t pool;  // the calling thread's device's pool, set per call
     ~DevBuf() {
-        if (p) cudaFree(p);
+        if (p) cudaFreeAsync(p, st);
     }
     template <typename T>
     T* as() const {
         return static_cast<T*>(p);
     }
-    cudaError_t alloc(size_t bytes) { return cudaMalloc(&p, bytes > 0 ? bytes : 16); }
+    cudaError_t alloc(size_t bytes, cudaStream_t s) {
+        st = s;
+        return cudaMallocFromPoolAsync(&p, bytes > 0 ? bytes : 16, pool, s);
+    }
 };
+thread_local cudaMemPool_t DevBuf::pool = nullptr;
+
+__global__ void k_lohi_init(int* lohi) {
+    const int t = threadIdx.x;
+    if (t < kTables) {
+        lohi[t] = INT_MAX;
+        lohi[kTables + t] = INT_MIN;
+    }
+}
 
 int grid_for(int64_t n, int threads) { return (int)std::max<int64_t>(1, (n + threads - 1) / threads); }
+
+// the most bins a count needs: 16 coordinate tables of at most 2^15 symbols, the coset table's 2
+constexpr uint32_t kMaxBins = 16u * 32768u + 2u;
 
 struct GpuEncoder {
     cudaStream_t st;
     int nsm = 148;
     const float* W;
     int64_t rows, cols, nq, nvec;
-    DevBuf d_lohi, d_counts;
+    DevBuf d_lohi, d_counts;  // (the counts buffer holds kMaxBins)
 
     cudaError_t alphabet(const int32_t* f, int64_t n, Hist& al) {
-        int init[2 * kTables];
-        for (int t = 0; t < kTables; ++t) {
-            init[t] = INT_MAX;
-            init[kTables + t] = INT_MIN;
-        }
-        cudaError_t e = cudaMemcpyAsync(d_lohi.p, init, sizeof(init), cudaMemcpyHostToDevice, st);
-        if (e != cudaSuccess) return e;
+        k_lohi_init<<<1, 32, 0, st>>>(d_lohi.as<int>());
+        cudaError_t e;
         k_alphabet<<<std::min(grid_for(n, 256), 8 * nsm), 256, 0, st>>>(f, n, d_lohi.as<int>());
         int got[2 * kTables];
         e = cudaMemcpyAsync(got, d_lohi.p, sizeof(got), cudaMemcpyDeviceToHost, st);
@@ -337,13 +440,12 @@ struct GpuEncoder {
             ca.tbase[t] = nb;
             nb += (uint32_t)tabs[t].count.size();
         }
-        DevBuf d;
-        cudaError_t e = d.alloc(sizeof(unsigned long long) * nb);
-        if (e == cudaSuccess) e = cudaMemsetAsync(d.p, 0, sizeof(unsigned long long) * nb, st);
+        if (nb > kMaxBins) return cudaErrorInvalidValue;  // alphabets are checked against 2^b first
+        cudaError_t e = cudaMemsetAsync(d_counts.p, 0, sizeof(unsigned long long) * nb, st);
         if (e != cudaSuccess) return e;
-        k_count<<<std::min(grid_for(n, 256), 4 * nsm), 256, 0, st>>>(f, n, ca, nb, d.as<unsigned long long>());
+        k_count<<<std::min(grid_for(n, 256), 4 * nsm), 256, 0, st>>>(f, n, ca, nb, d_counts.as<unsigned long long>());
         std::vector<unsigned long long> h(nb);
-        e = cudaMemcpyAsync(h.data(), d.p, sizeof(unsigned long long) * nb, cudaMemcpyDeviceToHost, st);
+        e = cudaMemcpyAsync(h.data(), d_counts.p, sizeof(unsigned long long) * nb, cudaMemcpyDeviceToHost, st);
         if (e == cudaSuccess) e = cudaStreamSynchronize(st);
         if (e != cudaSuccess) return e;
         for (int t = 0; t < kTables; ++t) {
@@ -396,15 +498,18 @@ extern "C" ep_status ep_encode_tensor_gpu(void* stream, const float* W, int64_t 
             cudaDeviceGetAttribute(&g.nsm, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
             return EP_ECUDA;
         const cudaStream_t st = g.st;
+        if (pool_of(dev, DevBuf::pool) != cudaSuccess) return EP_ECUDA;
         DevBuf d_norms, d_srows, d_sf, d_fields, d_scales;
-        if (g.d_lohi.alloc(sizeof(int) * 2 * kTables) != cudaSuccess || d_norms.alloc(sizeof(double) * rows) ||
-            d_fields.alloc(sizeof(int32_t) * kFields * (size_t)nvec) || d_scales.alloc(sizeof(float) * rows))
+        if (g.d_lohi.alloc(sizeof(int) * 2 * kTables, st) != cudaSuccess ||
+            g.d_counts.alloc(sizeof(unsigned long long) * kMaxBins, st) || d_norms.alloc(sizeof(double) * rows, st) ||
+            d_fields.alloc(sizeof(int32_t) * kFields * (size_t)nvec, st) || d_scales.alloc(sizeof(float) * rows, st))
             return EP_ECUDA;
-        k_norms<<<grid_for(rows, 128), 128, 0, st>>>(W, rows, cols, d_norms.as<double>());
+        k_norms<<<grid_for(rows, 32), 32, 0, st>>>(W, rows, cols, d_norms.as<double>());
 
         const std::vector<int64_t> srows = host::sample_rows(rows, cols, o);
         const int64_t rs = (int64_t)srows.size(), ns = rs * nq;
-        if (d_srows.alloc(sizeof(int64_t) * rs) || d_sf.alloc(sizeof(int32_t) * kFields * (size_t)ns)) return EP_ECUDA;
+        if (d_srows.alloc(sizeof(int64_t) * rs, st) || d_sf.alloc(sizeof(int32_t) * kFields * (size_t)ns, st))
+            return EP_ECUDA;
         if (cudaMemcpyAsync(d_srows.p, srows.data(), sizeof(int64_t) * rs, cudaMemcpyHostToDevice, st) != cudaSuccess)
             return EP_ECUDA;
 
@@ -453,7 +558,7 @@ extern "C" ep_status ep_encode_tensor_gpu(void* stream, const float* W, int64_t 
             }
             break;
         }
-        k_refit<<<grid_for(rows, 128), 128, 0, st>>>(W, rows, cols, nq, d_fields.as<int32_t>(), d_scales.as<float>());
+        k_refit<<<grid_for(rows, 32), 32, 0, st>>>(W, rows, cols, nq, d_fields.as<int32_t>(), d_scales.as<float>());
 
         Table tabs[kTables];
         if (g.count(d_fields.as<int32_t>(), nvec, al, tabs) != cudaSuccess) return EP_ECUDA;
@@ -474,9 +579,10 @@ extern "C" ep_status ep_encode_tensor_gpu(void* stream, const float* W, int64_t 
             }
         }
         DevBuf d_freq, d_cum, d_scratch, d_nwords, d_states, d_off, d_payload;
-        if (d_freq.alloc(4 * hf.size()) || d_cum.alloc(4 * hc.size()) ||
-            d_scratch.alloc(sizeof(uint16_t) * (size_t)kFields * (size_t)V * (size_t)T) || d_nwords.alloc(4 * T) ||
-            d_states.alloc(sizeof(uint32_t) * kLanes * (size_t)T) || d_off.alloc(4 * T))
+        if (d_freq.alloc(4 * hf.size(), st) || d_cum.alloc(4 * hc.size(), st) ||
+            d_scratch.alloc(sizeof(uint16_t) * (size_t)kFields * (size_t)V * (size_t)T, st) ||
+            d_nwords.alloc(4 * T, st) || d_states.alloc(sizeof(uint32_t) * kLanes * (size_t)T, st) ||
+            d_off.alloc(4 * T, st))
             return EP_ECUDA;
         if (cudaMemcpyAsync(d_freq.p, hf.data(), 4 * hf.size(), cudaMemcpyHostToDevice, st) ||
             cudaMemcpyAsync(d_cum.p, hc.data(), 4 * hc.size(), cudaMemcpyHostToDevice, st))
@@ -497,7 +603,7 @@ extern "C" ep_status ep_encode_tensor_gpu(void* stream, const float* W, int64_t 
             words += nw[t];
         }
         if (words > 0xFFFFFFFFull) return EP_EINVAL;
-        if (d_payload.alloc(sizeof(uint16_t) * std::max<uint64_t>(words, 1)) ||
+        if (d_payload.alloc(sizeof(uint16_t) * std::max<uint64_t>(words, 1), st) ||
             cudaMemcpyAsync(d_off.p, off.data(), 4 * T, cudaMemcpyHostToDevice, st))
             return EP_ECUDA;
         k_copy_out<<<(unsigned)T, 256, 0, st>>>(d_scratch.as<uint16_t>(), V, d_nwords.as<uint32_t>(),
