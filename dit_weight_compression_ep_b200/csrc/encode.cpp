@@ -529,7 +529,10 @@ ep_blob* new_blob(int64_t rows, int64_t cols, int b, int64_t V, int64_t T, uint6
     bl->ntiles = (int)T;
     bl->payload_words = words;
     bl->payload_alloc_words = (words + 7) / 8 * 8;
-    bl->payload = (uint16_t*)std::calloc(std::max<size_t>(bl->payload_alloc_words, 8), sizeof(uint16_t));
+    // the caller writes words [0, words); only the padding up to a multiple of 8 words is zeroed here
+    const size_t alloc_words = std::max<size_t>(bl->payload_alloc_words, 8);
+    bl->payload = (uint16_t*)std::malloc(alloc_words * sizeof(uint16_t));
+    if (bl->payload) std::memset(bl->payload + words, 0, (alloc_words - words) * sizeof(uint16_t));
     bl->tile_index = (uint32_t*)std::malloc(sizeof(uint32_t) * (size_t)(kTileWords * T + 1));
     int64_t nf = 0;
     for (int t = 0; t < kTables; ++t) nf += tabs[t].A;

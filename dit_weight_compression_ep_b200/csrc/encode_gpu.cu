@@ -162,7 +162,8 @@ __global__ void k_quantize(const float* W, int64_t cols, int64_t nq, const doubl
 }
 
 // [min, max] of every table's symbols over vectors [0, nvec) (lohi: 17 minima, then 17 maxima).
-__global__ void k_alphabet(const int32_t* fields, int64_t nvec, int* lohi) {
+constexpr int kAlphaWarps = 8;
+__global__ void __launch_bounds__(32 * kAlphaWarps) k_alphabet(const int32_t* fields, int64_t nvec, int* lohi) {
     int lo[kTables], hi[kTables];
 #pragma unroll
     for (int t = 0; t < kTables; ++t) {
@@ -187,6 +188,9 @@ __global__ void k_alphabet(const int32_t* fields, int64_t nvec, int* lohi) {
             }
         }
     }
+    // warp, then block, then one atomic per table per block (the 34 words are shared by every block)
+    __shared__ int part[kAlphaWarps][2 * kTables];
+    const int wid = threadIdx.x >> 5, lane = threadIdx.x & 31;
 #pragma unroll
     for (int t = 0; t < kTables; ++t) {
         int a = lo[t], b = hi[t];
@@ -194,10 +198,18 @@ __global__ void k_alphabet(const int32_t* fields, int64_t nvec, int* lohi) {
             a = min(a, __shfl_xor_sync(0xFFFFFFFFu, a, o));
             b = max(b, __shfl_xor_sync(0xFFFFFFFFu, b, o));
         }
-        if ((threadIdx.x & 31) == 0) {
-            if (a != INT_MAX) atomicMin(lohi + t, a);
-            if (b != INT_MIN) atomicMax(lohi + kTables + t, b);
+        if (lane == 0) {
+            part[wid][t] = a;
+            part[wid][kTables + t] = b;
         }
+    }
+    __syncthreads();
+    if (threadIdx.x < 2 * kTables) {
+        const int i = threadIdx.x;
+        int v = part[0][i];
+        for (int w = 1; w < kAlphaWarps; ++w) v = i < kTables ? min(v, part[w][i]) : max(v, part[w][i]);
+        if (i < kTables && v != INT_MAX) atomicMin(lohi + i, v);
+        if (i >= kTables && v != INT_MIN) atomicMax(lohi + i, v);
     }
 }
 
@@ -413,7 +425,8 @@ struct GpuEncoder {
     cudaError_t alphabet(const int32_t* f, int64_t n, Hist& al) {
         k_lohi_init<<<1, 32, 0, st>>>(d_lohi.as<int>());
         cudaError_t e;
-        k_alphabet<<<std::min(grid_for(n, 256), 8 * nsm), 256, 0, st>>>(f, n, d_lohi.as<int>());
+        k_alphabet<<<std::min(grid_for(n, 32 * kAlphaWarps), 2 * nsm), 32 * kAlphaWarps, 0, st>>>(f, n,
+                                                                                                 d_lohi.as<int>());
         int got[2 * kTables];
         e = cudaMemcpyAsync(got, d_lohi.p, sizeof(got), cudaMemcpyDeviceToHost, st);
         if (e == cudaSuccess) e = cudaStreamSynchronize(st);

@@ -67,8 +67,9 @@ int64_t side_bytes(const Hist& al, int64_t ntiles, int64_t rows, bool container)
 // ideal code length of the ns sampled vectors scaled to nvec, plus side_bytes.
 double estimate_bpp(Table* tabs, const Hist& al, int b, int64_t nvec, int64_t ns, int64_t ntiles, int64_t rows,
                     int64_t cols, bool container);
-// A blob with its header and tables written and its payload (zeroed, rounded up to 8 words),
-// tile index and row scales allocated for the caller to fill; nullptr when out of memory.
+// A blob with its header and tables written and its payload (rounded up to 8 words, the words
+// past `words` zeroed), tile index and row scales allocated for the caller to fill; nullptr
+// when out of memory.
 ep_blob* new_blob(int64_t rows, int64_t cols, int b, int64_t V, int64_t T, uint64_t words, const Table* tabs);
 // Stored bytes and bits per weight of a filled blob.
 void finish_blob(ep_blob* bl, double s, bool container);

@@ -121,3 +121,24 @@ def test_dit_block_at_mixed_rates_full_size():
             lo, hi = t * per, min((t + 1) * per, blob.rows * blob.cols)
             assert_parity(got[lo:hi], oracle_decode(blob, ep.BF16, t, t + 1), ep.BF16, f"{kinds[k]} tile {t}")
     assert ep.decode_status() == 0
+
+
+def test_one_tensor_per_sm_and_the_limit():
+    """As many tensors as SMs (each on one SM), then one more: refused on the host."""
+    import torch
+
+    nsm = torch.cuda.get_device_properties(0).multi_processor_count
+    rng = np.random.default_rng(77)
+    blobs = []
+    for k in range(nsm):
+        rows, cols = int(rng.integers(1, 40)), 8 * int(rng.integers(1, 64))
+        W = (rng.standard_normal((rows, cols)) * 0.02).astype(np.float32)
+        blobs.append(ep.encode_tensor(W, float(rng.choice([2.5, 4.0, 8.0])), tile_vectors=int(rng.integers(8, 200))))
+    dbs = [ep.DeviceBlob(b) for b in blobs]
+    items = [(db, ep.prepare_lut(db), None) for db in dbs]
+    outs = ep.DecodeBatch(items, ep.BF16).run()
+    assert ep.decode_status() == 0
+    for k, (blob, o) in enumerate(zip(blobs, outs)):
+        assert_parity(to_raw(o), oracle_decode(blob, ep.BF16), ep.BF16, f"item {k}")
+    with pytest.raises(ep.EntroPackError):
+        ep.DecodeBatch(items + items[:1], ep.BF16)

@@ -95,3 +95,10 @@ def test_rdo_is_not_on_the_gpu_path():
 
     with pytest.raises(ep.EntroPackError):
         ep.encode_tensor_gpu(torch.zeros((8, 64), device="cuda"), 4.0, rdo_candidates=4)
+
+
+@pytest.mark.parametrize("bpp", [2.0, 8.0])
+def test_llm_prefill_shape_with_outliers(bpp):
+    """25600x5120 (131 M weights) with 0.05 % outliers at 10 sigma: wide alphabets, b = 12 at
+    8 bpp; the same blob as the packer."""
+    _same(synth.generate(synth.llm_prefill(False)), bpp)
