@@ -254,7 +254,7 @@ def run_ours(args, rank: int, world: int, local_rank: int):
     torch.cuda.synchronize(dev)
     if ep.decode_status(stream) != 0 or not torch.equal(sets[0][1].view(torch.int16), ref.view(torch.int16)):
         raise RuntimeError("prepared decode differs from the per-call decode")
-    prep_ms = None
+    local_prep = -1.0  # every rank takes the same barrier and reduction, whatever happens here
     try:
         pg = torch.cuda.CUDAGraph()
         with torch.cuda.graph(pg, stream=stream):
@@ -263,8 +263,11 @@ def run_ours(args, rank: int, world: int, local_rank: int):
         with torch.cuda.stream(stream):
             pg.replay()
         torch.cuda.synchronize(dev)
-        if world > 1:
-            dist.barrier()
+    except RuntimeError:  # capture unsupported here: no prepared figure
+        pg = None
+    if world > 1:
+        dist.barrier()
+    if pg is not None:
         pa, pb = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         with torch.cuda.stream(stream):
             pa.record(stream)
@@ -272,10 +275,10 @@ def run_ours(args, rank: int, world: int, local_rank: int):
                 pg.replay()
             pb.record(stream)
         torch.cuda.synchronize(dev)
-        (prep_ms,) = reduce_max([pa.elapsed_time(pb) / args.steps], world, dev)
+        local_prep = pa.elapsed_time(pb) / args.steps
         del pg
-    except RuntimeError:  # capture unsupported here: no prepared figure
-        prep_ms = None
+    prep_max, neg_min = reduce_max([local_prep, -local_prep], world, dev)
+    prep_ms = prep_max if -neg_min >= 0.0 else None  # None unless every rank has a figure
     if ep.decode_status(stream) != 0:
         raise RuntimeError("prepared decode reported a corrupt stream")
 
