@@ -507,9 +507,17 @@ extern "C" ep_status ep_encode_tensor_gpu(void* stream, const float* W, int64_t 
         g.nq = nq;
         g.nvec = nvec;
         int dev = 0;
-        if (cudaGetDevice(&dev) != cudaSuccess ||
+        if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64 ||
             cudaDeviceGetAttribute(&g.nsm, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
             return EP_ECUDA;
+        // W must be memory the current device can read: a host pointer would fault the first kernel
+        cudaPointerAttributes pa = {};
+        if (cudaPointerGetAttributes(&pa, W) != cudaSuccess) {
+            cudaGetLastError();  // clear the error of an unknown pointer
+            return EP_EINVAL;
+        }
+        if (!((pa.type == cudaMemoryTypeDevice && pa.device == dev) || pa.type == cudaMemoryTypeManaged))
+            return EP_EINVAL;
         const cudaStream_t st = g.st;
         if (pool_of(dev, DevBuf::pool) != cudaSuccess) return EP_ECUDA;
         DevBuf d_norms, d_srows, d_sf, d_fields, d_scales;

@@ -125,7 +125,9 @@ ep_status ep_encode_tensor(const float* W, int64_t rows, int64_t cols, double ta
  * host's order, without multiply-add contraction, and the estimates' bits come
  * from exact counts (paper §3.1 pipeline; §3.4, §3.5, §3.6, App. C.1, C.3).
  *   stream  cudaStream_t to launch on (the call synchronises it several times).
- *   W       device, float32 [rows, cols] row-major, 4-byte aligned; not modified.
+ *   W       device, float32 [rows, cols] row-major, 4-byte aligned; not modified.  A
+ *           pointer that is not device memory of the current device (or managed
+ *           memory) is refused with EP_EINVAL before any launch.
  *   opts    as ep_encode_tensor; num_threads is ignored and rdo_candidates > 1
  *           (the per-row refinement) returns EP_EUNSUPPORTED.
  * Scratch is allocated with cudaMalloc and freed before the call returns (about

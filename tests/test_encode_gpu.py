@@ -102,3 +102,19 @@ def test_llm_prefill_shape_with_outliers(bpp):
     """25600x5120 (131 M weights) with 0.05 % outliers at 10 sigma: wide alphabets, b = 12 at
     8 bpp; the same blob as the packer."""
     _same(synth.generate(synth.llm_prefill(False)), bpp)
+
+
+def test_host_pointer_is_refused_before_any_launch():
+    """A host buffer passed as the weights: refused on the host (no kernel reads it)."""
+    import ctypes as C
+
+    W = np.zeros((16, 64), np.float32)
+    o = ep._lib._Opts(0, 0, 0, 0, 0, 0, 0, 0, 0)
+    out = C.POINTER(ep._lib._Blob)()
+    rc = ep.lib().ep_encode_tensor_gpu(None, W.ctypes.data, 16, 64, 4.0, C.byref(o), C.byref(out))
+    assert rc == ep._lib.STATUS_CODES["EP_EINVAL"]
+    # the device still works
+    import torch
+
+    _same(np.ones((4, 16), np.float32) * 0.01, 4.0)
+    torch.cuda.synchronize()
