@@ -64,6 +64,26 @@ class _BatchItem(C.Structure):
     ]
 
 
+class _DevBlob(C.Structure):
+    _fields_ = [
+        ("rows", C.c_int64),
+        ("cols", C.c_int64),
+        ("b", C.c_int),
+        ("V", C.c_int),
+        ("ntiles", C.c_int),
+        ("payload_words", C.c_uint64),
+        ("payload_alloc_words", C.c_size_t),
+        ("freq_bytes", C.c_size_t),
+        ("payload", C.c_void_p),
+        ("tile_index", C.c_void_p),
+        ("freq_tables", C.c_void_p),
+        ("row_scales", C.c_void_p),
+        ("s", C.c_double),
+        ("stored_bpp", C.c_double),
+        ("stored_bytes", C.c_int64),
+    ]
+
+
 class _Blob(C.Structure):
     _fields_ = [
         ("rows", C.c_int64),
@@ -102,6 +122,11 @@ def lib() -> C.CDLL:
         L.ep_encode_tensor_gpu.argtypes = [P, P, C.c_int64, C.c_int64, C.c_double, C.POINTER(_Opts),
                                            C.POINTER(C.POINTER(_Blob))]
         L.ep_encode_tensor_gpu.restype = C.c_int
+        L.ep_encode_tensor_gpu_device.argtypes = [P, P, C.c_int, C.c_int64, C.c_int64, C.c_double,
+                                                  C.POINTER(_Opts), C.POINTER(_DevBlob)]
+        L.ep_encode_tensor_gpu_device.restype = C.c_int
+        L.ep_free_device_blob.argtypes = [C.POINTER(_DevBlob)]
+        L.ep_free_device_blob.restype = None
         L.ep_free_blob.argtypes = [C.POINTER(_Blob)]
         L.ep_free_blob.restype = None
         L.ep_decode_tensor.argtypes = [P, P, P, P, P, C.c_int64, C.c_int64, C.c_int, P]
@@ -129,7 +154,8 @@ def lib() -> C.CDLL:
     return _lib
 
 
-EXPORTED = ("ep_encode_tensor", "ep_encode_tensor_gpu", "ep_free_blob", "ep_decode_tensor", "ep_decode_tensor_noalloc", "ep_decode_prepare",
+EXPORTED = ("ep_encode_tensor", "ep_encode_tensor_gpu", "ep_encode_tensor_gpu_device", "ep_free_device_blob",
+            "ep_free_blob", "ep_decode_tensor", "ep_decode_tensor_noalloc", "ep_decode_prepare",
             "ep_decode_tensor_prepared", "ep_batch_create", "ep_decode_batch", "ep_batch_free", "ep_batch_apportion",
             "ep_decode_status", "ep_status_string")
 
@@ -196,13 +222,20 @@ def encode_tensor(W: np.ndarray, target_bpp: float, *, prob_bits: int = 0, tile_
 def encode_tensor_gpu(W, target_bpp: float, *, prob_bits: int = 0, tile_vectors: int = 0, sample_vectors: int = 0,
                       search_steps: int = 0, seed: int = 0, has_container_scales: bool = False,
                       rdo_candidates: int = 0, stream=None) -> Blob:
-    """Compress a float32 CUDA matrix with ep_encode_tensor_gpu: the same blob as encode_tensor, its
-    full-tensor stages on the GPU (launched on `stream`, default torch's current stream).  The
-    per-row refinement (rdo_candidates > 1) is not on this path: EP_EUNSUPPORTED."""
+    """Compress a float32 or bfloat16 CUDA matrix on the GPU into a host Blob: the same bytes as
+    encode_tensor on the float32 values (ep_encode_tensor_gpu; bfloat16 goes through
+    ep_encode_tensor_gpu_device and a copy back).  Launched on `stream` (default torch's current
+    stream).  The per-row refinement (rdo_candidates > 1) is not on this path: EP_EUNSUPPORTED."""
     import torch
 
-    if not (isinstance(W, torch.Tensor) and W.is_cuda and W.dtype == torch.float32 and W.dim() == 2):
-        raise ValueError("W must be a 2-D float32 CUDA tensor")
+    if not (isinstance(W, torch.Tensor) and W.is_cuda and W.dtype in (torch.float32, torch.bfloat16) and W.dim() == 2):
+        raise ValueError("W must be a 2-D float32 or bfloat16 CUDA tensor")
+    if W.dtype == torch.bfloat16:
+        db = encode_tensor_gpu_to_device(W, target_bpp, prob_bits=prob_bits, tile_vectors=tile_vectors,
+                                         sample_vectors=sample_vectors, search_steps=search_steps, seed=seed,
+                                         has_container_scales=has_container_scales, rdo_candidates=rdo_candidates,
+                                         stream=stream)
+        return db.to_host()
     W = W.contiguous()
     o = _Opts(prob_bits, tile_vectors, sample_vectors, search_steps, seed, int(has_container_scales), 0,
               int(rdo_candidates), 0)
@@ -213,6 +246,57 @@ def encode_tensor_gpu(W, target_bpp: float, *, prob_bits: int = 0, tile_vectors:
     if rc:
         raise EntroPackError(rc, "ep_encode_tensor_gpu")
     return _take_blob(out)
+
+
+def encode_tensor_gpu_to_device(W, target_bpp: float, *, prob_bits: int = 0, tile_vectors: int = 0,
+                                sample_vectors: int = 0, search_steps: int = 0, seed: int = 0,
+                                has_container_scales: bool = False, rdo_candidates: int = 0,
+                                stream=None) -> "DeviceBlob":
+    """Compress a float32 or bfloat16 CUDA matrix with ep_encode_tensor_gpu_device and keep the result on
+    the GPU: a DeviceBlob ready for the decoders (its arrays are copied into torch-owned tensors and
+    the library's buffers freed)."""
+    import torch
+
+    if not (isinstance(W, torch.Tensor) and W.is_cuda and W.dtype in (torch.float32, torch.bfloat16) and W.dim() == 2):
+        raise ValueError("W must be a 2-D float32 or bfloat16 CUDA tensor")
+    W = W.contiguous()
+    o = _Opts(prob_bits, tile_vectors, sample_vectors, search_steps, seed, int(has_container_scales), 0,
+              int(rdo_candidates), 0)
+    st = stream if stream is not None else torch.cuda.current_stream(W.device)
+    d = _DevBlob()
+    rc = lib().ep_encode_tensor_gpu_device(C.c_void_p(st.cuda_stream), W.data_ptr(), int(W.dtype == torch.bfloat16),
+                                           W.shape[0], W.shape[1], float(target_bpp), C.byref(o), C.byref(d))
+    if rc:
+        raise EntroPackError(rc, "ep_encode_tensor_gpu_device")
+    try:
+        def take(ptr, n, typestr, dtype):
+            if n == 0:
+                return torch.empty(0, dtype=dtype, device=W.device)
+            view = torch.as_tensor(_CudaMem(ptr, n, typestr), device=W.device)
+            return view.clone()  # a copy the caching allocator owns; the library's buffer is freed below
+
+        T = d.ntiles
+        db = DeviceBlob.__new__(DeviceBlob)
+        db.rows, db.cols, db.b, db.V, db.ntiles = d.rows, d.cols, d.b, d.V, T
+        db.payload = take(d.payload, max(int(d.payload_alloc_words), 8), "<i2", torch.int16)
+        db.tile_index = take(d.tile_index, 33 * T + 1, "<i4", torch.int32)
+        db.freq_tables = take(d.freq_tables, int(d.freq_bytes), "|u1", torch.uint8)
+        db.row_scales = take(d.row_scales, int(d.rows), "<f4", torch.float32)
+        db.read_bytes = 2 * int(d.payload_words) + 4 * (33 * T + 1) + int(d.freq_bytes) + 4 * int(d.rows)
+        db.payload_words, db.s, db.stored_bpp, db.stored_bytes = int(d.payload_words), d.s, d.stored_bpp, \
+            int(d.stored_bytes)
+        st.synchronize()
+        return db
+    finally:
+        lib().ep_free_device_blob(C.byref(d))
+
+
+class _CudaMem:
+    """A device buffer of the library, seen through the CUDA array interface (no copy)."""
+
+    def __init__(self, ptr: int, n: int, typestr: str):
+        self.__cuda_array_interface__ = {"shape": (n,), "typestr": typestr, "data": (int(ptr), False),
+                                         "version": 3, "strides": None}
 
 
 def _take_blob(out) -> Blob:
@@ -244,6 +328,19 @@ class DeviceBlob:
         self.freq_tables = torch.from_numpy(blob.freq_tables).to(device)
         self.row_scales = torch.from_numpy(blob.row_scales).to(device)
         self.read_bytes = blob.stored_device_bytes()
+
+
+def _device_blob_to_host(self) -> Blob:
+    """The arrays of a GPU-encoded DeviceBlob copied into a host Blob (same bytes)."""
+    import torch
+
+    pay = self.payload.cpu().numpy().view(np.uint16)
+    return Blob(self.rows, self.cols, self.b, self.V, self.ntiles, pay, self.payload_words,
+                self.tile_index.cpu().numpy().view(np.uint32), self.freq_tables.cpu().numpy(),
+                self.row_scales.cpu().numpy(), self.s, self.stored_bpp, self.stored_bytes)
+
+
+DeviceBlob.to_host = _device_blob_to_host
 
 
 def _torch_dtype(dt: int):

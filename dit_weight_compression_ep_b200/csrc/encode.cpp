@@ -534,16 +534,24 @@ ep_blob* new_blob(int64_t rows, int64_t cols, int b, int64_t V, int64_t T, uint6
     bl->payload = (uint16_t*)std::malloc(alloc_words * sizeof(uint16_t));
     if (bl->payload) std::memset(bl->payload + words, 0, (alloc_words - words) * sizeof(uint16_t));
     bl->tile_index = (uint32_t*)std::malloc(sizeof(uint32_t) * (size_t)(kTileWords * T + 1));
-    int64_t nf = 0;
-    for (int t = 0; t < kTables; ++t) nf += tabs[t].A;
-    bl->freq_bytes = (size_t)(table_header_bytes(kTables) + 2 * nf);
+    bl->freq_bytes = table_bytes(tabs);
     bl->freq_tables = (uint8_t*)std::calloc(bl->freq_bytes, 1);
     bl->row_scales = (float*)std::malloc(sizeof(float) * (size_t)rows);
     if (!bl->payload || !bl->tile_index || !bl->freq_tables || !bl->row_scales) {
         ep_free_blob(bl);
         return nullptr;
     }
-    uint8_t* h = bl->freq_tables;
+    write_tables(bl->freq_tables, rows, cols, b, V, T, tabs);
+    return bl;
+}
+
+size_t table_bytes(const Table* tabs) {
+    int64_t nf = 0;
+    for (int t = 0; t < kTables; ++t) nf += tabs[t].A;
+    return (size_t)(table_header_bytes(kTables) + 2 * nf);
+}
+
+void write_tables(uint8_t* h, int64_t rows, int64_t cols, int b, int64_t V, int64_t T, const Table* tabs) {
     put32(h + 0, kMagic);
     put32(h + 4, kVersion);
     put32(h + 8, (uint32_t)b);
@@ -564,14 +572,17 @@ ep_blob* new_blob(int64_t rows, int64_t cols, int b, int64_t V, int64_t T, uint6
             fo += 2;
         }
     }
-    return bl;
+}
+
+int64_t stored_bytes(uint64_t words, int64_t T, size_t freq_bytes, int64_t rows, bool container) {
+    return (int64_t)(2 * words) + (int64_t)(4 * ((size_t)kTileWords * T + 1)) + (int64_t)freq_bytes + 4 * rows +
+           (container ? 4 * rows : 0);
 }
 
 void finish_blob(ep_blob* bl, double s, bool container) {
     const int64_t rows = bl->rows;
     bl->s = s;
-    bl->stored_bytes = (int64_t)(2 * bl->payload_words) + (int64_t)(4 * ((size_t)kTileWords * bl->ntiles + 1)) +
-                       (int64_t)bl->freq_bytes + 4 * rows + (container ? 4 * rows : 0);
+    bl->stored_bytes = stored_bytes(bl->payload_words, bl->ntiles, bl->freq_bytes, rows, container);
     bl->stored_bpp = 8.0 * (double)bl->stored_bytes / (double)(rows * bl->cols);
 }
 

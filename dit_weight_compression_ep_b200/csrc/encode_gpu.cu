@@ -479,179 +479,315 @@ struct GpuEncoder {
 }  // namespace
 }  // namespace ep
 
+namespace ep {
+namespace {
+
+// bf16 weights widened to float32 (exact), so that both inputs run the same stages
+__global__ void k_widen_bf16(const uint16_t* src, int64_t n, float* dst) {
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x)
+        dst[i] = __uint_as_float((uint32_t)src[i] << 16);
+}
+
+// Tile records [offset, state_0..31] and the final offset, from the offsets and states.
+__global__ void k_tile_index(int64_t T, const uint32_t* off, const uint32_t* states, uint32_t total, uint32_t* tix) {
+    const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (i > kTileWords * T) return;
+    const int64_t t = i / kTileWords, j = i - t * kTileWords;
+    tix[i] = t == T ? total : (j == 0 ? off[t] : states[kLanes * t + (j - 1)]);
+}
+
+// Argument checks shared by both entry points; fills V and T.
+ep_status check_encode_args(const void* W, int64_t rows, int64_t cols, double target_bpp, const ep_encode_opts& o,
+                            int64_t& V, int64_t& T) {
+    if (!W || rows <= 0 || cols <= 0 || !(target_bpp > 0.0)) return EP_EINVAL;
+    if (o.rdo_candidates > 1) return EP_EUNSUPPORTED;  // the per-row refinement stays on the CPU packer
+    const int b = o.prob_bits > 0 ? o.prob_bits : (target_bpp <= 7.0 ? 11 : 12);
+    if (b < kMinB || b > kMaxB) return EP_EINVAL;
+    const int64_t nq = (cols + 7) / 8, nvec = rows * nq;
+    if (nvec >= (1ll << 31)) return EP_EINVAL;
+    V = o.tile_vectors > 0 ? o.tile_vectors : std::max<int64_t>(32, host::tile_symbols_for(target_bpp) / 9);
+    T = (nvec + V - 1) / V;
+    if (T >= (1ll << 31) / kTileWords) return EP_EINVAL;
+    return EP_OK;
+}
+
+// The current device, its SM count and its encoder pool; W checked to be memory it can read.
+ep_status device_for(const void* W, int& dev, int& nsm) {
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64 ||
+        cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+        return EP_ECUDA;
+    // a host pointer would fault the first kernel
+    cudaPointerAttributes pa = {};
+    if (cudaPointerGetAttributes(&pa, W) != cudaSuccess) {
+        cudaGetLastError();  // clear the error of an unknown pointer
+        return EP_EINVAL;
+    }
+    if (!((pa.type == cudaMemoryTypeDevice && pa.device == dev) || pa.type == cudaMemoryTypeManaged)) return EP_EINVAL;
+    return pool_of(dev, DevBuf::pool) == cudaSuccess ? EP_OK : EP_ECUDA;
+}
+
+// One encode's results, on the device in pool buffers (freed in stream order with it).
+struct Encoded {
+    DevBuf payload, scales, off, states;  // words, rows, T, 32 T
+    uint64_t words = 0;
+    int b = 0;
+    double s = 0.0;
+    Table tabs[kTables];
+};
+
+// The stages of ep_encode_tensor_gpu on float32 weights W (device) into `r`.
+ep_status encode_core(cudaStream_t st, int nsm, const float* W, int64_t rows, int64_t cols, double target_bpp,
+                      const ep_encode_opts& o, int64_t V, int64_t T, Encoded& r) {
+    const int64_t nq = (cols + 7) / 8, nvec = rows * nq;
+    const bool container = o.has_container_scales != 0;
+    int b = o.prob_bits > 0 ? o.prob_bits : (target_bpp <= 7.0 ? 11 : 12);
+    GpuEncoder g;
+    g.st = st;
+    g.nsm = nsm;
+    g.W = W;
+    g.rows = rows;
+    g.cols = cols;
+    g.nq = nq;
+    g.nvec = nvec;
+    DevBuf d_norms, d_srows, d_sf, d_fields;
+    if (g.d_lohi.alloc(sizeof(int) * 2 * kTables, st) != cudaSuccess ||
+        g.d_counts.alloc(sizeof(unsigned long long) * kMaxBins, st) || d_norms.alloc(sizeof(double) * rows, st) ||
+        d_fields.alloc(sizeof(int32_t) * kFields * (size_t)nvec, st) || r.scales.alloc(sizeof(float) * rows, st))
+        return EP_ECUDA;
+    k_norms<<<grid_for(rows, 32), 32, 0, st>>>(W, rows, cols, d_norms.as<double>());
+
+    const std::vector<int64_t> srows = host::sample_rows(rows, cols, o);
+    const int64_t rs = (int64_t)srows.size(), ns = rs * nq;
+    if (d_srows.alloc(sizeof(int64_t) * rs, st) || d_sf.alloc(sizeof(int32_t) * kFields * (size_t)ns, st))
+        return EP_ECUDA;
+    if (cudaMemcpyAsync(d_srows.p, srows.data(), sizeof(int64_t) * rs, cudaMemcpyHostToDevice, st) != cudaSuccess)
+        return EP_ECUDA;
+
+    auto estimate = [&](double s, double& est) -> cudaError_t {
+        cudaError_t e = g.quantize(d_norms.as<double>(), d_srows.as<int64_t>(), rs, s, d_sf.as<int32_t>());
+        Hist al;
+        if (e == cudaSuccess) e = g.alphabet(d_sf.as<int32_t>(), ns, al);
+        if (e != cudaSuccess) return e;
+        if (al.amax_coord() > (1ull << b)) {
+            est = INFINITY;
+            return cudaSuccess;
+        }
+        Table tabs[kTables];
+        e = g.count(d_sf.as<int32_t>(), ns, al, tabs);
+        if (e == cudaSuccess) est = host::estimate_bpp(tabs, al, b, nvec, ns, T, rows, cols, container);
+        return e;
+    };
+    auto quantize_all = [&](double s, Hist& al) -> cudaError_t {
+        cudaError_t e = g.quantize(d_norms.as<double>(), nullptr, rows, s, d_fields.as<int32_t>());
+        return e == cudaSuccess ? g.alphabet(d_fields.as<int32_t>(), nvec, al) : e;
+    };
+
+    // the scale search and the b escalation, decided on the host as in the CPU packer
+    const int steps = o.search_steps > 0 ? o.search_steps : 12;
+    double s = 1.0;
+    Hist al;
+    for (;;) {
+        double lo = 1e-3, hi = 8.0;
+        for (int it = 0; it < steps; ++it) {
+            s = std::sqrt(lo * hi);
+            double est = 0.0;
+            if (estimate(s, est) != cudaSuccess) return EP_ECUDA;
+            if (est > target_bpp) lo = s;
+            else hi = s;
+        }
+        s = std::sqrt(lo * hi);
+        if (quantize_all(s, al) != cudaSuccess) return EP_ECUDA;
+        if (al.amax_coord() <= (1ull << b)) break;
+        if (b < kMaxB) {
+            ++b;
+            continue;
+        }
+        while (al.amax_coord() > (1ull << b)) {
+            s = 1.05 * s * (double)al.amax_coord() / (double)(1u << b);
+            if (quantize_all(s, al) != cudaSuccess) return EP_ECUDA;
+        }
+        break;
+    }
+    k_refit<<<grid_for(rows, 32), 32, 0, st>>>(W, rows, cols, nq, d_fields.as<int32_t>(), r.scales.as<float>());
+
+    if (g.count(d_fields.as<int32_t>(), nvec, al, r.tabs) != cudaSuccess) return EP_ECUDA;
+    for (int t = 0; t < kTables; ++t) {
+        if (r.tabs[t].A > (1u << b)) return EP_EALPHABET;
+        host::normalise(r.tabs[t], b);
+    }
+
+    // rANS: the tables to the device, a warp per tile into scratch, then the words in order
+    RansArgs ra;
+    std::vector<uint32_t> hf, hc;
+    for (int t = 0; t < kTables; ++t) {
+        ra.tmin[t] = r.tabs[t].min;
+        ra.tbase[t] = (uint32_t)hf.size();
+        for (size_t k = 0; k < r.tabs[t].freq.size(); ++k) {
+            hf.push_back(r.tabs[t].freq[k]);
+            hc.push_back(r.tabs[t].cum[k]);
+        }
+    }
+    DevBuf d_freq, d_cum, d_scratch, d_nwords;
+    if (d_freq.alloc(4 * hf.size(), st) || d_cum.alloc(4 * hc.size(), st) ||
+        d_scratch.alloc(sizeof(uint16_t) * (size_t)kFields * (size_t)V * (size_t)T, st) ||
+        d_nwords.alloc(4 * T, st) || r.states.alloc(sizeof(uint32_t) * kLanes * (size_t)T, st) ||
+        r.off.alloc(4 * T, st))
+        return EP_ECUDA;
+    if (cudaMemcpyAsync(d_freq.p, hf.data(), 4 * hf.size(), cudaMemcpyHostToDevice, st) ||
+        cudaMemcpyAsync(d_cum.p, hc.data(), 4 * hc.size(), cudaMemcpyHostToDevice, st))
+        return EP_ECUDA;
+    ra.freq = d_freq.as<uint32_t>();
+    ra.cum = d_cum.as<uint32_t>();
+    k_rans<<<grid_for(T * 32, 128), 128, 0, st>>>(d_fields.as<int32_t>(), nvec, V, T, b, ra,
+                                                  d_scratch.as<uint16_t>(), d_nwords.as<uint32_t>(),
+                                                  r.states.as<uint32_t>());
+    std::vector<uint32_t> nw((size_t)T), off((size_t)T);
+    if (cudaMemcpyAsync(nw.data(), d_nwords.p, 4 * T, cudaMemcpyDeviceToHost, st) || cudaStreamSynchronize(st))
+        return EP_ECUDA;
+    uint64_t words = 0;
+    for (int64_t t = 0; t < T; ++t) {
+        if (words >= 0xFFFFFFFFull) return EP_EINVAL;
+        off[t] = (uint32_t)words;
+        words += nw[t];
+    }
+    if (words > 0xFFFFFFFFull) return EP_EINVAL;
+    if (r.payload.alloc(sizeof(uint16_t) * std::max<uint64_t>(words, 1), st) ||
+        cudaMemcpyAsync(r.off.p, off.data(), 4 * T, cudaMemcpyHostToDevice, st))
+        return EP_ECUDA;
+    k_copy_out<<<(unsigned)T, 256, 0, st>>>(d_scratch.as<uint16_t>(), V, d_nwords.as<uint32_t>(), r.off.as<uint32_t>(),
+                                            r.payload.as<uint16_t>());
+    r.words = words;
+    r.b = b;
+    r.s = s;
+    return cudaGetLastError() == cudaSuccess ? EP_OK : EP_ECUDA;  // the callers synchronise
+}
+
+}  // namespace
+}  // namespace ep
+
 extern "C" ep_status ep_encode_tensor_gpu(void* stream, const float* W, int64_t rows, int64_t cols,
                                           double target_bpp, const ep_encode_opts* opts, ep_blob** out) {
     using namespace ep;
     if (!W || !out) return EP_EINVAL;
     *out = nullptr;
-    if (rows <= 0 || cols <= 0 || !(target_bpp > 0.0)) return EP_EINVAL;
     if ((reinterpret_cast<uintptr_t>(W) & 3u) != 0) return EP_EINVAL;
     ep_encode_opts o{};
     if (opts) o = *opts;
-    if (o.rdo_candidates > 1) return EP_EUNSUPPORTED;  // the per-row refinement stays on the CPU packer
-    int b = o.prob_bits > 0 ? o.prob_bits : (target_bpp <= 7.0 ? 11 : 12);
-    if (b < kMinB || b > kMaxB) return EP_EINVAL;
-    const int64_t nq = (cols + 7) / 8, nvec = rows * nq;
-    if (nvec >= (1ll << 31)) return EP_EINVAL;
-    const int64_t V = o.tile_vectors > 0 ? o.tile_vectors : std::max<int64_t>(32, host::tile_symbols_for(target_bpp) / 9);
-    const int64_t T = (nvec + V - 1) / V;
-    if (T >= (1ll << 31) / kTileWords) return EP_EINVAL;
-    const bool container = o.has_container_scales != 0;
-
+    int64_t V = 0, T = 0;
+    ep_status as = check_encode_args(W, rows, cols, target_bpp, o, V, T);
+    if (as != EP_OK) return as;
     try {
-        GpuEncoder g;
-        g.st = static_cast<cudaStream_t>(stream);
-        g.W = W;
-        g.rows = rows;
-        g.cols = cols;
-        g.nq = nq;
-        g.nvec = nvec;
-        int dev = 0;
-        if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64 ||
-            cudaDeviceGetAttribute(&g.nsm, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
-            return EP_ECUDA;
-        // W must be memory the current device can read: a host pointer would fault the first kernel
-        cudaPointerAttributes pa = {};
-        if (cudaPointerGetAttributes(&pa, W) != cudaSuccess) {
-            cudaGetLastError();  // clear the error of an unknown pointer
-            return EP_EINVAL;
-        }
-        if (!((pa.type == cudaMemoryTypeDevice && pa.device == dev) || pa.type == cudaMemoryTypeManaged))
-            return EP_EINVAL;
-        const cudaStream_t st = g.st;
-        if (pool_of(dev, DevBuf::pool) != cudaSuccess) return EP_ECUDA;
-        DevBuf d_norms, d_srows, d_sf, d_fields, d_scales;
-        if (g.d_lohi.alloc(sizeof(int) * 2 * kTables, st) != cudaSuccess ||
-            g.d_counts.alloc(sizeof(unsigned long long) * kMaxBins, st) || d_norms.alloc(sizeof(double) * rows, st) ||
-            d_fields.alloc(sizeof(int32_t) * kFields * (size_t)nvec, st) || d_scales.alloc(sizeof(float) * rows, st))
-            return EP_ECUDA;
-        k_norms<<<grid_for(rows, 32), 32, 0, st>>>(W, rows, cols, d_norms.as<double>());
-
-        const std::vector<int64_t> srows = host::sample_rows(rows, cols, o);
-        const int64_t rs = (int64_t)srows.size(), ns = rs * nq;
-        if (d_srows.alloc(sizeof(int64_t) * rs, st) || d_sf.alloc(sizeof(int32_t) * kFields * (size_t)ns, st))
-            return EP_ECUDA;
-        if (cudaMemcpyAsync(d_srows.p, srows.data(), sizeof(int64_t) * rs, cudaMemcpyHostToDevice, st) != cudaSuccess)
-            return EP_ECUDA;
-
-        auto estimate = [&](double s, double& est) -> cudaError_t {
-            cudaError_t e = g.quantize(d_norms.as<double>(), d_srows.as<int64_t>(), rs, s, d_sf.as<int32_t>());
-            Hist al;
-            if (e == cudaSuccess) e = g.alphabet(d_sf.as<int32_t>(), ns, al);
-            if (e != cudaSuccess) return e;
-            if (al.amax_coord() > (1ull << b)) {
-                est = INFINITY;
-                return cudaSuccess;
-            }
-            Table tabs[kTables];
-            e = g.count(d_sf.as<int32_t>(), ns, al, tabs);
-            if (e == cudaSuccess) est = host::estimate_bpp(tabs, al, b, nvec, ns, T, rows, cols, container);
-            return e;
-        };
-        auto quantize_all = [&](double s, Hist& al) -> cudaError_t {
-            cudaError_t e = g.quantize(d_norms.as<double>(), nullptr, rows, s, d_fields.as<int32_t>());
-            return e == cudaSuccess ? g.alphabet(d_fields.as<int32_t>(), nvec, al) : e;
-        };
-
-        // the scale search and the b escalation, decided on the host as in the CPU packer
-        const int steps = o.search_steps > 0 ? o.search_steps : 12;
-        double s = 1.0;
-        Hist al;
-        for (;;) {
-            double lo = 1e-3, hi = 8.0;
-            for (int it = 0; it < steps; ++it) {
-                s = std::sqrt(lo * hi);
-                double est = 0.0;
-                if (estimate(s, est) != cudaSuccess) return EP_ECUDA;
-                if (est > target_bpp) lo = s;
-                else hi = s;
-            }
-            s = std::sqrt(lo * hi);
-            if (quantize_all(s, al) != cudaSuccess) return EP_ECUDA;
-            if (al.amax_coord() <= (1ull << b)) break;
-            if (b < kMaxB) {
-                ++b;
-                continue;
-            }
-            while (al.amax_coord() > (1ull << b)) {
-                s = 1.05 * s * (double)al.amax_coord() / (double)(1u << b);
-                if (quantize_all(s, al) != cudaSuccess) return EP_ECUDA;
-            }
-            break;
-        }
-        k_refit<<<grid_for(rows, 32), 32, 0, st>>>(W, rows, cols, nq, d_fields.as<int32_t>(), d_scales.as<float>());
-
-        Table tabs[kTables];
-        if (g.count(d_fields.as<int32_t>(), nvec, al, tabs) != cudaSuccess) return EP_ECUDA;
-        for (int t = 0; t < kTables; ++t) {
-            if (tabs[t].A > (1u << b)) return EP_EALPHABET;
-            host::normalise(tabs[t], b);
-        }
-
-        // rANS: the tables to the device, a warp per tile into scratch, then the words in order
-        RansArgs ra;
-        std::vector<uint32_t> hf, hc;
-        for (int t = 0; t < kTables; ++t) {
-            ra.tmin[t] = tabs[t].min;
-            ra.tbase[t] = (uint32_t)hf.size();
-            for (size_t k = 0; k < tabs[t].freq.size(); ++k) {
-                hf.push_back(tabs[t].freq[k]);
-                hc.push_back(tabs[t].cum[k]);
-            }
-        }
-        DevBuf d_freq, d_cum, d_scratch, d_nwords, d_states, d_off, d_payload;
-        if (d_freq.alloc(4 * hf.size(), st) || d_cum.alloc(4 * hc.size(), st) ||
-            d_scratch.alloc(sizeof(uint16_t) * (size_t)kFields * (size_t)V * (size_t)T, st) ||
-            d_nwords.alloc(4 * T, st) || d_states.alloc(sizeof(uint32_t) * kLanes * (size_t)T, st) ||
-            d_off.alloc(4 * T, st))
-            return EP_ECUDA;
-        if (cudaMemcpyAsync(d_freq.p, hf.data(), 4 * hf.size(), cudaMemcpyHostToDevice, st) ||
-            cudaMemcpyAsync(d_cum.p, hc.data(), 4 * hc.size(), cudaMemcpyHostToDevice, st))
-            return EP_ECUDA;
-        ra.freq = d_freq.as<uint32_t>();
-        ra.cum = d_cum.as<uint32_t>();
-        k_rans<<<grid_for(T * 32, 128), 128, 0, st>>>(d_fields.as<int32_t>(), nvec, V, T, b, ra,
-                                                      d_scratch.as<uint16_t>(), d_nwords.as<uint32_t>(),
-                                                      d_states.as<uint32_t>());
-        std::vector<uint32_t> nw((size_t)T), off((size_t)T);
-        if (cudaMemcpyAsync(nw.data(), d_nwords.p, 4 * T, cudaMemcpyDeviceToHost, st) ||
-            cudaStreamSynchronize(st))
-            return EP_ECUDA;
-        uint64_t words = 0;
-        for (int64_t t = 0; t < T; ++t) {
-            if (words >= 0xFFFFFFFFull) return EP_EINVAL;
-            off[t] = (uint32_t)words;
-            words += nw[t];
-        }
-        if (words > 0xFFFFFFFFull) return EP_EINVAL;
-        if (d_payload.alloc(sizeof(uint16_t) * std::max<uint64_t>(words, 1), st) ||
-            cudaMemcpyAsync(d_off.p, off.data(), 4 * T, cudaMemcpyHostToDevice, st))
-            return EP_ECUDA;
-        k_copy_out<<<(unsigned)T, 256, 0, st>>>(d_scratch.as<uint16_t>(), V, d_nwords.as<uint32_t>(),
-                                                d_off.as<uint32_t>(), d_payload.as<uint16_t>());
-
-        ep_blob* bl = host::new_blob(rows, cols, b, V, T, words, tabs);
+        int dev = 0, nsm = 0;
+        if ((as = device_for(W, dev, nsm)) != EP_OK) return as;
+        const cudaStream_t st = static_cast<cudaStream_t>(stream);
+        Encoded r;
+        if ((as = encode_core(st, nsm, W, rows, cols, target_bpp, o, V, T, r)) != EP_OK) return as;
+        ep_blob* bl = host::new_blob(rows, cols, r.b, V, T, r.words, r.tabs);
         if (!bl) return EP_ENOMEM;
-        std::vector<uint32_t> states((size_t)kLanes * T);
-        cudaError_t e = cudaMemcpyAsync(bl->payload, d_payload.p, 2 * words, cudaMemcpyDeviceToHost, st);
+        std::vector<uint32_t> states((size_t)kLanes * T), offs((size_t)T);
+        cudaError_t e = cudaMemcpyAsync(bl->payload, r.payload.p, 2 * r.words, cudaMemcpyDeviceToHost, st);
         if (e == cudaSuccess)
-            e = cudaMemcpyAsync(states.data(), d_states.p, 4 * states.size(), cudaMemcpyDeviceToHost, st);
+            e = cudaMemcpyAsync(states.data(), r.states.p, 4 * states.size(), cudaMemcpyDeviceToHost, st);
+        if (e == cudaSuccess) e = cudaMemcpyAsync(offs.data(), r.off.p, 4 * T, cudaMemcpyDeviceToHost, st);
         if (e == cudaSuccess)
-            e = cudaMemcpyAsync(bl->row_scales, d_scales.p, sizeof(float) * rows, cudaMemcpyDeviceToHost, st);
+            e = cudaMemcpyAsync(bl->row_scales, r.scales.p, sizeof(float) * rows, cudaMemcpyDeviceToHost, st);
         if (e == cudaSuccess) e = cudaStreamSynchronize(st);
         if (e != cudaSuccess) {
             ep_free_blob(bl);
             return EP_ECUDA;
         }
         for (int64_t t = 0; t < T; ++t) {
-            bl->tile_index[kTileWords * t] = off[t];
+            bl->tile_index[kTileWords * t] = offs[t];
             for (int j = 0; j < kLanes; ++j) bl->tile_index[kTileWords * t + 1 + j] = states[(size_t)kLanes * t + j];
         }
-        bl->tile_index[kTileWords * T] = (uint32_t)words;
-        host::finish_blob(bl, s, container);
+        bl->tile_index[kTileWords * T] = (uint32_t)r.words;
+        host::finish_blob(bl, r.s, o.has_container_scales != 0);
         *out = bl;
         return EP_OK;
     } catch (const std::bad_alloc&) {
         return EP_ENOMEM;
     }
+}
+
+extern "C" ep_status ep_encode_tensor_gpu_device(void* stream, const void* W, int w_is_bf16, int64_t rows,
+                                                 int64_t cols, double target_bpp, const ep_encode_opts* opts,
+                                                 ep_device_blob* out) {
+    using namespace ep;
+    if (!W || !out) return EP_EINVAL;
+    *out = ep_device_blob{};
+    if ((reinterpret_cast<uintptr_t>(W) & (w_is_bf16 ? 1u : 3u)) != 0) return EP_EINVAL;
+    ep_encode_opts o{};
+    if (opts) o = *opts;
+    int64_t V = 0, T = 0;
+    ep_status as = check_encode_args(W, rows, cols, target_bpp, o, V, T);
+    if (as != EP_OK) return as;
+    try {
+        int dev = 0, nsm = 0;
+        if ((as = device_for(W, dev, nsm)) != EP_OK) return as;
+        const cudaStream_t st = static_cast<cudaStream_t>(stream);
+        DevBuf wide;
+        const float* W32 = static_cast<const float*>(W);
+        if (w_is_bf16) {
+            const int64_t n = rows * cols;
+            if (wide.alloc(sizeof(float) * (size_t)n, st) != cudaSuccess) return EP_ECUDA;
+            k_widen_bf16<<<std::min(grid_for(n, 256), 16 * nsm), 256, 0, st>>>(static_cast<const uint16_t*>(W), n,
+                                                                              wide.as<float>());
+            W32 = wide.as<float>();
+        }
+        Encoded r;
+        if ((as = encode_core(st, nsm, W32, rows, cols, target_bpp, o, V, T, r)) != EP_OK) return as;
+        // the stream's own buffers, outliving the call
+        ep_device_blob d = {};
+        d.rows = rows;
+        d.cols = cols;
+        d.b = r.b;
+        d.V = (int)V;
+        d.ntiles = (int)T;
+        d.payload_words = r.words;
+        d.payload_alloc_words = (r.words + 7) / 8 * 8;
+        const size_t alloc_words = std::max<size_t>(d.payload_alloc_words, 8);
+        d.freq_bytes = host::table_bytes(r.tabs);
+        std::vector<uint8_t> ft(d.freq_bytes, 0);
+        host::write_tables(ft.data(), rows, cols, r.b, V, T, r.tabs);
+        void *pp = nullptr, *pt = nullptr, *pf = nullptr, *ps = nullptr;
+        cudaError_t e = cudaMalloc(&pp, 2 * alloc_words);
+        if (e == cudaSuccess) e = cudaMalloc(&pt, 4 * ((size_t)kTileWords * T + 1));
+        if (e == cudaSuccess) e = cudaMalloc(&pf, d.freq_bytes);
+        if (e == cudaSuccess) e = cudaMalloc(&ps, sizeof(float) * rows);
+        d.payload = static_cast<uint16_t*>(pp);
+        d.tile_index = static_cast<uint32_t*>(pt);
+        d.freq_tables = static_cast<uint8_t*>(pf);
+        d.row_scales = static_cast<float*>(ps);
+        if (e == cudaSuccess) e = cudaMemcpyAsync(pp, r.payload.p, 2 * r.words, cudaMemcpyDeviceToDevice, st);
+        if (e == cudaSuccess) e = cudaMemsetAsync(d.payload + r.words, 0, 2 * (alloc_words - r.words), st);
+        if (e == cudaSuccess) {
+            k_tile_index<<<grid_for(kTileWords * T + 1, 256), 256, 0, st>>>(T, r.off.as<uint32_t>(),
+                                                                            r.states.as<uint32_t>(),
+                                                                            (uint32_t)r.words, d.tile_index);
+            e = cudaGetLastError();
+        }
+        if (e == cudaSuccess) e = cudaMemcpyAsync(pf, ft.data(), d.freq_bytes, cudaMemcpyHostToDevice, st);
+        if (e == cudaSuccess) e = cudaMemcpyAsync(ps, r.scales.p, sizeof(float) * rows, cudaMemcpyDeviceToDevice, st);
+        if (e == cudaSuccess) e = cudaStreamSynchronize(st);  // ft (host) is freed on return
+        if (e != cudaSuccess) {
+            ep_free_device_blob(&d);
+            return EP_ECUDA;
+        }
+        d.s = r.s;
+        d.stored_bytes = host::stored_bytes(r.words, T, d.freq_bytes, rows, o.has_container_scales != 0);
+        d.stored_bpp = 8.0 * (double)d.stored_bytes / (double)(rows * cols);
+        *out = d;
+        return EP_OK;
+    } catch (const std::bad_alloc&) {
+        return EP_ENOMEM;
+    }
+}
+
+extern "C" void ep_free_device_blob(ep_device_blob* d) {
+    if (!d) return;
+    if (d->payload) cudaFree(d->payload);
+    if (d->tile_index) cudaFree(d->tile_index);
+    if (d->freq_tables) cudaFree(d->freq_tables);
+    if (d->row_scales) cudaFree(d->row_scales);
+    *d = ep_device_blob{};
 }

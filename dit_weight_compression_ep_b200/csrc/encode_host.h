@@ -71,6 +71,11 @@ double estimate_bpp(Table* tabs, const Hist& al, int b, int64_t nvec, int64_t ns
 // past `words` zeroed), tile index and row scales allocated for the caller to fill; nullptr
 // when out of memory.
 ep_blob* new_blob(int64_t rows, int64_t cols, int b, int64_t V, int64_t T, uint64_t words, const Table* tabs);
+// Bytes of the table header and frequencies, and their writer (into a zeroed buffer of that size).
+size_t table_bytes(const Table* tabs);
+void write_tables(uint8_t* h, int64_t rows, int64_t cols, int b, int64_t V, int64_t T, const Table* tabs);
+// Stored bytes of a stream: payload, tile records, tables, row scales (and container scales).
+int64_t stored_bytes(uint64_t words, int64_t T, size_t freq_bytes, int64_t rows, bool container);
 // Stored bytes and bits per weight of a filled blob.
 void finish_blob(ep_blob* bl, double s, bool container);
 

@@ -138,6 +138,42 @@ ep_status ep_encode_tensor(const float* W, int64_t rows, int64_t cols, double ta
 ep_status ep_encode_tensor_gpu(void* stream, const float* W, int64_t rows, int64_t cols, double target_bpp,
                                const ep_encode_opts* opts, ep_blob** out);
 
+/*
+ * A compressed tensor in device memory, as ep_encode_tensor_gpu_device returns
+ * it: the four stored arrays of ep_blob (the same bytes), each in its own
+ * cudaMalloc allocation that the struct owns (free with ep_free_device_blob).
+ * The buffers meet ep_decode_tensor's alignment and padding rules.
+ */
+typedef struct {
+    int64_t rows, cols;
+    int b, V, ntiles;
+    uint64_t payload_words;      /* words of payload (the last tile's end offset) */
+    size_t payload_alloc_words;  /* payload_words rounded up to 8 (the tail is zero) */
+    size_t freq_bytes;
+    uint16_t* payload;           /* device */
+    uint32_t* tile_index;        /* device, 33 * ntiles + 1 words */
+    uint8_t* freq_tables;        /* device, freq_bytes */
+    float* row_scales;           /* device, rows */
+    double s, stored_bpp;
+    int64_t stored_bytes;
+} ep_device_blob;
+
+/*
+ * ep_encode_tensor_gpu_device -- ep_encode_tensor_gpu with the compressed
+ * tensor left in device memory (no copy to the host): for a model whose
+ * weights are loaded to the GPU and compressed there.  W is float32 (w_is_bf16
+ * = 0, 4-byte aligned) or bfloat16 (w_is_bf16 = 1, 2-byte aligned; widened to
+ * float32 exactly on the GPU, so the bytes are those of the packer on the
+ * widened matrix).  *out receives the arrays in new device allocations; the
+ * scratch is freed before the call returns.  Errors as ep_encode_tensor_gpu
+ * (on an error *out is left empty).
+ */
+ep_status ep_encode_tensor_gpu_device(void* stream, const void* W, int w_is_bf16, int64_t rows, int64_t cols,
+                                      double target_bpp, const ep_encode_opts* opts, ep_device_blob* out);
+
+/* Free the device arrays of an ep_device_blob and clear it (NULL and empty blobs are allowed). */
+void ep_free_device_blob(ep_device_blob* blob);
+
 /* Free a blob returned by ep_encode_tensor or ep_encode_tensor_gpu (NULL is allowed). */
 void ep_free_blob(ep_blob* blob);
 

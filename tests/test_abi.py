@@ -129,3 +129,24 @@ def test_gpu_encoder_refuses_bad_arguments_on_host(lib):
     assert call(prob_bits=8) == EINVAL
     assert call(rdo=4) == EUNSUP                        # the per-row refinement stays on the CPU packer
     assert call(rows=1 << 20, cols=1 << 14) == EINVAL  # 2^31 vectors
+
+
+def test_gpu_device_encoder_refuses_bad_arguments_on_host(lib):
+    EINVAL, EUNSUP = ep._lib.STATUS_CODES["EP_EINVAL"], ep._lib.STATUS_CODES["EP_EUNSUPPORTED"]
+    good = C.c_void_p(0x10000)
+    d = ep._lib._DevBlob()
+
+    def call(W=good, bf16=0, rows=64, cols=64, bpp=4.0, rdo=0, out=True):
+        o = ep._lib._Opts(0, 0, 0, 0, 0, 0, 0, rdo, 0)
+        return lib.ep_encode_tensor_gpu_device(None, W, bf16, rows, cols, bpp, C.byref(o), C.byref(d) if out else None)
+
+    assert call(W=None) == EINVAL
+    assert call(out=False) == EINVAL
+    assert call(W=C.c_void_p(0x10002)) == EINVAL           # float32 needs 4-byte alignment
+    assert call(W=C.c_void_p(0x10001), bf16=1) == EINVAL   # bfloat16 needs 2
+    assert call(rows=0) == EINVAL
+    assert call(bpp=-1.0) == EINVAL
+    assert call(rdo=3) == EUNSUP
+    assert not d.payload and not d.tile_index
+    lib.ep_free_device_blob(None)
+    lib.ep_free_device_blob(C.byref(d))

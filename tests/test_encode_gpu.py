@@ -118,3 +118,40 @@ def test_host_pointer_is_refused_before_any_launch():
 
     _same(np.ones((4, 16), np.float32) * 0.01, 4.0)
     torch.cuda.synchronize()
+
+
+def _host_arrays(blob):
+    """The stored arrays (payload words up to the final offset; the allocation padding is zero in both)."""
+    return (blob.payload[:blob.payload_words], blob.tile_index, blob.freq_tables, blob.row_scales.view(np.uint32))
+
+
+@pytest.mark.parametrize("rows,cols,bpp", [(256, 512, 4.0), (17, 1001, 8.0), (3, 5, 2.3)])
+def test_device_output_equals_the_packer_and_decodes(rows, cols, bpp):
+    """ep_encode_tensor_gpu_device: the packer's bytes, left on the GPU, decoded there to the
+    oracle's values."""
+    import torch
+
+    rng = np.random.default_rng(rows + cols)
+    W = (rng.standard_t(5, (rows, cols)) * 0.02).astype(np.float32)
+    cpu = ep.encode_tensor(W, bpp)
+    db = ep.encode_tensor_gpu_to_device(torch.from_numpy(W).cuda(), bpp)
+    got = db.to_host()
+    for a, b in zip(_host_arrays(got), _host_arrays(cpu)):
+        np.testing.assert_array_equal(a, b)
+    assert (got.s, got.stored_bpp, got.b, got.V, got.ntiles) == (cpu.s, cpu.stored_bpp, cpu.b, cpu.V, cpu.ntiles)
+    out = ep.decode_tensor(db, ep.BF16)
+    assert ep.decode_status() == 0
+    assert_parity(to_raw(out), oracle_decode(cpu, ep.BF16), ep.BF16, "device blob")
+
+
+@pytest.mark.parametrize("rows,cols", [(3840, 3840), (33, 101)])
+def test_bf16_weights_encode_like_their_float32_values(rows, cols):
+    """bfloat16 input is widened exactly: the bytes of the packer on the float32 values."""
+    import torch
+
+    W = torch.from_numpy(synth.generate(synth.dit_attn_proj())[:rows, :cols].copy()).to(torch.bfloat16).cuda()
+    ref = ep.encode_tensor(W.float().cpu().numpy(), 5.0)
+    got = ep.encode_tensor_gpu(W, 5.0)
+    for a, b in zip(_host_arrays(got), _host_arrays(ref)):
+        np.testing.assert_array_equal(a, b)
+    assert got.s == ref.s
