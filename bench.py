@@ -794,9 +794,10 @@ def run_encode(args):
 
 
 def run_linear(args):
-    """A linear layer whose weight is stored compressed: decode it with the library, then the
-    library GEMM (cuBLAS through torch), against the same GEMM with the weight resident
-    (BF16 X @ W^T; FP8-e4m3 `_scaled_mm` with per-row weight scales; INT8 `_int_mm`).  The
+    """A linear layer whose weight is stored compressed (CompressedLinear: decode with the library's
+    prepared table, then the library GEMM, cuBLAS through torch), against the same GEMM with the
+    weight resident (BF16 X @ W^T; FP8-e4m3 `_scaled_mm` with per-row weight scales; INT8 `_int_mm`
+    with the per-token and per-row scales).  The
     3840x10240 layer at 4 bpp, tokens 256 .. 16384; each time is the minimum of 15 runs, each
     after a 256 MiB L2 flush.  Prints a markdown table and JSON lines."""
     import torch
@@ -838,7 +839,8 @@ def run_linear(args):
     routes.append(("fp8 e4m3", ep.DeviceBlob(blob8), ep.FP8_E4M3, W8, torch.empty_like(W8)))
     wscale = torch.from_numpy(wsc).to(dev).view(1, -1)
     # INT8 container, per-row scales
-    vali, _ = synth.to_int8_container(W)
+    vali, wsci = synth.to_int8_container(W)
+    wscale_i = torch.from_numpy(wsci).to(dev).view(1, -1)
     blobi = ep.encode_tensor(vali, TARGET, has_container_scales=True)
     Wi = torch.from_numpy(vali).to(dev).to(torch.int8)
     routes.append(("int8", ep.DeviceBlob(blobi), ep.INT8, Wi, torch.empty_like(Wi)))
@@ -850,19 +852,26 @@ def run_linear(args):
         Xi = X.mul(20).round().clamp(-127, 127).to(torch.int8)
         xs = torch.ones(tokens, 1, device=dev)
         for name, dbr, dt, Wres, Wdec in routes:
+            # the resident side runs the same GEMM (and scaling) as CompressedLinear's route
             if name == "bf16":
+                lin = ep.CompressedLinear(dbr, "bf16", scratch=Wdec)
                 gemm = lambda Wm: torch.matmul(Xb, Wm.t())
+                call = lambda lin=lin: lin(Xb)
             elif name == "fp8 e4m3":
+                lin = ep.CompressedLinear(dbr, "fp8", weight_scales=wscale, scratch=Wdec)
                 gemm = lambda Wm: torch._scaled_mm(X8, Wm.t(), scale_a=xs, scale_b=wscale, out_dtype=torch.bfloat16)
+                call = lambda lin=lin: lin(X8, xs)
             else:
-                gemm = lambda Wm: torch._int_mm(Xi, Wm.t())
+                lin = ep.CompressedLinear(dbr, "int8", weight_scales=wscale_i, scratch=Wdec)
+                gemm = lambda Wm: (torch._int_mm(Xi, Wm.t()).float() * xs * wscale_i).to(torch.bfloat16)
+                call = lambda lin=lin: lin(Xi, xs)
             try:
                 t_res = tmin(lambda: gemm(Wres))
             except Exception as exc:  # a route torch's GEMMs do not offer on this device
                 print(json.dumps({"route": name, "tokens": tokens, "unavailable": str(exc)[:160]}), flush=True)
                 continue
-            t_dec = tmin(lambda: ep.decode_tensor(dbr, dt, out=Wdec))
-            t_both = tmin(lambda: (ep.decode_tensor(dbr, dt, out=Wdec), gemm(Wdec)))
+            t_dec = tmin(lambda lin=lin: lin.decoded_weight())
+            t_both = tmin(call)
             r = {"route": name, "tokens": tokens, "gemm_resident_us": round(t_res, 2), "decode_us": round(t_dec, 2),
                  "decode_then_gemm_us": round(t_both, 2), "overhead": round(t_both / t_res - 1.0, 4)}
             out.append(r)
