@@ -150,3 +150,21 @@ def test_gpu_device_encoder_refuses_bad_arguments_on_host(lib):
     assert not d.payload and not d.tile_index
     lib.ep_free_device_blob(None)
     lib.ep_free_device_blob(C.byref(d))
+
+
+def test_header_compiles_as_c99(tmp_path):
+    """include/entropack.h is a C header: every declaration compiles as strict C99."""
+    import shutil
+    import subprocess
+
+    cc = shutil.which("gcc") or shutil.which("cc")
+    if cc is None:
+        pytest.skip("no C compiler")
+    src = tmp_path / "h.c"
+    src.write_text('#include "entropack.h"\n'
+                   "int main(void) { ep_device_blob d = {0}; ep_batch_item it = {0}; ep_encode_opts o = {0};\n"
+                   "  (void)d; (void)it; (void)o; return (int)EP_LUT_BYTES - 131104; }\n")
+    exe = tmp_path / "h"
+    subprocess.run([cc, "-std=c99", "-Wall", "-Wextra", "-Werror", "-pedantic", "-I", os.path.join(ROOT, "include"),
+                    str(src), "-o", str(exe)], check=True)
+    assert subprocess.run([str(exe)]).returncode == 0
