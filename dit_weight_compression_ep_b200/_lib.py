@@ -221,11 +221,11 @@ def encode_tensor(W: np.ndarray, target_bpp: float, *, prob_bits: int = 0, tile_
 
 def encode_tensor_gpu(W, target_bpp: float, *, prob_bits: int = 0, tile_vectors: int = 0, sample_vectors: int = 0,
                       search_steps: int = 0, seed: int = 0, has_container_scales: bool = False,
-                      rdo_candidates: int = 0, stream=None) -> Blob:
+                      rdo_candidates: int = 0, rdo_sweeps: int = 0, stream=None) -> Blob:
     """Compress a float32 or bfloat16 CUDA matrix on the GPU into a host Blob: the same bytes as
     encode_tensor on the float32 values (ep_encode_tensor_gpu; bfloat16 goes through
     ep_encode_tensor_gpu_device and a copy back).  Launched on `stream` (default torch's current
-    stream).  The per-row refinement (rdo_candidates > 1) is not on this path: EP_EUNSUPPORTED."""
+    stream).  rdo_candidates > 1 runs the per-row refinement (App. C.2) on the GPU as well."""
     import torch
 
     if not (isinstance(W, torch.Tensor) and W.is_cuda and W.dtype in (torch.float32, torch.bfloat16) and W.dim() == 2):
@@ -234,11 +234,11 @@ def encode_tensor_gpu(W, target_bpp: float, *, prob_bits: int = 0, tile_vectors:
         db = encode_tensor_gpu_to_device(W, target_bpp, prob_bits=prob_bits, tile_vectors=tile_vectors,
                                          sample_vectors=sample_vectors, search_steps=search_steps, seed=seed,
                                          has_container_scales=has_container_scales, rdo_candidates=rdo_candidates,
-                                         stream=stream)
+                                         rdo_sweeps=rdo_sweeps, stream=stream)
         return db.to_host()
     W = W.contiguous()
     o = _Opts(prob_bits, tile_vectors, sample_vectors, search_steps, seed, int(has_container_scales), 0,
-              int(rdo_candidates), 0)
+              int(rdo_candidates), int(rdo_sweeps))
     st = stream if stream is not None else torch.cuda.current_stream(W.device)
     out = C.POINTER(_Blob)()
     rc = lib().ep_encode_tensor_gpu(C.c_void_p(st.cuda_stream), W.data_ptr(), W.shape[0], W.shape[1],
@@ -250,7 +250,7 @@ def encode_tensor_gpu(W, target_bpp: float, *, prob_bits: int = 0, tile_vectors:
 
 def encode_tensor_gpu_to_device(W, target_bpp: float, *, prob_bits: int = 0, tile_vectors: int = 0,
                                 sample_vectors: int = 0, search_steps: int = 0, seed: int = 0,
-                                has_container_scales: bool = False, rdo_candidates: int = 0,
+                                has_container_scales: bool = False, rdo_candidates: int = 0, rdo_sweeps: int = 0,
                                 stream=None) -> "DeviceBlob":
     """Compress a float32 or bfloat16 CUDA matrix with ep_encode_tensor_gpu_device and keep the result on
     the GPU: a DeviceBlob ready for the decoders (its arrays are copied into torch-owned tensors and
@@ -261,7 +261,7 @@ def encode_tensor_gpu_to_device(W, target_bpp: float, *, prob_bits: int = 0, til
         raise ValueError("W must be a 2-D float32 or bfloat16 CUDA tensor")
     W = W.contiguous()
     o = _Opts(prob_bits, tile_vectors, sample_vectors, search_steps, seed, int(has_container_scales), 0,
-              int(rdo_candidates), 0)
+              int(rdo_candidates), int(rdo_sweeps))
     st = stream if stream is not None else torch.cuda.current_stream(W.device)
     d = _DevBlob()
     rc = lib().ep_encode_tensor_gpu_device(C.c_void_p(st.cuda_stream), W.data_ptr(), int(W.dtype == torch.bfloat16),

@@ -31,6 +31,7 @@ namespace {
 
 using host::Hist;
 using host::normalise;
+using host::rdo_ratios;
 using host::Table;
 using host::tile_symbols_for;
 
@@ -196,34 +197,6 @@ void count_fields(const int32_t* f, int64_t nvec, const Hist& al, Table* tabs, i
 
 // ------------------------------------------------- per-row refinement (RDO)
 
-// Paper §3.5, App. C.2: K candidate ratios in [0.70, 1.45]: 1 first, then the
-// log-midpoint of the widest interval between neighbours and the range ends
-// (ties: the lower interval); nested in K.
-void rdo_ratios(int K, double* rho) {
-    double pts[2 + 64];
-    int n = 3;
-    pts[0] = 0.70;
-    pts[1] = 1.0;
-    pts[2] = 1.45;
-    rho[0] = 1.0;
-    for (int k = 1; k < K && k < 64; ++k) {
-        int best = 0;
-        double wbest = -1.0;
-        for (int i = 0; i + 1 < n; ++i) {
-            const double w = std::log(pts[i + 1] / pts[i]);
-            if (w > wbest) {
-                wbest = w;
-                best = i;
-            }
-        }
-        const double mid = std::sqrt(pts[best] * pts[best + 1]);
-        for (int i = n; i > best + 1; --i) pts[i] = pts[i - 1];
-        pts[best + 1] = mid;
-        ++n;
-        rho[k] = mid;
-    }
-}
-
 // Ideal code length of one row's fields under the tables, symbols in order; a
 // symbol the tables give no frequency costs b bits.
 double row_bits(const int32_t* f, int64_t nq, const Table* tabs, int b) {
@@ -319,32 +292,7 @@ void rdo_refine(const float* W, int64_t rows, int64_t cols, const std::vector<do
                     cr[i] = ok[i] ? row_bits(cf.data() + (size_t)((k * rows + r) * rowf), nq, model, b) : INFINITY;
                 }
         });
-        double lo = -80.0, hi = 80.0;
-        for (int it = 0; it <= 64; ++it) {
-            const double t = it < 64 ? 0.5 * (lo + hi) : hi;
-            const double lam = std::exp2(t);
-            parallel_for(rows, nthreads, [&](int64_t a, int64_t e) {
-                for (int64_t r = a; r < e; ++r) {
-                    int best = 0;
-                    double jbest = cd[(size_t)r] + lam * cr[(size_t)r];
-                    for (int k = 1; k < K; ++k) {
-                        const double j = cd[(size_t)(k * rows + r)] + lam * cr[(size_t)(k * rows + r)];
-                        if (j < jbest) {
-                            jbest = j;
-                            best = k;
-                        }
-                    }
-                    sel[(size_t)r] = best;
-                    rsel[(size_t)r] = cr[(size_t)(best * rows + r)];
-                }
-            });
-            double total = 0.0;
-            for (int64_t r = 0; r < rows; ++r) total += rsel[(size_t)r];
-            if (it < 64) {
-                if (total <= budget) hi = t;
-                else lo = t;
-            }
-        }
+        host::rdo_bisect(cd.data(), cr.data(), rows, K, budget, nthreads, sel.data());
         parallel_for(rows, nthreads, [&](int64_t a, int64_t e) {
             for (int64_t r = a; r < e; ++r)
                 std::memcpy(fields.data() + (size_t)(r * rowf), cf.data() + (size_t)((sel[(size_t)r] * rows + r) * rowf),
@@ -423,6 +371,34 @@ struct Encoder {
 
 namespace host {
 
+// Paper §3.5, App. C.2: K candidate ratios in [0.70, 1.45]: 1 first, then the
+// log-midpoint of the widest interval between neighbours and the range ends
+// (ties: the lower interval); nested in K.
+void rdo_ratios(int K, double* rho) {
+    double pts[2 + 64];
+    int n = 3;
+    pts[0] = 0.70;
+    pts[1] = 1.0;
+    pts[2] = 1.45;
+    rho[0] = 1.0;
+    for (int k = 1; k < K && k < 64; ++k) {
+        int best = 0;
+        double wbest = -1.0;
+        for (int i = 0; i + 1 < n; ++i) {
+            const double w = std::log(pts[i + 1] / pts[i]);
+            if (w > wbest) {
+                wbest = w;
+                best = i;
+            }
+        }
+        const double mid = std::sqrt(pts[best] * pts[best + 1]);
+        for (int i = n; i > best + 1; --i) pts[i] = pts[i - 1];
+        pts[best + 1] = mid;
+        ++n;
+        rho[k] = mid;
+    }
+}
+
 // Frequencies at M = 2^b: f = max(1, floor(count*M/total + 1/2)) for present
 // symbols; the excess comes off the largest f > 1 one unit at a time (lowest
 // symbol on ties), a shortfall goes to the most frequent symbol (lowest on ties).
@@ -463,6 +439,36 @@ void normalise(Table& tb, int b) {
         tb.freq[best] += (uint32_t)(M - sum);
     }
     for (uint32_t s = 0; s < tb.A; ++s) tb.cum[s + 1] = tb.cum[s] + tb.freq[s];
+}
+
+void rdo_bisect(const double* cd, const double* cr, int64_t rows, int K, double budget, int nthreads, int* sel) {
+    std::vector<double> rsel((size_t)rows);
+    double lo = -80.0, hi = 80.0;
+    for (int it = 0; it <= 64; ++it) {
+        const double t = it < 64 ? 0.5 * (lo + hi) : hi;
+        const double lam = std::exp2(t);
+        parallel_for(rows, nthreads, [&](int64_t a, int64_t e) {
+            for (int64_t r = a; r < e; ++r) {
+                int best = 0;
+                double jbest = cd[(size_t)r] + lam * cr[(size_t)r];
+                for (int k = 1; k < K; ++k) {
+                    const double j = cd[(size_t)(k * rows + r)] + lam * cr[(size_t)(k * rows + r)];
+                    if (j < jbest) {
+                        jbest = j;
+                        best = k;
+                    }
+                }
+                sel[(size_t)r] = best;
+                rsel[(size_t)r] = cr[(size_t)(best * rows + r)];
+            }
+        });
+        double total = 0.0;
+        for (int64_t r = 0; r < rows; ++r) total += rsel[(size_t)r];
+        if (it < 64) {
+            if (total <= budget) hi = t;
+            else lo = t;
+        }
+    }
 }
 
 int64_t tile_symbols_for(double target) {

@@ -13,7 +13,7 @@
 //   - the rANS step is integer arithmetic; a warp encodes a tile, lane j holding the tile's
 //     lane j, and each step's words are placed in the order the host emits them.
 // What runs on the host: the sample choice, the search's decisions, the b escalation, table
-// normalisation and the blob header.  The per-row refinement (App. C.2) is not on this path.
+// normalisation, the per-row refinement's lambda bisection (App. C.2) and the blob header.
 
 #include <cuda_runtime.h>
 #include <stdint.h>
@@ -21,6 +21,7 @@
 #include <algorithm>
 #include <climits>
 #include <mutex>
+#include <thread>
 #include <cmath>
 #include <new>
 #include <vector>
@@ -245,11 +246,15 @@ __global__ void k_count(const int32_t* fields, int64_t nvec, CountArgs ca, uint3
 }
 
 // Row scales: the least-squares scale <w, y> / <y, y> over the real entries, sums in index
-// order (y = z + c/2 rebuilt from the fields), 0 for a zero denominator.  Same ring as k_norms,
-// with the fields of the chunk's four vectors (36 words a row) beside its 32 weights.
+// order (y = z + c/2 rebuilt from the fields), 0 for a zero denominator.  DIST: instead, the
+// distortion sum (w - sigma y)^2 in index order with sigma = sg_in[row] (the refinement's
+// candidates, App. C.2).  Same ring as k_norms, with the fields of the chunk's four vectors
+// (36 words a row) beside its 32 weights.
 constexpr int kRefitDepth = 4;
-__global__ void __launch_bounds__(32) k_refit(const float* W, int64_t rows, int64_t cols, int64_t nq,
-                                               const int32_t* fields, float* scales) {
+template <bool DIST>
+__global__ void __launch_bounds__(32) k_rowpass(const float* W, int64_t rows, int64_t cols, int64_t nq,
+                                                 const int32_t* fields, const float* sg_in, float* scales,
+                                                 double* dist) {
     __shared__ float rw[kRefitDepth][32][33];
     __shared__ int32_t rf[kRefitDepth][32][37];
     const int lane = threadIdx.x & 31;
@@ -272,6 +277,7 @@ __global__ void __launch_bounds__(32) k_refit(const float* W, int64_t rows, int6
     };
     for (int64_t c = 0; c < kRefitDepth - 1; ++c) issue(c);
     double sn = 0.0, sd = 0.0;
+    const double sg = DIST && lane < nr ? (double)sg_in[r0 + lane] : 0.0;
     for (int64_t c = 0; c < nch; ++c) {
         issue(c + kRefitDepth - 1);
         cp_async_wait<kRefitDepth - 1>();
@@ -280,7 +286,7 @@ __global__ void __launch_bounds__(32) k_refit(const float* W, int64_t rows, int6
         const int n = cols - 32 * c < 32 ? (int)(cols - 32 * c) : 32;
         const float* w = &rw[slot][lane][0];
         const int32_t* f = &rf[slot][lane][0];
-        for (int k0 = 0; k0 < n; k0 += 8) {
+        for (int k0 = 0; k0 < n && lane < nr; k0 += 8) {  // (lanes past the last row add nothing)
             const int32_t* v = f + kFields * (k0 >> 3);
             const double half_c = 0.5 * v[0];
             long long s7 = 0;
@@ -289,14 +295,103 @@ __global__ void __launch_bounds__(32) k_refit(const float* W, int64_t rows, int6
             for (int k = 0; k < m; ++k) {
                 const long long z = k < 7 ? (long long)v[1 + k] : 2LL * v[8] + (s7 & 1LL);
                 const double y = (double)z + half_c;
-                sn += (double)w[k0 + k] * y;
-                sd += y * y;
+                if constexpr (DIST) {
+                    const double er = (double)w[k0 + k] - sg * y;
+                    sn += er * er;
+                } else {
+                    sn += (double)w[k0 + k] * y;
+                    sd += y * y;
+                }
             }
         }
         __syncwarp();
     }
     cp_async_wait<0>();
-    if (lane < nr) scales[r0 + lane] = sd == 0.0 ? 0.0f : (float)(sn / sd);
+    if (lane < nr) {
+        if constexpr (DIST) dist[r0 + lane] = sn;
+        else scales[r0 + lane] = sd == 0.0 ? 0.0f : (float)(sn / sd);
+    }
+}
+
+// The refinement's admissibility: a row's candidate is admissible when every symbol lies in the
+// baseline tables' alphabets (ok[row] cleared otherwise; the caller sets it to 1 first).
+struct AlphaArgs {
+    int tmin[kTables];
+    uint32_t A[kTables];
+};
+__global__ void k_admissible(const int32_t* fields, int64_t nvec, int64_t nq, AlphaArgs aa, uint8_t* ok) {
+    for (int64_t g = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; g < nvec; g += (int64_t)gridDim.x * blockDim.x) {
+        const int32_t* v = fields + kFields * g;
+        bool in = true;
+#pragma unroll
+        for (int m = 0; m < kFields; ++m) {
+            const int t = table_index(m, v[0] & 1);
+            const int64_t i = (int64_t)v[m] - aa.tmin[t];
+            in = in && aa.A[t] != 0 && i >= 0 && i < (int64_t)aa.A[t];
+        }
+        if (!in) ok[g / nq] = 0;
+    }
+}
+
+// A row's ideal code length under tables (the refinement's rate): the cost of every symbol, in
+// vector and field order, summed in that order; cost = b - log2 f from a host-made table, b for
+// a symbol the tables give no frequency.  Same ring as k_rowpass, fields only.
+struct CostArgs {
+    int tmin[kTables];
+    uint32_t A[kTables];
+    uint32_t base[kTables];
+    double b;
+    const double* cost;
+};
+__global__ void __launch_bounds__(32) k_row_bits(const int32_t* fields, int64_t rows, int64_t nq, CostArgs ca,
+                                                  double* bits) {
+    __shared__ int32_t rf[kRefitDepth][32][37];
+    const int lane = threadIdx.x & 31;
+    const int64_t r0 = (int64_t)blockIdx.x * 32;
+    const int nr = rows - r0 < 32 ? (int)(rows - r0) : 32;
+    const int64_t nch = (nq + 3) / 4;
+    auto issue = [&](int64_t c) {
+        if (c < nch) {
+            const int slot = (int)(c % kRefitDepth);
+            const int64_t nv = nq - 4 * c < 4 ? nq - 4 * c : 4;
+            for (int rr = 0; rr < nr; ++rr) {
+                const int32_t* f = fields + kFields * ((r0 + rr) * nq + 4 * c);
+                if (lane < kFields * nv) cp_async4(&rf[slot][rr][lane], f + lane);
+                if (lane + 32 < kFields * nv) cp_async4(&rf[slot][rr][lane + 32], f + lane + 32);
+            }
+        }
+        cp_async_commit();
+    };
+    for (int64_t c = 0; c < kRefitDepth - 1; ++c) issue(c);
+    double acc = 0.0;
+    for (int64_t c = 0; c < nch; ++c) {
+        issue(c + kRefitDepth - 1);
+        cp_async_wait<kRefitDepth - 1>();
+        __syncwarp();
+        const int nv = nq - 4 * c < 4 ? (int)(nq - 4 * c) : 4;
+        const int32_t* f = &rf[(int)(c % kRefitDepth)][lane][0];
+        // lanes past the last row have no copies in the slot: they add nothing (their slots hold
+        // stale words, which must not index the tables)
+        for (int q = 0; q < nv && lane < nr; ++q) {
+            const int32_t* v = f + kFields * q;
+            for (int m = 0; m < kFields; ++m) {
+                const int t = table_index(m, v[0] & 1);
+                const int64_t i = (int64_t)v[m] - ca.tmin[t];
+                acc += (ca.A[t] != 0 && i >= 0 && i < (int64_t)ca.A[t]) ? ca.cost[ca.base[t] + (uint32_t)i] : ca.b;
+            }
+        }
+        __syncwarp();
+    }
+    cp_async_wait<0>();
+    if (lane < nr) bits[r0 + lane] = acc;
+}
+
+// fields[row] = candidate sel[row]'s fields of that row (candidates k-major, rows per candidate)
+__global__ void k_gather(const int32_t* cf, const int* sel, int64_t rows, int64_t rowf, int32_t* fields) {
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < rows * rowf; i += (int64_t)gridDim.x * blockDim.x) {
+        const int64_t r = i / rowf;
+        fields[i] = cf[(int64_t)sel[r] * rows * rowf + i];
+    }
 }
 
 // rANS, one warp per tile: lane j encodes the tile's lane j (vectors 32 r + j), steps in
@@ -500,7 +595,6 @@ __global__ void k_tile_index(int64_t T, const uint32_t* off, const uint32_t* sta
 ep_status check_encode_args(const void* W, int64_t rows, int64_t cols, double target_bpp, const ep_encode_opts& o,
                             int64_t& V, int64_t& T) {
     if (!W || rows <= 0 || cols <= 0 || !(target_bpp > 0.0)) return EP_EINVAL;
-    if (o.rdo_candidates > 1) return EP_EUNSUPPORTED;  // the per-row refinement stays on the CPU packer
     const int b = o.prob_bits > 0 ? o.prob_bits : (target_bpp <= 7.0 ? 11 : 12);
     if (b < kMinB || b > kMaxB) return EP_EINVAL;
     const int64_t nq = (cols + 7) / 8, nvec = rows * nq;
@@ -608,7 +702,106 @@ ep_status encode_core(cudaStream_t st, int nsm, const float* W, int64_t rows, in
         }
         break;
     }
-    k_refit<<<grid_for(rows, 32), 32, 0, st>>>(W, rows, cols, nq, d_fields.as<int32_t>(), r.scales.as<float>());
+    k_rowpass<false><<<grid_for(rows, 32), 32, 0, st>>>(W, rows, cols, nq, d_fields.as<int32_t>(), nullptr,
+                                                        r.scales.as<float>(), nullptr);
+
+    if (o.rdo_candidates > 1) {
+        // App. C.2, as the CPU packer's rdo_refine: candidates at rho_k s, each refitted, its
+        // distortion and admissibility; the rates priced under the current tables; the lambda
+        // bisection and the selection on the host (host::rdo_bisect); the tables rebuilt
+        const int K = o.rdo_candidates < 64 ? o.rdo_candidates : 64;
+        const int sweeps = o.rdo_sweeps > 0 ? o.rdo_sweeps : 1;
+        const int64_t rowf = kFields * nq;
+        double rho[64];
+        host::rdo_ratios(K, rho);
+        Table base[kTables];
+        if (g.count(d_fields.as<int32_t>(), nvec, al, base) != cudaSuccess) return EP_ECUDA;
+        for (int t = 0; t < kTables; ++t) host::normalise(base[t], b);
+        DevBuf d_cf, d_cs, d_cd, d_cr, d_ok, d_sel;
+        if (d_cf.alloc(sizeof(int32_t) * (size_t)K * (size_t)nvec * kFields, st) ||
+            d_cs.alloc(sizeof(float) * (size_t)K * rows, st) || d_cd.alloc(sizeof(double) * (size_t)K * rows, st) ||
+            d_cr.alloc(sizeof(double) * (size_t)K * rows, st) || d_ok.alloc((size_t)K * rows, st) ||
+            d_sel.alloc(sizeof(int) * rows, st) || cudaMemsetAsync(d_ok.p, 1, (size_t)K * rows, st))
+            return EP_ECUDA;
+        AlphaArgs aa;
+        for (int t = 0; t < kTables; ++t) {
+            aa.tmin[t] = base[t].min;
+            aa.A[t] = base[t].A;
+        }
+        auto cand = [&](int k) { return d_cf.as<int32_t>() + (size_t)k * (size_t)nvec * kFields; };
+        for (int k = 0; k < K; ++k) {
+            if (g.quantize(d_norms.as<double>(), nullptr, rows, rho[k] * s, cand(k)) != cudaSuccess) return EP_ECUDA;
+            k_rowpass<false><<<grid_for(rows, 32), 32, 0, st>>>(W, rows, cols, nq, cand(k), nullptr,
+                                                                d_cs.as<float>() + (size_t)k * rows, nullptr);
+            k_rowpass<true><<<grid_for(rows, 32), 32, 0, st>>>(W, rows, cols, nq, cand(k),
+                                                               d_cs.as<float>() + (size_t)k * rows, nullptr,
+                                                               d_cd.as<double>() + (size_t)k * rows);
+            k_admissible<<<std::min(grid_for(nvec, 256), 8 * nsm), 256, 0, st>>>(cand(k), nvec, nq, aa,
+                                                                               d_ok.as<uint8_t>() + (size_t)k * rows);
+        }
+        // every candidate's rate under `tabs` into out[k * rows + r] (k < nk)
+        auto price = [&](const Table* tabs, int nk, double* out) -> cudaError_t {
+            CostArgs ca;
+            std::vector<double> cost;
+            for (int t = 0; t < kTables; ++t) {
+                ca.tmin[t] = tabs[t].min;
+                ca.A[t] = tabs[t].A;
+                ca.base[t] = (uint32_t)cost.size();
+                for (uint32_t i = 0; i < tabs[t].A; ++i) {
+                    const uint32_t fr = tabs[t].freq[i];
+                    cost.push_back((double)b - std::log2((double)(fr ? fr : 1u)));
+                }
+            }
+            ca.b = (double)b;  // a symbol without a frequency: b - log2 1
+            DevBuf d_cost;
+            cudaError_t e = d_cost.alloc(sizeof(double) * std::max<size_t>(cost.size(), 1), st);
+            if (e == cudaSuccess && !cost.empty())
+                e = cudaMemcpyAsync(d_cost.p, cost.data(), sizeof(double) * cost.size(), cudaMemcpyHostToDevice, st);
+            if (e != cudaSuccess) return e;
+            ca.cost = d_cost.as<double>();
+            for (int k = 0; k < nk; ++k)
+                k_row_bits<<<grid_for(rows, 32), 32, 0, st>>>(cand(k), rows, nq, ca, d_cr.as<double>() + (size_t)k * rows);
+            e = cudaMemcpyAsync(out, d_cr.p, sizeof(double) * (size_t)nk * rows, cudaMemcpyDeviceToHost, st);
+            return e == cudaSuccess ? cudaStreamSynchronize(st) : e;
+        };
+        std::vector<double> cd((size_t)K * rows), cr((size_t)K * rows), rsel((size_t)rows);
+        std::vector<uint8_t> ok((size_t)K * rows);
+        std::vector<int> sel((size_t)rows, 0);
+        if (price(base, 1, rsel.data()) != cudaSuccess) return EP_ECUDA;  // the baseline's ideal code length
+        double budget = 0.0;
+        for (int64_t rr = 0; rr < rows; ++rr) budget += rsel[(size_t)rr];
+        if (cudaMemcpyAsync(cd.data(), d_cd.p, sizeof(double) * cd.size(), cudaMemcpyDeviceToHost, st) ||
+            cudaMemcpyAsync(ok.data(), d_ok.p, ok.size(), cudaMemcpyDeviceToHost, st) || cudaStreamSynchronize(st))
+            return EP_ECUDA;
+        const int nthreads = (int)std::max(1u, std::thread::hardware_concurrency());
+        Table next[kTables];
+        const Table* model = base;
+        for (int sw = 0; sw < sweeps; ++sw) {
+            if (price(model, K, cr.data()) != cudaSuccess) return EP_ECUDA;
+            for (size_t i = 0; i < cr.size(); ++i)
+                if (!ok[i]) cr[i] = INFINITY;
+            host::rdo_bisect(cd.data(), cr.data(), rows, K, budget, nthreads, sel.data());
+            if (cudaMemcpyAsync(d_sel.p, sel.data(), sizeof(int) * rows, cudaMemcpyHostToDevice, st)) return EP_ECUDA;
+            k_gather<<<std::min(grid_for(rows * rowf, 256), 16 * nsm), 256, 0, st>>>(d_cf.as<int32_t>(),
+                                                                                   d_sel.as<int>(), rows, rowf,
+                                                                                   d_fields.as<int32_t>());
+            Hist aln;
+            if (g.alphabet(d_fields.as<int32_t>(), nvec, aln) != cudaSuccess ||
+                g.count(d_fields.as<int32_t>(), nvec, aln, next) != cudaSuccess)
+                return EP_ECUDA;
+            for (int t = 0; t < kTables; ++t) host::normalise(next[t], b);
+            model = next;
+        }
+        // the chosen candidates' row scales
+        std::vector<float> cs((size_t)K * rows), sc((size_t)rows);
+        if (cudaMemcpyAsync(cs.data(), d_cs.p, sizeof(float) * cs.size(), cudaMemcpyDeviceToHost, st) ||
+            cudaStreamSynchronize(st))
+            return EP_ECUDA;
+        for (int64_t rr = 0; rr < rows; ++rr) sc[(size_t)rr] = cs[(size_t)sel[(size_t)rr] * rows + rr];
+        if (cudaMemcpyAsync(r.scales.p, sc.data(), sizeof(float) * rows, cudaMemcpyHostToDevice, st) ||
+            g.alphabet(d_fields.as<int32_t>(), nvec, al) != cudaSuccess)
+            return EP_ECUDA;
+    }
 
     if (g.count(d_fields.as<int32_t>(), nvec, al, r.tabs) != cudaSuccess) return EP_ECUDA;
     for (int t = 0; t < kTables; ++t) {

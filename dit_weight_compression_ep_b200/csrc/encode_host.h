@@ -57,6 +57,12 @@ struct Table {
 
 // Frequencies at 2^b from counts (fills freq and cum).
 void normalise(Table& tb, int b);
+// The per-row refinement's K candidate ratios (App. C.2), nested in K (K <= 64).
+void rdo_ratios(int K, double* rho);
+// The refinement's selection (App. C.2): bisect log2 lambda on [-80, 80] (64 steps) for the smallest
+// lambda whose per-row choices argmin_k cd[k][r] + lambda cr[k][r] (ties: lowest k; arrays k-major,
+// rows per candidate) have total rate <= budget; the last lambda's choices into sel[rows].
+void rdo_bisect(const double* cd, const double* cr, int64_t rows, int K, double budget, int nthreads, int* sel);
 // S of the pages' tile sizing for a target rate (V = max(32, S / 9)).
 int64_t tile_symbols_for(double target);
 // The rows of the scale search's sample, in sample order.

@@ -119,7 +119,9 @@ ep_status ep_encode_tensor(const float* W, int64_t rows, int64_t cols, double ta
  * stages on the GPU: row normalisation, the quantisation of the sampled rows
  * for every step of the scale search and of the whole tensor, the symbol
  * counts, the row-scale refit and the tiled rANS (one warp per tile).  The
- * search's decisions, the table normalisation and the header stay on the host.
+ * search's decisions, the table normalisation, the per-row refinement's lambda
+ * bisection (App. C.2; the candidates are quantised, refitted and priced on the
+ * GPU) and the header stay on the host.
  * The blob is byte for byte the one ep_encode_tensor returns for the same
  * matrix and options: every floating-point step is the host's operation in the
  * host's order, without multiply-add contraction, and the estimates' bits come
@@ -128,8 +130,7 @@ ep_status ep_encode_tensor(const float* W, int64_t rows, int64_t cols, double ta
  *   W       device, float32 [rows, cols] row-major, 4-byte aligned; not modified.  A
  *           pointer that is not device memory of the current device (or managed
  *           memory) is refused with EP_EINVAL before any launch.
- *   opts    as ep_encode_tensor; num_threads is ignored and rdo_candidates > 1
- *           (the per-row refinement) returns EP_EUNSUPPORTED.
+ *   opts    as ep_encode_tensor (num_threads is ignored).
  * Scratch is allocated with cudaMalloc and freed before the call returns (about
  * 36 + 18 bytes per vector of eight weights).  On EP_OK *out holds a host blob
  * (free with ep_free_blob).  Errors: EP_EINVAL, EP_EUNSUPPORTED, EP_EALPHABET,

@@ -127,7 +127,6 @@ def test_gpu_encoder_refuses_bad_arguments_on_host(lib):
     assert call(W=C.c_void_p(0x10002)) == EINVAL      # not 4-byte aligned
     assert call(prob_bits=16) == EINVAL
     assert call(prob_bits=8) == EINVAL
-    assert call(rdo=4) == EUNSUP                        # the per-row refinement stays on the CPU packer
     assert call(rows=1 << 20, cols=1 << 14) == EINVAL  # 2^31 vectors
 
 
@@ -146,7 +145,7 @@ def test_gpu_device_encoder_refuses_bad_arguments_on_host(lib):
     assert call(W=C.c_void_p(0x10001), bf16=1) == EINVAL   # bfloat16 needs 2
     assert call(rows=0) == EINVAL
     assert call(bpp=-1.0) == EINVAL
-    assert call(rdo=3) == EUNSUP
+    assert call(bf16=1, rows=1 << 20, cols=1 << 14) == EINVAL
     assert not d.payload and not d.tile_index
     lib.ep_free_device_blob(None)
     lib.ep_free_device_blob(C.byref(d))

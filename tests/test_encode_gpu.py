@@ -90,11 +90,18 @@ def test_dit_layers(kind, bpp):
     _same(synth.generate(synth.dit_stack_layer(1, kind)), bpp)
 
 
-def test_rdo_is_not_on_the_gpu_path():
-    import torch
+@pytest.mark.parametrize("K,sweeps,rows,cols", [(2, 1, 64, 512), (4, 2, 96, 1024), (5, 1, 17, 1001), (8, 3, 40, 256)])
+def test_per_row_refinement(K, sweeps, rows, cols):
+    """App. C.2 on the GPU: the packer's bytes for every candidate count and sweep count."""
+    rng = np.random.default_rng(K * 10 + sweeps)
+    W = np.empty((rows, cols), np.float32)
+    for r in range(rows):
+        W[r] = rng.standard_t([2.5, 4, 8, 30][r % 4], cols) * 0.02 * np.exp(rng.normal(0, 0.5))
+    _same(W, 3.0, rdo_candidates=K, rdo_sweeps=sweeps, tile_vectors=200)
 
-    with pytest.raises(ep.EntroPackError):
-        ep.encode_tensor_gpu(torch.zeros((8, 64), device="cuda"), 4.0, rdo_candidates=4)
+
+def test_per_row_refinement_full_size():
+    _same(synth.generate(synth.headline()), 3.0, rdo_candidates=4)
 
 
 @pytest.mark.parametrize("bpp", [2.0, 8.0])
