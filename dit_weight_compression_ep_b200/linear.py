@@ -13,7 +13,7 @@ prepared once, when the layer is built) and multiplies with the library GEMM thr
 Layers that run one after another can share one scratch buffer (pass the same tensor)."""
 from __future__ import annotations
 
-from ._lib import BF16, FP8_E4M3, INT8, DeviceBlob, _torch_dtype, decode_tensor_prepared, prepare_lut
+from ._lib import BF16, FP8_E4M3, INT8, DecodeBatch, DeviceBlob, _torch_dtype, decode_tensor_prepared, prepare_lut
 
 ROUTES = {"bf16": BF16, "fp8": FP8_E4M3, "int8": INT8}
 
@@ -49,12 +49,13 @@ class CompressedLinear:
         """Decode the weight into the scratch buffer (on `stream`, default torch's current stream)."""
         return decode_tensor_prepared(self.weight, self.lut, self.dtype, out=self.scratch, stream=stream)
 
-    def __call__(self, x, x_scale=None):
+    def __call__(self, x, x_scale=None, decode: bool = True):
         """x: [tokens, in_features]; bf16 for the bf16 route, float8_e4m3fn (fp8) or int8 (int8) with
-        x_scale [tokens, 1] float32 for the others.  Returns bf16 [tokens, out_features]."""
+        x_scale [tokens, 1] float32 for the others.  Returns bf16 [tokens, out_features].
+        decode=False multiplies by the scratch as it stands (a LinearGroup decoded it)."""
         import torch
 
-        W = self.decoded_weight()
+        W = self.decoded_weight() if decode else self.scratch
         if self.route == "bf16":
             y = torch.matmul(x, W.t())
         else:
@@ -67,3 +68,26 @@ class CompressedLinear:
         if self.bias is not None:
             y = y + self.bias
         return y
+
+
+class LinearGroup:
+    """Several CompressedLinear layers whose weights are decoded together in one launch
+    (ep_decode_batch: the SMs shared out among the weights), e.g. the linear layers of one
+    transformer block before the block runs.  The layers need distinct scratch buffers and one
+    route dtype; call the layers with decode=False after run()."""
+
+    def __init__(self, layers):
+        layers = list(layers)
+        if not layers:
+            raise ValueError("an empty group")
+        if len({lay.dtype for lay in layers}) != 1:
+            raise ValueError("the layers of a group share one route dtype")
+        ptrs = [lay.scratch.data_ptr() for lay in layers]
+        if len(set(ptrs)) != len(ptrs):
+            raise ValueError("the layers of a group need distinct scratch buffers")
+        self.layers = layers
+        self.batch = DecodeBatch([(lay.weight, lay.lut, lay.scratch) for lay in layers], layers[0].dtype)
+
+    def run(self, stream=None):
+        """Decode every layer's weight into its scratch (one launch on `stream`)."""
+        self.batch.run(stream=stream)

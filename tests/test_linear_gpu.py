@@ -86,3 +86,25 @@ def test_layers_sharing_one_scratch():
     with pytest.raises(ValueError):
         ep.CompressedLinear(ep.DeviceBlob(blobs[0]), "bf16", scratch=torch.empty(10, dtype=torch.bfloat16,
                                                                                   device="cuda"))
+
+
+def test_group_decode_then_calls():
+    """A LinearGroup decodes its layers' weights in one batch launch; the calls with decode=False
+    give the same bits as calls that decode one layer at a time."""
+    import torch
+
+    blobs = [ep.encode_tensor(synth.generate(synth.small_fp32(seed=s)), bpp) for s, bpp in ((7, 3.0), (8, 5.0),
+                                                                                               (9, 8.0))]
+    lins = [ep.CompressedLinear(ep.DeviceBlob(b), "bf16") for b in blobs]
+    group = ep.LinearGroup(lins)
+    x = (torch.randn(48, 512, device="cuda") * 0.5).to(torch.bfloat16)
+    for lin in lins:
+        lin.scratch.zero_()
+    group.run()
+    got = [lin(x, decode=False) for lin in lins]
+    want = [torch.matmul(x, _oracle_weight(b, ep.BF16, torch.bfloat16).t()) for b in blobs]
+    assert ep.decode_status() == 0
+    for g, w in zip(got, want):
+        assert torch.equal(g, w)
+    with pytest.raises(ValueError):
+        ep.LinearGroup([lins[0], lins[0]])  # one scratch twice
