@@ -131,8 +131,10 @@ ep_status ep_encode_tensor(const float* W, int64_t rows, int64_t cols, double ta
  *           pointer that is not device memory of the current device (or managed
  *           memory) is refused with EP_EINVAL before any launch.
  *   opts    as ep_encode_tensor (num_threads is ignored).
- * Scratch is allocated with cudaMalloc and freed before the call returns (about
- * 36 + 18 bytes per vector of eight weights).  On EP_OK *out holds a host blob
+ * Scratch (about 54 bytes per vector of eight weights, more with the per-row
+ * refinement: 36 per vector per candidate) comes in stream order from a memory
+ * pool the library creates per device, which keeps up to 1 GiB between calls
+ * and returns the rest to the device.  On EP_OK *out holds a host blob
  * (free with ep_free_blob).  Errors: EP_EINVAL, EP_EUNSUPPORTED, EP_EALPHABET,
  * EP_ENOMEM, EP_ECUDA.
  */
@@ -165,8 +167,9 @@ typedef struct {
  * weights are loaded to the GPU and compressed there.  W is float32 (w_is_bf16
  * = 0, 4-byte aligned) or bfloat16 (w_is_bf16 = 1, 2-byte aligned; widened to
  * float32 exactly on the GPU, so the bytes are those of the packer on the
- * widened matrix).  *out receives the arrays in new device allocations; the
- * scratch is freed before the call returns.  Errors as ep_encode_tensor_gpu
+ * widened matrix).  *out receives the arrays in new device allocations
+ * (cudaMalloc); the scratch comes from the same pool as ep_encode_tensor_gpu's
+ * (a bfloat16 matrix adds 4 bytes per weight).  Errors as ep_encode_tensor_gpu
  * (on an error *out is left empty).
  */
 ep_status ep_encode_tensor_gpu_device(void* stream, const void* W, int w_is_bf16, int64_t rows, int64_t cols,
