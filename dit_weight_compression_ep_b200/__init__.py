@@ -11,3 +11,4 @@ from ._lib import (BF16, FP16, FP8_E4M3, INT8, FP32, LATTICE_I32, UINT8, Blob, D
                    decode_tensor_prepared, encode_tensor, encode_tensor_gpu, encode_tensor_gpu_to_device, lib,
                    prepare_lut)
 from .linear import CompressedLinear, LinearGroup  # noqa: F401,E402
+from .package import load_package, load_package_to_device, save_package  # noqa: F401,E402
