@@ -328,6 +328,8 @@ class DeviceBlob:
         self.freq_tables = torch.from_numpy(blob.freq_tables).to(device)
         self.row_scales = torch.from_numpy(blob.row_scales).to(device)
         self.read_bytes = blob.stored_device_bytes()
+        self.payload_words, self.s = int(blob.payload_words), blob.s
+        self.stored_bpp, self.stored_bytes = blob.stored_bpp, blob.stored_bytes
 
 
 def _device_blob_to_host(self) -> Blob:

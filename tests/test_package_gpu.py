@@ -27,3 +27,15 @@ def test_load_package_to_device_and_decode(tmp_path):
         out = ep.decode_tensor(dev[name], ep.BF16)
         assert ep.decode_status() == 0
         assert_parity(to_raw(out), oracle_decode(blob, ep.BF16), ep.BF16, name)
+
+
+def test_device_blob_round_trips_to_host():
+    import torch
+
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    blob = ep.encode_tensor(synth.generate(synth.small_fp32(seed=10)), 5.0)
+    back = ep.DeviceBlob(blob).to_host()
+    np.testing.assert_array_equal(back.payload[:blob.payload_words], blob.payload[:blob.payload_words])
+    np.testing.assert_array_equal(back.tile_index, blob.tile_index)
+    assert (back.payload_words, back.s, back.stored_bytes) == (blob.payload_words, blob.s, blob.stored_bytes)
