@@ -325,6 +325,51 @@ def run_ours(args, rank: int, world: int, local_rank: int):
     if ep.decode_status(stream) != 0:
         raise RuntimeError("e2e decode reported a corrupt stream")
 
+    # ---- weight offload: each step streams the compressed layer from pinned host memory, decodes
+    # it on the GPU and reads 16 bytes of the result back (the weights are consumed on the GPU);
+    # beside it, the host-to-device time of the same layer in bf16
+    def off_step(i):
+        db, out, h_out, st = slots[i % 2]
+        with torch.cuda.stream(st):
+            db.payload.copy_(h_pay, non_blocking=True)
+            db.tile_index.copy_(h_tix, non_blocking=True)
+            db.freq_tables.copy_(h_ft, non_blocking=True)
+            db.row_scales.copy_(h_rs, non_blocking=True)
+            ep.decode_tensor(db, ep.BF16, out=out, stream=st)
+            h_probe[i % 2].copy_(out.view(-1)[:8], non_blocking=True)
+
+    h_probe = [torch.empty(8, dtype=torch.bfloat16).pin_memory() for _ in range(2)]
+    for i in range(3):
+        off_step(i)
+    torch.cuda.synchronize(dev)
+    if world > 1:
+        dist.barrier()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for _, _, _, st in slots:
+        st.wait_event(a)
+    for i in range(e2e_steps):
+        off_step(i)
+    for _, _, _, st in slots:
+        stream.wait_stream(st)
+    b.record(stream)
+    torch.cuda.synchronize(dev)
+    h_bf16 = torch.empty((blob.rows, blob.cols), dtype=torch.bfloat16).pin_memory()
+    d_bf16 = torch.empty_like(h_bf16, device=dev)
+    a2, b2 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        for _ in range(3):
+            d_bf16.copy_(h_bf16, non_blocking=True)
+        a2.record(stream)
+        for _ in range(e2e_steps):
+            d_bf16.copy_(h_bf16, non_blocking=True)
+        b2.record(stream)
+    torch.cuda.synchronize(dev)
+    off_ms, bf16_h2d_ms = reduce_max([a.elapsed_time(b) / e2e_steps, a2.elapsed_time(b2) / e2e_steps], world, dev)
+    del d_bf16, h_bf16
+    if ep.decode_status(stream) != 0:
+        raise RuntimeError("offload decode reported a corrupt stream")
+
     # ---- context: a torch bf16 matmul of the same layer with 4096 tokens
     X = torch.randn(4096, blob.cols, dtype=torch.bfloat16, device=dev)
     Wd = sets[0][1]
@@ -370,6 +415,12 @@ def run_ours(args, rank: int, world: int, local_rank: int):
                 "d2h_bytes_per_step": d2h, "steps": e2e_steps,
                 "how": "pinned host stream in, decode, pinned host weights out; two slots on two streams "
                        "alternate so one step's copy back overlaps the next step's copy in"},
+        "e2e_offload": {"value": round(weak_value(world, numel, off_ms), 3), "unit": UNIT, "ms_per_step": round(off_ms, 4),
+                        "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": 16,
+                        "bf16_h2d_ms_same_layer": round(bf16_h2d_ms, 4),
+                        "how": "each step: the compressed layer from pinned host memory, decoded on the GPU, 16 bytes "
+                               "of the result read back (weights consumed on the GPU); two slots on two streams; "
+                               "bf16_h2d_ms_same_layer: copying the same layer's bf16 weights instead"},
         "prepared": None if prep_ms is None else {
             "value": round(weak_value(world, numel, prep_ms), 2), "unit": UNIT, "ms_per_step": round(prep_ms, 5),
             "frac": round(alg_bytes / (prep_ms * 1e-3) / 1e9 / peak, 4),
