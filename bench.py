@@ -41,7 +41,7 @@ METRIC = "decoded G weights/s and achieved HBM GB/s vs B200 peak (BF16 out, 4 bp
 UNIT = "G weights/s"
 ROWS, COLS, TARGET = 3840, 10240, 4.0
 WORKLOAD = "3840x10240 bf16 Student-t(6)*0.02 weight (DiT FFN down projection), 4 bpp, decode to bf16"
-# the pages' 0.23 ms for a 39.3 M-weight layer, BF16 out, 4 bpp, on one H20 (context only)
+# the pages' 0.23 ms for a 39.3 M-weight layer, BF16 out, 4 bpp, on one H20 ([tables] Table 6; context only)
 PAGES_GWPS = 39321600 / 0.23e-3 / 1e9
 ROTATE = 4
 L2_BYTES = 126 * 1024 * 1024
