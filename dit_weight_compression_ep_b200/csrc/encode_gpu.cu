@@ -214,15 +214,16 @@ __global__ void __launch_bounds__(32 * kAlphaWarps) k_alphabet(const int32_t* fi
     }
 }
 
-// Counts of every table's symbols over vectors [0, nvec): per-CTA shared histograms when the
-// tables' bins fit (nbins <= kSmemBins), global atomics otherwise.
-constexpr int kSmemBins = 12288;
+// Counts of every table's symbols over vectors [0, nvec): per-CTA shared histograms (dynamic
+// shared memory, nbins words) when the tables' bins fit (nbins <= kSmemBins: up to 224 KiB, which
+// holds the alphabets of b <= 12 at high rates), global atomics otherwise.
+constexpr int kSmemBins = 56 * 1024;
 struct CountArgs {
     int tmin[kTables];
     uint32_t tbase[kTables];
 };
 __global__ void k_count(const int32_t* fields, int64_t nvec, CountArgs ca, uint32_t nbins, unsigned long long* counts) {
-    __shared__ uint32_t sh[kSmemBins];
+    extern __shared__ uint32_t sh[];
     const bool in_smem = nbins <= (uint32_t)kSmemBins;
     if (in_smem)
         for (uint32_t i = threadIdx.x; i < nbins; i += blockDim.x) sh[i] = 0;
@@ -551,7 +552,17 @@ struct GpuEncoder {
         if (nb > kMaxBins) return cudaErrorInvalidValue;  // alphabets are checked against 2^b first
         cudaError_t e = cudaMemsetAsync(d_counts.p, 0, sizeof(unsigned long long) * nb, st);
         if (e != cudaSuccess) return e;
-        k_count<<<std::min(grid_for(n, 256), 4 * nsm), 256, 0, st>>>(f, n, ca, nb, d_counts.as<unsigned long long>());
+        const bool in_smem = nb <= (uint32_t)kSmemBins;
+        const size_t smem = in_smem ? sizeof(uint32_t) * nb : 0;
+        if (in_smem && smem > 48 * 1024) {
+            e = cudaFuncSetAttribute(k_count, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     (int)(sizeof(uint32_t) * kSmemBins));
+            if (e != cudaSuccess) return e;
+        }
+        // grid: as many CTAs as fit with that much shared memory (at least one per SM)
+        const int per_sm = smem > 0 ? std::max(1, (int)((200 * 1024) / smem)) : 4;
+        k_count<<<std::min(grid_for(n, 256), std::min(4, per_sm) * nsm), 256, smem, st>>>(
+            f, n, ca, nb, d_counts.as<unsigned long long>());
         std::vector<unsigned long long> h(nb);
         e = cudaMemcpyAsync(h.data(), d_counts.p, sizeof(unsigned long long) * nb, cudaMemcpyDeviceToHost, st);
         if (e == cudaSuccess) e = cudaStreamSynchronize(st);
