@@ -1,4 +1,5 @@
-// encode_gpu.cu -- ep_encode_tensor_gpu: the packer with its full-tensor stages on the GPU.
+// encode_gpu.cu -- ep_encode_tensor_gpu (host blob out) and ep_encode_tensor_gpu_device
+// (device blob out; float32 or bfloat16 in): the packer with its full-tensor stages on the GPU.
 //
 // EntroPack paper §3.1 pipeline, as in encode.cpp: row normalisation, the sampled-row scale
 // search (§3.4, App. C.1), full-tensor E8 quantisation (§1, Conway & Sloane 1982), the row-scale
@@ -20,10 +21,10 @@
 
 #include <algorithm>
 #include <climits>
-#include <mutex>
-#include <thread>
 #include <cmath>
+#include <mutex>
 #include <new>
+#include <thread>
 #include <vector>
 
 #include "encode_host.h"
