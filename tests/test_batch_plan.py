@@ -89,3 +89,27 @@ def test_batch_create_and_launch_refuse_bad_arguments():
     assert lib.ep_batch_create(arr, 1, 7, C.byref(h)) == EUNSUP
     assert lib.ep_decode_batch(None, None) == EINVAL
     lib.ep_batch_free(None)
+
+
+def test_share_out_properties_random():
+    """Random batches: every tensor gets 1..T SMs; together they use all SMs unless the tensors have
+    fewer tiles than that; the share-out is deterministic.  (It may depend on the tensors' order
+    where the cost model ties, e.g. tensors of one tile per warp, where more SMs change nothing.)"""
+    from hypothesis import given, settings
+    from hypothesis import strategies as st
+
+    tensor = st.tuples(st.integers(1, 20000), st.sampled_from([32, 455, 910, 1820, 3640]),
+                       st.sampled_from([9, 10, 11, 12, 13]))
+
+    @settings(max_examples=200, deadline=None)
+    @given(st.lists(tensor, min_size=1, max_size=40), st.integers(40, 160))
+    def check(ts, G):
+        T = [t[0] for t in ts]
+        V = [t[1] for t in ts]
+        b = [t[2] for t in ts]
+        c = ep.batch_apportion(T, V, b, G)
+        assert all(1 <= ci <= ti for ci, ti in zip(c, T))
+        assert sum(c) == min(G, sum(T))
+        assert c == ep.batch_apportion(T, V, b, G)
+
+    check()
