@@ -151,6 +151,43 @@ def test_gpu_device_encoder_refuses_bad_arguments_on_host(lib):
     lib.ep_free_device_blob(C.byref(d))
 
 
+def test_a_c_program_links_and_calls_the_library(tmp_path, lib):
+    """A plain C99 program links against libentropack.so and calls it through the header: status
+    strings and calls the host refuses before any CUDA work (safe on any machine)."""
+    import shutil
+    import subprocess
+
+    from dit_weight_compression_ep_b200 import build as b
+
+    cc = shutil.which("gcc") or shutil.which("cc")
+    if cc is None:
+        pytest.skip("no C compiler")
+    src = tmp_path / "use.c"
+    src.write_text(r"""
+#include <stdio.h>
+#include <string.h>
+#include "entropack.h"
+int main(void) {
+    if (strcmp(ep_status_string(EP_OK), "ok") != 0) return 1;
+    if (ep_decode_tensor(NULL, NULL, NULL, NULL, NULL, 64, 64, EP_BF16, NULL) != EP_EINVAL) return 2;
+    if (ep_decode_prepare(NULL, NULL, 64, 64, NULL, EP_LUT_BYTES) != EP_EINVAL) return 3;
+    ep_blob* out = NULL;
+    if (ep_encode_tensor(NULL, 4, 4, 4.0, NULL, &out) != EP_EINVAL || out != NULL) return 4;
+    int64_t T = 10, V = 100; int bb = 11, counts[1];
+    if (ep_batch_apportion(1, &T, &V, &bb, 148, counts) != EP_OK || counts[0] != 10) return 5;
+    ep_free_blob(NULL);
+    printf("c ok\n");
+    return 0;
+}
+""")
+    exe = tmp_path / "use"
+    libdir = os.path.dirname(b.SO)
+    subprocess.run([cc, "-std=c99", "-Wall", "-Werror", "-I", os.path.join(ROOT, "include"), str(src), "-o", str(exe),
+                    "-L", libdir, "-l:" + os.path.basename(b.SO), "-Wl,-rpath," + libdir], check=True)
+    r = subprocess.run([str(exe)], capture_output=True, text=True)
+    assert r.returncode == 0 and r.stdout.strip() == "c ok", (r.returncode, r.stdout, r.stderr)
+
+
 def test_header_compiles_as_c99(tmp_path):
     """include/entropack.h is a C header: every declaration compiles as strict C99."""
     import shutil
