@@ -320,3 +320,23 @@ def convert(x: np.ndarray, dtype: int) -> np.ndarray:
     out = np.zeros(x.size, _NP_OUT[dtype])
     lib().epo_convert(_p(x), x.size, dtype, _p(out))
     return out
+
+
+def linear(W: np.ndarray, x: np.ndarray) -> np.ndarray:
+    """A linear layer's output y = x W^T in float64, from the weight's decoded values ([paper] §4.3,
+    Fig. 5: the weight is reconstructed, then multiplied).  The reference for decode-then-GEMM and
+    for a GEMM that decodes its weight operand itself; the matrix product is the library's, on
+    float64 copies of the inputs."""
+    return np.asarray(x, np.float64) @ np.asarray(W, np.float64).T
+
+
+def linear_tolerance(W: np.ndarray, x: np.ndarray, out_unit: float) -> np.ndarray:
+    """Per-element bound on |y_gemm - y| for a GEMM that forms exact products and accumulates in
+    float32 in any order, then rounds to an output format of unit roundoff out_unit: the standard
+    dot-product bound gamma_K sum|x_k w_k| (gamma_K = K u / (1 - K u), u = 2^-24, K the inner
+    dimension), plus out_unit |y| for the final rounding."""
+    K = np.asarray(W).shape[1]
+    u = 2.0 ** -24
+    gamma = K * u / (1.0 - K * u)
+    absdot = np.abs(np.asarray(x, np.float64)) @ np.abs(np.asarray(W, np.float64)).T
+    return gamma * absdot * (1.0 + out_unit) + out_unit * np.abs(linear(W, x))
