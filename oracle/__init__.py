@@ -1,9 +1,12 @@
 """Plain CPU oracle of the EntroPack codec (TEST INFRASTRUCTURE).
 
 Only the tests, ``__graft_entry__.smoke()`` and the CPU-baseline leg of
-``bench.py`` may import this package.  The arithmetic lives in ``ep_oracle.c``
-(plain C, double precision, no threads, no SIMD); this module only builds it and
-marshals numpy arrays through ctypes.  It shares nothing with the library in
+``bench.py`` may import this package.  The codec's arithmetic lives in
+``ep_oracle.c`` (plain C, double precision, no threads, no SIMD); this module
+builds it and marshals numpy arrays through ctypes.  The one function written
+here is ``linear`` (with ``linear_tolerance``): the float64 product of a decoded
+weight, which is the reference for a linear layer (pinned in
+``tests/test_oracle_linear.py``).  It shares nothing with the library in
 ``dit_weight_compression_ep_b200``.
 
 Each C function cites the passage of the EntroPack paper it follows; the header
