@@ -108,3 +108,29 @@ def test_group_decode_then_calls():
         assert torch.equal(g, w)
     with pytest.raises(ValueError):
         ep.LinearGroup([lins[0], lins[0]])  # one scratch twice
+
+
+def test_bf16_route_within_the_fp64_oracle_bound():
+    """The bf16 route against the float64 product of the oracle's decoded weight, within the bound
+    for float32 accumulation in any order plus the bf16 output rounding."""
+    import torch
+
+    import oracle
+
+    W = synth.generate(synth.headline())[:256, :2048].copy()
+    blob = ep.encode_tensor(W, 4.0)
+    lin = ep.CompressedLinear(ep.DeviceBlob(blob), "bf16")
+    x = (torch.randn(64, 2048, device="cuda") * 0.5).to(torch.bfloat16)
+    # the bound assumes float32 accumulation: no reduced-precision split-K reductions
+    keep = torch.backends.cuda.matmul.allow_bf16_reduced_precision_reduction
+    torch.backends.cuda.matmul.allow_bf16_reduced_precision_reduction = False
+    try:
+        y = lin(x).float().cpu().numpy().astype(np.float64)
+    finally:
+        torch.backends.cuda.matmul.allow_bf16_reduced_precision_reduction = keep
+    Wd = oracle.decode_blob(blob, oracle.FP32).astype(np.float32)  # exact: sigma * y in float32
+    Wb = torch.from_numpy(Wd).to(torch.bfloat16).float().numpy()     # the bf16 weight the route multiplies
+    xb = x.float().cpu().numpy()
+    ref = oracle.linear(Wb, xb)
+    tol = oracle.linear_tolerance(Wb, xb, 2.0 ** -8)
+    assert np.all(np.abs(y - ref) <= tol)
