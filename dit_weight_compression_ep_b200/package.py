@@ -8,7 +8,8 @@ Layout (all little-endian, the library's stored representation unchanged):
   `<layer>.row_scales`   F32  one per row
 The safetensors metadata holds the format name and, per layer, its shape and geometry (rows,
 cols, b, V, tiles, payload words, the search's scale, stored bytes and bpp).  The sidecar repeats
-that and adds the package totals: numel, stored bytes and bpp = 8 * sum(stored bytes) / sum(numel).
+that and adds the package totals: numel, stored bytes, bpp = 8 * sum(stored bytes) / sum(numel)
+and the linear-weight compression ratio against bf16, bpp / 16 (the pages' two package metrics).
 """
 from __future__ import annotations
 
@@ -50,8 +51,9 @@ def save_package(path: str, blobs: dict, extra: dict | None = None) -> dict:
     numel = sum(v["rows"] * v["cols"] for v in layers.values())
     stored = sum(v["stored_bytes"] for v in layers.values())
     save_file(tensors, path, metadata={"format": FORMAT, "layers": json.dumps(layers, sort_keys=True)})
+    bpp = 8.0 * stored / numel if numel else 0.0
     side = {"format": FORMAT, "package": os.path.basename(path), "layers": layers, "numel": numel,
-            "stored_bytes": stored, "bpp": 8.0 * stored / numel if numel else 0.0}
+            "stored_bytes": stored, "bpp": bpp, "ratio_vs_bf16": bpp / 16.0}
     if extra is not None:
         side["extra"] = extra
     with open(_sidecar_path(path), "w") as f:

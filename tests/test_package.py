@@ -44,6 +44,7 @@ def test_round_trip_and_sidecar(tmp_path, blobs):
     numel = sum(b.rows * b.cols for b in blobs.values())
     stored = sum(b.stored_bytes for b in blobs.values())
     assert side["bpp"] == pytest.approx(8.0 * stored / numel) and side["extra"] == {"note": "synthetic"}
+    assert side["ratio_vs_bf16"] == pytest.approx(side["bpp"] / 16.0)
 
 
 def test_plain_safetensors_reads_it(tmp_path, blobs):
