@@ -32,10 +32,16 @@
  *             cursor, code length near the entropy), tile layout (Table 5),
  *             dtype conversions (library conversions; the INT8 and UINT8
  *             readings on their own edge cases and numpy), splitmix64 (published
- *             outputs), refit (least-squares optimality), normalise_freqs (sum,
- *             support and rounding invariants), scale search (rate lands near
- *             target, bracket property), stored bytes (closed form).
- *   parity unpinned (readings with no page value to check against): the choice
+ *             outputs), refit (least-squares optimality), normalize_freqs
+ *             (hand-worked counts -> frequencies of the reading below; sum,
+ *             support and coding-loss invariants on random counts),
+ *             sample_rows (a partial Fisher-Yates draw worked by hand from
+ *             published generator outputs; draws uniform over orders and rows),
+ *             scale search (rate lands near target, bracket property), stored
+ *             bytes (closed form).
+ *   parity unpinned (readings with no page value to check against; the pins
+ *             above check that the code follows each reading, not the reading
+ *             itself): the choice
  *             of row normaliser (RMS), the frequency normalisation rule, the
  *             sampling generator and order, the tie-breaks, the lane interleave
  *             order and the header byte layout.  They change the encoder's
