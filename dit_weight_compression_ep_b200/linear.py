@@ -73,7 +73,7 @@ class CompressedLinear:
 class LinearGroup:
     """Several CompressedLinear layers whose weights are decoded together in one launch
     (ep_decode_batch: the SMs shared out among the weights), e.g. the linear layers of one
-    transformer block before the block runs.  The layers need distinct scratch buffers and one
+    transformer block before the block runs.  The layers need non-overlapping scratch buffers and one
     route dtype; call the layers with decode=False after run()."""
 
     def __init__(self, layers):
@@ -82,9 +82,11 @@ class LinearGroup:
             raise ValueError("an empty group")
         if len({lay.dtype for lay in layers}) != 1:
             raise ValueError("the layers of a group share one route dtype")
-        ptrs = [lay.scratch.data_ptr() for lay in layers]
-        if len(set(ptrs)) != len(ptrs):
-            raise ValueError("the layers of a group need distinct scratch buffers")
+        # the batch writes every weight at once: the scratch byte ranges must not overlap
+        spans = sorted((lay.scratch.data_ptr(), lay.scratch.data_ptr() + lay.scratch.numel() * lay.scratch.element_size())
+                       for lay in layers)
+        if any(nxt[0] < cur[1] for cur, nxt in zip(spans, spans[1:])):
+            raise ValueError("the layers of a group need scratch buffers that do not overlap")
         self.layers = layers
         self.batch = DecodeBatch([(lay.weight, lay.lut, lay.scratch) for lay in layers], layers[0].dtype)
 

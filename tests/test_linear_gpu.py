@@ -108,6 +108,14 @@ def test_group_decode_then_calls():
         assert torch.equal(g, w)
     with pytest.raises(ValueError):
         ep.LinearGroup([lins[0], lins[0]])  # one scratch twice
+    # two views of one buffer at different offsets that overlap by a few elements
+    n = blobs[0].rows * blobs[0].cols
+    buf = torch.empty(2 * n - 16, dtype=torch.bfloat16, device="cuda")
+    a = ep.CompressedLinear(ep.DeviceBlob(blobs[0]), "bf16", scratch=buf[:n])
+    b = ep.CompressedLinear(ep.DeviceBlob(blobs[1]), "bf16", scratch=buf[n - 16:])
+    with pytest.raises(ValueError):
+        ep.LinearGroup([a, b])
+    ep.LinearGroup([a, ep.CompressedLinear(ep.DeviceBlob(blobs[1]), "bf16")])  # disjoint: accepted
 
 
 def test_bf16_route_within_the_fp64_oracle_bound():
@@ -128,9 +136,14 @@ def test_bf16_route_within_the_fp64_oracle_bound():
         y = lin(x).float().cpu().numpy().astype(np.float64)
     finally:
         torch.backends.cuda.matmul.allow_bf16_reduced_precision_reduction = keep
-    Wd = oracle.decode_blob(blob, oracle.FP32).astype(np.float32)  # exact: sigma * y in float32
-    Wb = torch.from_numpy(Wd).to(torch.bfloat16).float().numpy()     # the bf16 weight the route multiplies
+    # the oracle's own bf16 decode (its conversion is written from the format definition)
+    Wbits = oracle.decode_blob(blob, oracle.BF16).astype(np.uint32) << 16
+    Wb = Wbits.view(np.float32).astype(np.float64)
     xb = x.float().cpu().numpy()
     ref = oracle.linear(Wb, xb)
     tol = oracle.linear_tolerance(Wb, xb, 2.0 ** -8)
+    # the decoder may differ from the oracle by one bf16 unit in the last place per weight
+    # (the pages' tolerance for float outputs): sum_k |x_k| ulp(W_jk) more
+    ulp = np.ldexp(1.0, np.frexp(np.abs(Wb))[1] - 8)
+    tol = tol + np.abs(xb.astype(np.float64)) @ ulp.T
     assert np.all(np.abs(y - ref) <= tol)

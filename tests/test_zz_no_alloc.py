@@ -59,6 +59,10 @@ def test_noalloc_matches_decode_tensor_on_two_calls(which):
             assert ep.decode_status() == 0
             # the tests' tolerance: bit-exact against the existing entry point
             np.testing.assert_array_equal(_raw(out), want, err_msg=f"{which} dtype {dt} call {call}")
+        # the package's Python wrapper of the same entry point (argument order and types)
+        got = ep.decode_tensor_noalloc(db, dt)
+        assert ep.decode_status() == 0
+        np.testing.assert_array_equal(_raw(got), want, err_msg=f"{which} dtype {dt} through the wrapper")
 
 
 def test_noalloc_rejects_bad_sizes_on_host():
