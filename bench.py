@@ -150,6 +150,21 @@ def reduce_max(values, world: int, device=None):
     return [float(v) for v in t.cpu()]
 
 
+def relaunch(n: int, script: str, argv, timeout_s: float = 3600.0, capture: bool = False):
+    """Run `script argv` as n ranks on this node under torchrun, with a loopback rendezvous, and
+    wait for them: `bench.py --gpus N` does this when no launcher started it (every rank then
+    reads RANK / LOCAL_RANK / WORLD_SIZE from its environment).  Returns the CompletedProcess."""
+    import socket
+    import subprocess
+
+    with socket.socket() as so:
+        so.bind(("127.0.0.1", 0))
+        port = so.getsockname()[1]
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", f"--nproc-per-node={n}",
+           "--master-addr=127.0.0.1", f"--master-port={port}", script, *argv]
+    return subprocess.run(cmd, timeout=timeout_s, capture_output=capture, text=capture)
+
+
 def weak_value(world: int, units_per_rank: int, ms_per_step: float) -> float:
     """Whole-job throughput in G units/s: every rank's units over the slowest rank's step time."""
     return world * units_per_rank / (ms_per_step * 1e-3) / 1e9
@@ -474,7 +489,7 @@ def cpu_baseline(blob, seconds: float = 10.0):
                       f"{cores} threads, {dt:.1f} s"}
 
 
-def run_reference(args):
+def run_reference(args, world: int = 1):
     """The oracle as the reference arm: CPU decode, each step a bounded tile sample."""
     import oracle
 
@@ -497,7 +512,7 @@ def run_reference(args):
     value = weights / dt / 1e9
     sample = (f"tiles 0..{ranges[-1][1]} of the {blob.ntiles}-tile stream per step "
               f"({weights / args.steps / 1e6:.1f} M weights), {cores} threads")
-    return {"metric": METRIC, "value": round(value, 5), "unit": UNIT, "n_gpus": args.gpus, "steps": args.steps,
+    return {"metric": METRIC, "value": round(value, 5), "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": round(dt / args.steps * 1e3, 3), "higher_is_better": True,
             "scaling": "weak", "vs_baseline": round(value / PAGES_GWPS, 6), "dtype": "u32+f32", "data": "synthetic",
             "config": {"workload": WORKLOAD, "rows": ROWS, "cols": COLS, "target_bpp": TARGET, "out": "bf16"},
@@ -994,9 +1009,17 @@ def main():
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
+    if args.gpus < 1:
+        ap.error("--gpus must be at least 1")
+    one_gpu_mode = args.sweep or args.linear or args.dit or args.encode
+    if args.gpus > 1 and "WORLD_SIZE" not in os.environ and not one_gpu_mode:
+        # no launcher: start the N ranks here (one process per GPU) and pass on their status
+        sys.exit(relaunch(args.gpus, os.path.abspath(__file__), sys.argv[1:]).returncode)
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if not one_gpu_mode and world != args.gpus:
+        ap.error(f"--gpus {args.gpus}, but the launcher started {world} rank(s)")
 
     if args.sweep:
         run_sweep(args)
@@ -1013,7 +1036,7 @@ def main():
     if args.impl == "reference":
         if rank != 0:
             return
-        res = run_reference(args)
+        res = run_reference(args, world)
         print(json.dumps(res), flush=True)
         return
 
@@ -1026,6 +1049,8 @@ def main():
         torch.cuda.set_device(local_rank)
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
                                 device_id=torch.device("cuda", local_rank))
+        if dist.get_world_size() != args.gpus:  # the ranks NCCL sees are the GPUs the line reports
+            raise SystemExit(f"NCCL sees {dist.get_world_size()} ranks, --gpus {args.gpus}")
     try:
         res = run_ours(args, rank, world, local_rank)
     finally:

@@ -86,7 +86,7 @@ def test_reference_arm_prints_on_rank_zero_only(monkeypatch):
     monkeypatch.setattr(sys, "argv", ["bench.py", "--impl", "reference", "--gpus", "2", "--steps", "1",
                                       "--warmup", "3"])
     called = []
-    monkeypatch.setattr(bench, "run_reference", lambda args: called.append(args) or {})
+    monkeypatch.setattr(bench, "run_reference", lambda args, world: called.append(args) or {})
     buf = io.StringIO()
     with redirect_stdout(buf):
         bench.main()
@@ -99,7 +99,7 @@ def test_reference_arm_rank_zero_prints_one_line(monkeypatch):
     monkeypatch.setenv("LOCAL_RANK", "0")
     monkeypatch.setattr(sys, "argv", ["bench.py", "--impl", "reference", "--gpus", "2", "--steps", "1",
                                       "--warmup", "3"])
-    monkeypatch.setattr(bench, "run_reference", lambda args: {"impl": "reference", "n_gpus": args.gpus})
+    monkeypatch.setattr(bench, "run_reference", lambda args, world: {"impl": "reference", "n_gpus": world})
     buf = io.StringIO()
     with redirect_stdout(buf):
         bench.main()
@@ -118,3 +118,40 @@ def test_ranks_decode_distinct_tensors():
 
     a, b = synth.headline(seed=7 + 0), synth.headline(seed=7 + 1)
     assert (a.rows, a.cols) == (b.rows, b.cols) and a.seed != b.seed
+
+
+def test_gpus_must_match_the_launched_ranks(monkeypatch):
+    monkeypatch.setenv("RANK", "0")
+    monkeypatch.setenv("WORLD_SIZE", "2")
+    monkeypatch.setenv("LOCAL_RANK", "0")
+    monkeypatch.setattr(sys, "argv", ["bench.py", "--gpus", "4", "--warmup", "3"])
+    with pytest.raises(SystemExit):
+        bench.main()
+
+
+def test_gpus_two_without_a_launcher_starts_two_ranks(monkeypatch):
+    """bench.py --gpus 2 run directly re-launches itself as two ranks; nothing runs here."""
+    seen = []
+    monkeypatch.delenv("WORLD_SIZE", raising=False)
+    monkeypatch.setattr(sys, "argv", ["bench.py", "--gpus", "2", "--steps", "5", "--warmup", "3"])
+    monkeypatch.setattr(bench, "relaunch", lambda n, script, argv: seen.append((n, script, list(argv))) or
+                        type("R", (), {"returncode": 0})())
+    with pytest.raises(SystemExit) as ex:
+        bench.main()
+    assert ex.value.code == 0
+    assert seen == [(2, os.path.abspath(bench.__file__), ["--gpus", "2", "--steps", "5", "--warmup", "3"])]
+
+
+def test_relaunch_runs_two_gloo_ranks_with_the_timing_reduction():
+    """The launch path itself: two ranks under torchrun on CPU (gloo), each timing its own step,
+    the max over ranks taken by bench.reduce_max, one JSON line from rank 0 with n_gpus = 2."""
+    probe = os.path.join(os.path.dirname(os.path.abspath(__file__)), "rank_probe.py")
+    res = bench.relaunch(2, probe, ["--units", "1000000"], timeout_s=300, capture=True)
+    assert res.returncode == 0, res.stderr[-2000:]
+    lines = [ln for ln in res.stdout.splitlines() if ln.startswith("{")]
+    assert len(lines) == 1, res.stdout
+    out = json.loads(lines[0])
+    assert out["n_gpus"] == 2 and out["ranks_seen"] == 2
+    # rank 1 sleeps longer: the step time is the slower rank's, the value counts both ranks' units
+    assert out["ms_per_step"] >= out["rank_ms"][1] >= out["rank_ms"][0]
+    assert out["value"] == pytest.approx(bench.weak_value(2, 1000000, out["ms_per_step"]))
