@@ -69,15 +69,16 @@ def _kernel_sha():
 
 
 def _traffic_per_launch():
-    """DRAM bytes per launch from the committed ncu summary, if it was taken on this kernel source."""
+    """(DRAM bytes per launch, bytes the SMs wrote into L2 per launch) from the committed ncu
+    summary, if it was taken on this kernel source; (None, None) otherwise."""
     try:
         with open(os.path.join(ROOT, "profiles", "decode_headline_traffic.json")) as f:
             d = json.load(f)
         if d.get("kernel_sha") == _kernel_sha():
-            return float(d["dram_bytes_per_launch"])
+            return float(d["dram_bytes_per_launch"]), float(d["l2_write_bytes_from_sm"])
     except Exception:
         pass
-    return None
+    return None, None
 
 
 class Clocks:
@@ -407,7 +408,7 @@ def run_ours(args, rank: int, world: int, local_rank: int):
     peak, peak_kind = _peaks()
     alg_bytes = read_bytes + write_bytes
     achieved = alg_bytes / (avg_launch_ms * 1e-3) / 1e9
-    traffic = _traffic_per_launch()
+    traffic, l2_writes = _traffic_per_launch()
     cpu = cpu_baseline(blob, seconds=args.cpu_seconds) if world == 1 else None
     return {
         "metric": METRIC, "value": round(value, 2), "unit": UNIT, "n_gpus": world, "steps": args.steps,
@@ -423,6 +424,10 @@ def run_ours(args, rank: int, world: int, local_rank: int):
                    "encode_s": round(t_enc, 3)},
         "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
                      "frac": round(achieved / peak, 4), "traffic": traffic,
+                     "traffic_note": "dram read + write of one ncu capture; the write side is low because the "
+                                     "output is still dirty in L2 when the launch ends: the SMs' write sectors "
+                                     "into L2 are in sm_write_bytes_into_l2",
+                     "sm_write_bytes_into_l2": l2_writes,
                      "algorithmic_bytes_per_launch": alg_bytes, "read_bytes": read_bytes, "write_bytes": write_bytes,
                      "avg_launch_us": round(avg_launch_ms * 1e3, 3), "peak_kind": peak_kind},
         "cpu_baseline": cpu,
@@ -995,6 +1000,95 @@ def run_linear(args):
               f"{100 * r['overhead']:.1f} % |")
 
 
+PROBE_CHAINS = [
+    ("imad", "mad.lo.u32 (state update, addresses)"),
+    ("lds32+imad", "32-bit shared load (lookup-table entry) + its address multiply-add"),
+    ("lds16+imad", "16-bit shared load (payload word) + its address multiply-add"),
+    ("vote+imad", "and + compare + vote.ballot, folded back with a multiply-add"),
+    ("popc+imad", "popc, folded back with a multiply-add"),
+    ("shfl", "shift + shfl.idx (source lane from the value)"),
+    ("vote+and+popc+imad", "the renormalisation's word index"),
+    ("vote+and+popc+imad+lds16", "the word index, then the word's shared load"),
+    ("vote+and+popc+shfl+add", "the word index, then a shuffle instead of the address and load"),
+    ("redux+imad", "redux.sync.add, folded back with a multiply-add"),
+]
+
+
+def run_chain(args):
+    """The decode's chain latency and fixed cost: tensors of exactly one tile per SM (so one
+    warp per SM, nothing to hide a step's latency behind), at four tile sizes; a straight line
+    through (steps per tile, time) gives the fixed cost per call and the cycles per symbol step
+    at the sampled SM clock.  Also times the 3840x10240 headline the same way (eager launches,
+    four rotating copies).  Prints one JSON line."""
+    import numpy as np
+    import torch
+
+    import dit_weight_compression_ep_b200 as ep
+    from dit_weight_compression_ep_b200 import build
+
+    build.build()
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    rng = np.random.default_rng(0)
+
+    def timed(db, outs, n):
+        for i in range(5):
+            ep.decode_tensor(db, ep.BF16, out=outs[i % len(outs)])
+        torch.cuda.synchronize()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        for i in range(n):
+            ep.decode_tensor(db, ep.BF16, out=outs[i % len(outs)])
+        b.record()
+        torch.cuda.synchronize()
+        return a.elapsed_time(b) / n * 1e3
+
+    pts = []
+    for V in (320, 640, 1280, 2560):
+        W = (rng.standard_t(6, (sms * V // 128, 1024)) * 0.02).astype(np.float32)
+        blob = ep.encode_tensor(W, TARGET, tile_vectors=V, prob_bits=11)
+        assert blob.ntiles == sms
+        db = ep.DeviceBlob(blob)
+        outs = [torch.empty((blob.rows, blob.cols), dtype=torch.bfloat16, device="cuda")]
+        pts.append((9 * ((V + 31) // 32), timed(db, outs, 30)))
+    A = np.array([[1.0, s] for s, _ in pts])
+    (fixed, per), *_ = np.linalg.lstsq(A, np.array([u for _, u in pts]), rcond=None)
+    mhz = torch.cuda.clock_rate() if hasattr(torch.cuda, "clock_rate") else None
+    hb = ep.encode_tensor(_make_weights(), TARGET)
+    hdb = ep.DeviceBlob(hb)
+    houts = [torch.empty((hb.rows, hb.cols), dtype=torch.bfloat16, device="cuda") for _ in range(4)]
+    head = timed(hdb, houts, 50)
+    print(json.dumps({"chain": {"fixed_us": round(float(fixed), 2), "us_per_step": round(float(per), 5),
+                                "cycles_per_step_at_1965_mhz": round(float(per) * 1965, 1),
+                                "points_steps_us": [(s, round(u, 2)) for s, u in pts], "sm_clock_query_mhz": mhz},
+                      "headline_eager_us": round(head, 2)}), flush=True)
+
+
+def run_latency(args):
+    """Latencies of the operations on the decode step's dependent chain on this GPU: one warp,
+    dependent chains timed with clock64 (csrc/latency_probe.cu).  Prints a table and one JSON
+    line; the single operations follow by subtracting the multiply-add chain."""
+    import ctypes as C
+
+    from dit_weight_compression_ep_b200 import build
+
+    L = C.CDLL(build.build_probe())
+    L.ep_probe_latencies.argtypes = [C.POINTER(C.c_double), C.c_int]
+    L.ep_probe_latencies.restype = C.c_int
+    out = (C.c_double * len(PROBE_CHAINS))()
+    rc = L.ep_probe_latencies(out, len(PROBE_CHAINS))
+    if rc:
+        raise SystemExit(f"latency probe failed: CUDA error {rc}")
+    cyc = {name: round(out[k], 1) for k, (name, _) in enumerate(PROBE_CHAINS)}
+    imad = cyc["imad"]
+    print("| chain | cycles per iteration |\n|---|---|")
+    for name, what in PROBE_CHAINS:
+        print(f"| {what} | {cyc[name]} |")
+    derived = {"imad": imad, "lds32": round(cyc["lds32+imad"] - imad, 1), "lds16": round(cyc["lds16+imad"] - imad, 1),
+               "popc": round(cyc["popc+imad"] - imad, 1), "vote_with_and_setp": round(cyc["vote+imad"] - imad, 1),
+               "redux": round(cyc["redux+imad"] - imad, 1)}
+    print(json.dumps({"latency_cycles": cyc, "derived": derived}), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -1006,12 +1100,14 @@ def main():
     ap.add_argument("--linear", action="store_true", help="decode-then-GEMM against a resident weight (one GPU)")
     ap.add_argument("--dit", action="store_true", help="the whole DiT stack: per layer, prepared, block batches")
     ap.add_argument("--encode", action="store_true", help="conversion speed: CPU packer and GPU encoder")
+    ap.add_argument("--latency", action="store_true", help="latencies of the decode step's operations (one GPU)")
+    ap.add_argument("--chain", action="store_true", help="decode chain latency and fixed cost per call (one GPU)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
     if args.gpus < 1:
         ap.error("--gpus must be at least 1")
-    one_gpu_mode = args.sweep or args.linear or args.dit or args.encode
+    one_gpu_mode = args.sweep or args.linear or args.dit or args.encode or args.latency or args.chain
     if args.gpus > 1 and "WORLD_SIZE" not in os.environ and not one_gpu_mode:
         # no launcher: start the N ranks here (one process per GPU) and pass on their status
         sys.exit(relaunch(args.gpus, os.path.abspath(__file__), sys.argv[1:]).returncode)
@@ -1032,6 +1128,12 @@ def main():
         return
     if args.encode:
         run_encode(args)
+        return
+    if args.latency:
+        run_latency(args)
+        return
+    if args.chain:
+        run_chain(args)
         return
     if args.impl == "reference":
         if rank != 0:

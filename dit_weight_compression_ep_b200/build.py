@@ -1,4 +1,5 @@
-"""Build libentropack.so in-tree: the CUDA decoder (sm_100a) and the C++ packer.
+"""Build libentropack.so in-tree: the CUDA decoder (sm_100a) and the C++ packer; and
+libep_probe.so, the latency probe behind `bench.py --latency` (not part of the codec).
 
     python -m dit_weight_compression_ep_b200.build [--force] [--verbose]
 """
@@ -13,6 +14,8 @@ ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 SO = os.path.join(HERE, "libentropack.so")
+PROBE_SO = os.path.join(HERE, "libep_probe.so")
+PROBE_SRC = os.path.join(CSRC, "latency_probe.cu")
 BUILD = os.path.join(ROOT, "_build")
 
 CU_SOURCES = ["decode.cu", "encode_gpu.cu"]
@@ -63,7 +66,18 @@ def build(force: bool = False, verbose: bool = False) -> str:
     tmp = SO + f".tmp{os.getpid()}"
     subprocess.check_call([NVCC, *ARCH, "-shared", "-Xcompiler", "-fPIC", "-o", tmp, *objs, "-lpthread"])
     os.replace(tmp, SO)
+    build_probe(force)
     return SO
+
+
+def build_probe(force: bool = False) -> str:
+    """The latency probe as its own small library."""
+    if force or not os.path.exists(PROBE_SO) or os.path.getmtime(PROBE_SO) < os.path.getmtime(PROBE_SRC):
+        tmp = PROBE_SO + f".tmp{os.getpid()}"
+        subprocess.check_call([NVCC, *ARCH, "-O3", "-std=c++17", "-shared", "-Xcompiler", "-fPIC", PROBE_SRC,
+                               "-o", tmp])
+        os.replace(tmp, PROBE_SO)
+    return PROBE_SO
 
 
 if __name__ == "__main__":

@@ -524,11 +524,19 @@ struct Out<EP_FP32> {
 // table (2(k-1) + c).  Entry, low to high: f in B+1 bits (F) or f - 1 in B bits,
 // then z with an even bias (31 - 2B or 32 - 2B bits), then slot - cum in the top
 // B bits, so that f and slot - cum each come out in one operation.
+//
+// decode<K> returns the entry shifted right so that bits 1.. hold z + bias (kZMask
+// selects them, bit 0 is cleared by the mask): twice the biased coordinate, ready to be
+// OR-ed into the float magic of the reconstruction with the coset bit in bit 0.  For the
+// last field (m) the shift is one less, so that kZMask << 1 gives four times it.
 template <int B, bool F>
 struct PackedLut {
     static constexpr uint32_t kM = 1u << B;
     static constexpr int kB = B;
+    static constexpr bool kPacked = true;
     static constexpr uint32_t kZBias = F ? (1u << (30 - 2 * B)) : (1u << (31 - 2 * B));
+    static constexpr int kZShift = F ? B : B - 1;  // entry bit of z's lowest bit, minus one
+    static constexpr uint32_t kZMask = ((1u << (F ? 31 - 2 * B : 32 - 2 * B)) - 1u) << 1;
     uint32_t lut_s;
     uint32_t four;  // 4 and 2^32 - 4 * 2^B: run-time values, so that the address
     uint32_t m4;    // arithmetic stays integer multiply-adds
@@ -540,14 +548,13 @@ struct PackedLut {
         const uint32_t e = ld_s32<(2 * (K - 1)) * (int)kM * 4>(a);
         const uint32_t f = e & (F ? 2u * kM - 1u : kM - 1u);
         const uint32_t bias = e >> (32 - B);
-        const uint32_t zb = (e << B) >> (F ? 2 * B + 1 : 2 * B);
         if constexpr (F) {
             x = f * xs + bias;
         } else {
             x = f * xs + (xs + bias);
         }
         (void)bad;
-        return zb;
+        return K < 8 ? e >> kZShift : e >> (kZShift - 1);
     }
 };
 
@@ -558,6 +565,7 @@ struct PackedLut {
 template <bool PAIR>
 struct TwoLut {
     static constexpr int kB = 0;
+    static constexpr bool kPacked = false;
     static constexpr uint32_t kZBias = 0;
     uint32_t lut_s;  // slot table (tables in the order 2(k-1) + c)
     uint32_t b, mmask, half;  // b, 2^b - 1, 2 * entries per table (bytes per table)
@@ -594,6 +602,7 @@ struct TwoLut {
 // COARSE: 16 tables x 2^k buckets x 64-bit {cum | f << 16, z}; runtime b.
 struct CoarseLut {
     static constexpr int kB = 0;
+    static constexpr bool kPacked = false;
     static constexpr uint32_t kZBias = 0;
     uint32_t lut_s;  // shared address
     uint32_t b, mmask, sh, nb_shift;
@@ -742,15 +751,31 @@ __device__ __forceinline__ void tile_begin(const TileCtx& tc, const uint16_t* ti
 template <bool FULL>
 __device__ __forceinline__ void renorm(uint32_t& x, uint32_t xn, bool act, uint32_t& pb, uint32_t lt,
                                        const TileCtx& tc) {
-    const bool need = (FULL || act) && xn < kStateLow;
+    if constexpr (FULL) {
+        // every lane active: one predicate feeds the ballot, the word load and a predicated
+        // multiply-add that appends the word (x = xn otherwise)
+        asm("{\n\t.reg .pred p;\n\t.reg .b32 bal, t, w;\n\t"
+            "setp.lt.u32 p, %2, 32768;\n\t"
+            "vote.sync.ballot.b32 bal, p, -1;\n\t"
+            "and.b32 t, bal, %3;\n\t"
+            "popc.b32 t, t;\n\t"
+            "mad.lo.u32 t, t, %4, %1;\n\t"
+            "ld.shared.u16 w, [t];\n\t"
+            "mov.b32 %0, %2;\n\t"
+            "@p mad.lo.u32 %0, %2, %5, w;\n\t"
+            "popc.b32 t, bal;\n\t"
+            "mad.lo.u32 %1, t, %4, %1;\n\t}"
+            : "=r"(x), "+r"(pb)
+            : "r"(xn), "r"(lt), "r"(tc.two), "r"(tc.k64)
+            : "memory");
+        (void)act;
+        return;
+    }
+    const bool need = act && xn < kStateLow;
     const uint32_t bal = __ballot_sync(kFull, need);
     const uint32_t w = ld_s16(__popc(bal & lt) * tc.two + pb);
     const uint32_t xr = xn * tc.k64 + w;  // (xn << 16) | w
-    if (FULL) {
-        x = need ? xr : xn;
-    } else if (act) {
-        x = need ? xr : xn;
-    }
+    if (act) x = need ? xr : xn;
     pb = __popc(bal) * tc.two + pb;
 }
 
@@ -776,18 +801,31 @@ __device__ __forceinline__ void decode_round(void* out, const float sigma, const
     const auto cb = lut.coset_base(c & 1);
     bool badsym = false;
     const uint32_t magic = 0x4AC00000u + (uint32_t)c - 2u * Lut::kZBias;
+    // packed tables: 0x4AC00000 (1.5 * 2^22) has no bits below bit 22, so the coset bit and
+    // twice the biased coordinate are OR-ed in; the bias moves into the float subtraction
+    const uint32_t kc = 0x4AC00000u | (uint32_t)c;
+    constexpr float kYOff = 6291456.0f + (float)Lut::kZBias;  // exact: below 2^23
     uint32_t yb[8];
     float wf[8];
     uint32_t s7 = 0;
     uint32_t xn;
     // each coordinate's bits as soon as its field is known, so that this work can fill
-    // the gaps of the state chain
+    // the gaps of the state chain; the parity of z1..z7 is bit 1 of the XOR of the packed
+    // tables' shifted entries (the bias is even), or bit 0 of the sum of the others' z
 #define EP_FIELD(K)                                               \
     xn = x;                                                       \
     {                                                             \
         const uint32_t z_ = lut.template decode<K>(xn, cb, badsym); \
         renorm<FULL>(x, xn, act, pb, lt, tc);                     \
-        if (K < 8) {                                              \
+        if constexpr (Lut::kPacked) {                             \
+            if (K < 8) {                                          \
+                yb[K - 1] = (z_ & Lut::kZMask) | kc;              \
+                wf[K - 1] = sigma * (__uint_as_float(yb[K - 1]) - kYOff); \
+                s7 ^= z_;                                         \
+            } else {                                              \
+                yb[7] = (z_ & (Lut::kZMask << 1)) + (s7 & 2u) + (magic - 2u * Lut::kZBias); \
+            }                                                     \
+        } else if (K < 8) {                                       \
             yb[K - 1] = z_ * tc.two + magic;                      \
             wf[K - 1] = sigma * (__uint_as_float(yb[K - 1]) - 6291456.0f); \
             s7 += z_;                                             \
@@ -807,6 +845,9 @@ __device__ __forceinline__ void decode_round(void* out, const float sigma, const
     tl.x = x;
     if (badsym && act) corrupt = true;
 
+    // lattice output: 2y = the bits above the magic (coordinates 1..7 of packed tables
+    // carry twice their bias)
+    constexpr uint32_t kLat = 0x4AC00000u + (Lut::kPacked ? 2u * Lut::kZBias : 0u);
     if (act) {
         if constexpr (RAGGED) {
             // vector g holds elements row * cols + 8q .. of a row padded to whole vectors
@@ -816,7 +857,7 @@ __device__ __forceinline__ void decode_round(void* out, const float sigma, const
             if constexpr (DT == EP_LATTICE_I32) {
 #pragma unroll
                 for (int k = 0; k < 8; ++k)  // constant indices keep yb in registers
-                    if (k < n) reinterpret_cast<int*>(out)[e0 + k] = (int)(yb[k] - 0x4AC00000u);
+                    if (k < n) reinterpret_cast<int*>(out)[e0 + k] = (int)(yb[k] - (k < 7 ? kLat : 0x4AC00000u));
             } else {
                 wf[7] = sigma * (__uint_as_float(yb[7]) - 6291456.0f);
 #pragma unroll
@@ -825,9 +866,8 @@ __device__ __forceinline__ void decode_round(void* out, const float sigma, const
             }
         } else if constexpr (DT == EP_LATTICE_I32) {
             int4* o = reinterpret_cast<int4*>(out) + 2 * g;
-            o[0] = make_int4((int)(yb[0] - 0x4AC00000u), (int)(yb[1] - 0x4AC00000u), (int)(yb[2] - 0x4AC00000u),
-                             (int)(yb[3] - 0x4AC00000u));
-            o[1] = make_int4((int)(yb[4] - 0x4AC00000u), (int)(yb[5] - 0x4AC00000u), (int)(yb[6] - 0x4AC00000u),
+            o[0] = make_int4((int)(yb[0] - kLat), (int)(yb[1] - kLat), (int)(yb[2] - kLat), (int)(yb[3] - kLat));
+            o[1] = make_int4((int)(yb[4] - kLat), (int)(yb[5] - kLat), (int)(yb[6] - kLat),
                              (int)(yb[7] - 0x4AC00000u));
         } else {
             wf[7] = sigma * (__uint_as_float(yb[7]) - 6291456.0f);
@@ -1170,8 +1210,18 @@ __device__ __forceinline__ void decode_body(const Params& p, const uint32_t cta,
     run_decode<DT, RAGGED>(p, g, lut_s, fq, s_min, s_A, s_off, desc2, tc, rg, tl, first_i);
 }
 
+// With programmatic dependent launch (the prepared and batched decodes) the grid may start
+// while the kernel ahead of it in the stream is ending: wait for it before any global read,
+// and let the next kernel's launch go ahead (it waits the same way).  Without that launch
+// attribute (the cooperative per-call decode) both are no-ops.
+__device__ __forceinline__ void grid_dependency_wait() {
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 template <int DT, bool RAGGED>
 __global__ void __launch_bounds__(kThreads, 1) decode_kernel(Params p) {
+    grid_dependency_wait();
     decode_body<DT, RAGGED, false>(p, blockIdx.x, gridDim.x);
 }
 
@@ -1184,6 +1234,7 @@ struct alignas(16) BatchCta {
 
 template <int DT, bool RAGGED>
 __global__ void __launch_bounds__(kThreads, 1) decode_batch_kernel(const BatchCta* plan) {
+    grid_dependency_wait();
     const BatchCta c = plan[blockIdx.x];
     if (c.count == 0) return;
     decode_body<DT, RAGGED, true>(c.p, c.rank, c.count);
@@ -1309,11 +1360,18 @@ cudaError_t launch_decode(const Params& prm, cudaStream_t st, int num_sms) {
     cfg.dynamicSmemBytes = kSmemBytes;
     cfg.stream = st;
     cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeCooperative;
-    attr[0].val.cooperative = 1;
+    if (prm.prepared) {
+        // a prepared table needs no grid barrier: an ordinary launch that may be scheduled
+        // while the kernel ahead of it in the stream ends (programmatic dependent launch)
+        attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[0].val.programmaticStreamSerializationAllowed = 1;
+    } else {
+        // the grid barrier needs every CTA co-resident (a cooperative launch)
+        attr[0].id = cudaLaunchAttributeCooperative;
+        attr[0].val.cooperative = 1;
+    }
     cfg.attrs = attr;
-    // the grid barrier needs every CTA co-resident (a cooperative launch); a prepared table needs none
-    cfg.numAttrs = prm.prepared ? 0 : 1;
+    cfg.numAttrs = 1;
     return (prm.cols & 7) ? cudaLaunchKernelEx(&cfg, decode_kernel<DT, true>, prm)
                           : cudaLaunchKernelEx(&cfg, decode_kernel<DT, false>, prm);
 }
@@ -1337,6 +1395,11 @@ cudaError_t launch_batch(const BatchCta* plan, int ctas, bool ragged, cudaStream
     cfg.blockDim = dim3(kThreads);
     cfg.dynamicSmemBytes = kSmemBytes;
     cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;  // as a prepared decode
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
     return ragged ? cudaLaunchKernelEx(&cfg, decode_batch_kernel<DT, true>, plan)
                   : cudaLaunchKernelEx(&cfg, decode_batch_kernel<DT, false>, plan);
 }

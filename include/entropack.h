@@ -189,8 +189,13 @@ void ep_free_blob(ep_blob* blob);
  *   tiles        device, the payload; 16-byte aligned; the buffer must be
  *                readable up to the final offset rounded up to a multiple of 8
  *                words (the packer's payload_alloc_words).
- *   tile_index   device, uint32[33*T + 1], 4-byte aligned.
- *   freq_tables  device, the table header and frequencies, 16-byte aligned.
+ *   tile_index   device, uint32[33*T + 1], 4-byte aligned.  Its last word, the
+ *                final payload offset, is trusted: it must not exceed the words the
+ *                tiles buffer holds (the signature carries no payload length, so
+ *                the kernel bounds every payload read by that word and by the
+ *                tile offsets, which it checks against it).
+ *   freq_tables  device, the table header and frequencies, 16-byte aligned.  The
+ *                buffer must hold the frequencies its header describes.
  *   row_scales   device, float32[rows].
  *   rows, cols   the matrix shape; must match the header.
  *   out_dtype    one of ep_dtype.
@@ -200,10 +205,13 @@ void ep_free_blob(ep_blob* blob);
  * All buffers belong to the caller.  The library keeps one 128 KB workspace
  * per device (allocated with cudaMalloc and zeroed on the first call on that
  * device, so make the first call before any stream capture); every CTA writes
- * its share of the decode lookup table there and reads the whole table back.
- * Decodes on one device are ordered through that workspace: a call waits on
- * the GPU for the previous call, whatever stream it ran on (not applied while
- * the stream is being captured).
+ * its share of the decode lookup table there and reads the whole table back
+ * (a table built once across the grid costs less than one built in every
+ * CTA).  Decodes on one device are ordered through that workspace: a call
+ * waits on the GPU for the previous call, whatever stream it ran on (not
+ * applied while the stream is being captured), so per-call decodes on two
+ * streams run one after the other; prepared-table and batched decodes use no
+ * workspace and may overlap.
  * The call is asynchronous: it validates the arguments on the host and makes
  * one cooperative launch on the stream (one CTA per SM).  Argument errors
  * return at once (EP_EINVAL, EP_EUNSUPPORTED), launch errors as EP_ECUDA.  The
@@ -276,6 +284,9 @@ ep_status ep_decode_prepare(void* stream, const uint8_t* freq_tables, int64_t ro
  * The call uses no library workspace and no grid-wide barrier: it makes one
  * ordinary launch on the stream (one CTA per SM), so decodes on different
  * streams may run at the same time and nothing orders them but their streams.
+ * The launch allows programmatic dependent launch: the kernel may be scheduled
+ * while the kernel ahead of it in the stream is ending, and it waits for that
+ * kernel to complete before its first global-memory access.
  * A table whose layout does not match this tensor's header (b, LUT format, or
  * any table's minimum or alphabet size), or a buffer ep_decode_prepare did not
  * write, raises EP_ECORRUPT in the status word and nothing is decoded.  A table
@@ -335,7 +346,8 @@ ep_status ep_batch_create(const ep_batch_item* items, int n_items, ep_dtype out_
 
 /*
  * ep_decode_batch -- one launch on `stream` (an ordinary launch, one CTA per
- * SM) that decodes every tensor of the batch into its `out`.  Outputs, status
+ * SM, with programmatic dependent launch as ep_decode_tensor_prepared's) that
+ * decodes every tensor of the batch into its `out`.  Outputs, status
  * reporting and the checks of each tensor's header and table are those of
  * ep_decode_tensor_prepared.  The current device must be the one the batch was
  * created on (else EP_EINVAL).  Capturable in a CUDA graph.

@@ -134,6 +134,39 @@ def test_tiny_and_negative_scales():
     _check(blob, ALL_DT, "tiny scales")
 
 
+def test_two_tensors_on_two_streams_at_once():
+    """Two tensors decoded over and over on two streams with no ordering between the streams:
+    per call (the library orders its per-call decodes through its workspace) and with
+    prepared tables (no shared state: the launches may overlap on the GPU).  Every output
+    equals the oracle."""
+    import torch
+
+    blobs = [ep.encode_tensor(synth.generate(synth.headline())[:1024, :4096].copy(), 4.0),
+             ep.encode_tensor(synth.generate(synth.dit_attn_proj())[:2048, :2048].copy(), 8.0)]
+    dbs = [ep.DeviceBlob(b) for b in blobs]
+    outs = [torch.zeros((b.rows, b.cols), dtype=torch.bfloat16, device="cuda") for b in blobs]
+    streams = [torch.cuda.Stream(), torch.cuda.Stream()]
+    torch.cuda.synchronize()
+    ep.decode_status()
+    for _ in range(6):
+        for db, out, st in zip(dbs, outs, streams):
+            ep.decode_tensor(db, ep.BF16, out=out, stream=st)
+    torch.cuda.synchronize()
+    assert ep.decode_status() == 0
+    for b, out in zip(blobs, outs):
+        assert_parity(to_raw(out), oracle_decode(b, ep.BF16), ep.BF16, "two streams, per call")
+    luts = [ep.prepare_lut(db) for db in dbs]
+    pouts = [torch.zeros_like(o) for o in outs]
+    torch.cuda.synchronize()
+    for _ in range(6):
+        for db, lut, out, st in zip(dbs, luts, pouts, streams):
+            ep.decode_tensor_prepared(db, lut, ep.BF16, out=out, stream=st)
+    torch.cuda.synchronize()
+    assert ep.decode_status() == 0
+    for b, out in zip(blobs, pouts):
+        assert_parity(to_raw(out), oracle_decode(b, ep.BF16), ep.BF16, "two streams, prepared")
+
+
 def test_repeat_on_side_stream():
     import torch
 
