@@ -566,10 +566,11 @@ template <bool PAIR>
 struct TwoLut {
     static constexpr int kB = 0;
     static constexpr bool kPacked = false;
+    static constexpr bool kYbDirect = true;
     static constexpr uint32_t kZBias = 0;
     uint32_t lut_s;  // slot table (tables in the order 2(k-1) + c)
     uint32_t b, mmask, half;  // b, 2^b - 1, 2 * entries per table (bytes per table)
-    uint32_t desc_s;          // shared address of {record address, min} per table (same order)
+    uint32_t desc_s;          // shared address of {record address, 0x4AC00000 + c + 2 min (4 min for m)}
     const uint32_t* s_A;      // alphabet sizes, for the escape walk
     __device__ __forceinline__ uint32_t coset_base(int c) const { return (uint32_t)c; }
     template <int K>
@@ -595,7 +596,8 @@ struct TwoLut {
         const uint32_t c0 = ld_s16(ra), c1 = ld_s16(ra + 2u);
         x = (c1 - c0) * xs + (slot - c0);
         (void)bad;
-        return s + d.y;
+        // the coordinate's bits: 0x4AC00000 + 2z + c (fields 1..7), 0x4AC00000 + 4m + c (m)
+        return s * (K < 8 ? 2u : 4u) + d.y;
     }
 };
 
@@ -603,6 +605,7 @@ struct TwoLut {
 struct CoarseLut {
     static constexpr int kB = 0;
     static constexpr bool kPacked = false;
+    static constexpr bool kYbDirect = false;
     static constexpr uint32_t kZBias = 0;
     uint32_t lut_s;  // shared address
     uint32_t b, mmask, sh, nb_shift;
@@ -824,6 +827,14 @@ __device__ __forceinline__ void decode_round(void* out, const float sigma, const
                 s7 ^= z_;                                         \
             } else {                                              \
                 yb[7] = (z_ & (Lut::kZMask << 1)) + (s7 & 2u) + (magic - 2u * Lut::kZBias); \
+            }                                                     \
+        } else if constexpr (Lut::kYbDirect) {                    \
+            if (K < 8) {                                          \
+                yb[K - 1] = z_;                                   \
+                wf[K - 1] = sigma * (__uint_as_float(yb[K - 1]) - 6291456.0f); \
+                s7 ^= z_;                                         \
+            } else {                                              \
+                yb[7] = z_ + (s7 & 2u);                           \
             }                                                     \
         } else if (K < 8) {                                       \
             yb[K - 1] = z_ * tc.two + magic;                      \
@@ -1073,7 +1084,8 @@ __device__ __forceinline__ void decode_body(const Params& p, const uint32_t cta,
         const uint32_t A0 = __shfl_sync(kFull, A, 0);
         if (t >= 1 && t < kTables)
             reinterpret_cast<uint2*>(smem + kOffDesc2)[t - 1] =
-                make_uint2(smem_u32(smem + kOffLut + kTwoRec) + 2u * (incl - A - A0 + (uint32_t)(t - 1)), (uint32_t)lane_mn);
+                make_uint2(smem_u32(smem + kOffLut + kTwoRec) + 2u * (incl - A - A0 + (uint32_t)(t - 1)),
+                           0x4AC00000u + (uint32_t)((t - 1) & 1) + (uint32_t)lane_mn * (t >= 15 ? 4u : 2u));
     }
     // a prepared table: its trailer's loads go out now, with the prologue's other loads
     uint2 fp = make_uint2(0u, 0u);
