@@ -155,3 +155,20 @@ def test_relaunch_runs_two_gloo_ranks_with_the_timing_reduction():
     # rank 1 sleeps longer: the step time is the slower rank's, the value counts both ranks' units
     assert out["ms_per_step"] >= out["rank_ms"][1] >= out["rank_ms"][0]
     assert out["value"] == pytest.approx(bench.weak_value(2, 1000000, out["ms_per_step"]))
+
+
+def test_workload_option_names_its_target_and_description():
+    import argparse
+
+    head = bench._workload(argparse.Namespace(workload="headline"))
+    assert head == (bench.TARGET, bench.WORKLOAD)
+    for name, (bpp, desc) in bench.OTHER_WORKLOADS.items():
+        assert bench._workload(argparse.Namespace(workload=name)) == (bpp, desc)
+        assert "8 bpp" in desc and "b = 12" in desc
+
+
+def test_reference_arm_refuses_other_workloads(monkeypatch):
+    monkeypatch.delenv("WORLD_SIZE", raising=False)
+    monkeypatch.setattr(sys, "argv", ["bench.py", "--impl", "reference", "--workload", "dit-qkv-8", "--warmup", "3"])
+    with pytest.raises(SystemExit):
+        bench.main()
