@@ -3,6 +3,7 @@
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
     python bench.py --sweep      (every workload, one GPU: a table, not the bench line)
     python bench.py --linear     (decode-then-GEMM against a resident weight, one GPU)
+    python bench.py --gemv       (the fused decode-GEMV on 1 to 8 tokens, one GPU)
 
 One step = one ep_decode_tensor call: the whole hot path (tile setup, table
 staging, payload staging, rANS decode, lattice reconstruction, row rescale,
@@ -1023,6 +1024,69 @@ def run_linear(args):
               f"{100 * r['overhead']:.1f} % |")
 
 
+def run_gemv(args):
+    """A linear layer on 1, 2, 4 and 8 tokens whose weight is decoded inside the product
+    (ep_decode_gemv, prepared table and per call), against decoding the weight to BF16 with the
+    prepared table and then the GEMM (cuBLAS through torch), and against the GEMM on a resident BF16
+    weight.  The 3840x10240 layer at 4 bpp; each time is the minimum of 15 runs, each after a
+    256 MiB L2 flush.  Prints JSON lines and a markdown table."""
+    import torch
+
+    import dit_weight_compression_ep_b200 as ep
+    from dit_weight_compression_ep_b200 import build, synth
+
+    build.build()
+    dev = torch.device("cuda")
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+
+    def tmin(fn, runs=15):
+        for _ in range(3):
+            fn()
+        ts = []
+        for _ in range(runs):
+            flush.zero_()
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record()
+            fn()
+            b.record()
+            torch.cuda.synchronize()
+            ts.append(a.elapsed_time(b))
+        return min(ts) * 1e3
+
+    W = synth.generate(synth.headline())
+    rows, cols = W.shape
+    blob = ep.encode_tensor(W, TARGET)
+    db = ep.DeviceBlob(blob)
+    lut = ep.prepare_lut(db)
+    Wb = torch.from_numpy(W).to(dev).to(torch.bfloat16)
+    Wd = torch.empty_like(Wb)
+    stream_bytes = blob.stored_device_bytes()
+    out = []
+    for ntok in ep.GEMV_TOKENS:
+        x = torch.randn(ntok, cols, device=dev) * 0.5
+        xb = x.to(torch.bfloat16)
+        y = torch.empty(ntok, rows, device=dev)
+        t_res = tmin(lambda: torch.matmul(xb, Wb.t()))
+        t_fused = tmin(lambda: ep.decode_gemv(db, x, lut=lut, y=y))
+        t_fused_call = tmin(lambda: ep.decode_gemv(db, x, y=y))
+        t_dec = tmin(lambda: ep.decode_tensor_prepared(db, lut, ep.BF16, out=Wd))
+        t_both = tmin(lambda: torch.matmul(xb, ep.decode_tensor_prepared(db, lut, ep.BF16, out=Wd).t()))
+        if ep.decode_status() != 0:
+            raise RuntimeError("decode reported a corrupt stream")
+        r = {"tokens": ntok, "gemv_resident_bf16_us": round(t_res, 2), "fused_prepared_us": round(t_fused, 2),
+             "fused_per_call_us": round(t_fused_call, 2), "decode_prepared_us": round(t_dec, 2),
+             "decode_then_gemm_us": round(t_both, 2), "fused_vs_decode_then_gemm": round(t_both / t_fused, 3),
+             "fused_hbm_gbs": round((stream_bytes + x.nbytes + y.nbytes) / (t_fused * 1e-6) / 1e9, 1)}
+        out.append(r)
+        print(json.dumps(r), flush=True)
+    print("\n| tokens | GEMV, BF16 weight resident (µs) | fused decode-GEMV, prepared (µs) | fused, per call (µs) | "
+          "decode (µs) | decode then GEMM (µs) | decode then GEMM / fused |")
+    print("|---|---|---|---|---|---|---|")
+    for r in out:
+        print(f"| {r['tokens']} | {r['gemv_resident_bf16_us']} | {r['fused_prepared_us']} | {r['fused_per_call_us']} | "
+              f"{r['decode_prepared_us']} | {r['decode_then_gemm_us']} | {r['fused_vs_decode_then_gemm']} |")
+
+
 PROBE_CHAINS = [
     ("imad", "mad.lo.u32 (state update, addresses)"),
     ("lds32+imad", "32-bit shared load (lookup-table entry) + its address multiply-add"),
@@ -1121,6 +1185,7 @@ def main():
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--sweep", action="store_true", help="every workload's decode throughput (one GPU)")
     ap.add_argument("--linear", action="store_true", help="decode-then-GEMM against a resident weight (one GPU)")
+    ap.add_argument("--gemv", action="store_true", help="the fused decode-GEMV on 1 to 8 tokens (one GPU)")
     ap.add_argument("--dit", action="store_true", help="the whole DiT stack: per layer, prepared, block batches")
     ap.add_argument("--encode", action="store_true", help="conversion speed: CPU packer and GPU encoder")
     ap.add_argument("--latency", action="store_true", help="latencies of the decode step's operations (one GPU)")
@@ -1132,7 +1197,7 @@ def main():
         ap.error("--warmup must be at least 3")
     if args.gpus < 1:
         ap.error("--gpus must be at least 1")
-    one_gpu_mode = args.sweep or args.linear or args.dit or args.encode or args.latency or args.chain
+    one_gpu_mode = args.sweep or args.linear or args.gemv or args.dit or args.encode or args.latency or args.chain
     if args.gpus > 1 and "WORLD_SIZE" not in os.environ and not one_gpu_mode:
         # no launcher: start the N ranks here (one process per GPU) and pass on their status
         sys.exit(relaunch(args.gpus, os.path.abspath(__file__), sys.argv[1:]).returncode)
@@ -1147,6 +1212,9 @@ def main():
         return
     if args.linear:
         run_linear(args)
+        return
+    if args.gemv:
+        run_gemv(args)
         return
     if args.dit:
         run_dit(args)

@@ -137,6 +137,8 @@ def lib() -> C.CDLL:
         L.ep_decode_prepare.restype = C.c_int
         L.ep_decode_tensor_prepared.argtypes = [P, P, P, P, P, P, C.c_size_t, C.c_int64, C.c_int64, C.c_int, P]
         L.ep_decode_tensor_prepared.restype = C.c_int
+        L.ep_decode_gemv.argtypes = [P, P, P, P, P, P, C.c_size_t, C.c_int64, C.c_int64, P, C.c_int, P]
+        L.ep_decode_gemv.restype = C.c_int
         L.ep_batch_create.argtypes = [C.POINTER(_BatchItem), C.c_int, C.c_int, C.POINTER(C.c_void_p)]
         L.ep_batch_create.restype = C.c_int
         L.ep_decode_batch.argtypes = [P, P]
@@ -156,7 +158,8 @@ def lib() -> C.CDLL:
 
 EXPORTED = ("ep_encode_tensor", "ep_encode_tensor_gpu", "ep_encode_tensor_gpu_device", "ep_free_device_blob",
             "ep_free_blob", "ep_decode_tensor", "ep_decode_tensor_noalloc", "ep_decode_prepare",
-            "ep_decode_tensor_prepared", "ep_batch_create", "ep_decode_batch", "ep_batch_free", "ep_batch_apportion",
+            "ep_decode_tensor_prepared", "ep_decode_gemv", "ep_batch_create", "ep_decode_batch", "ep_batch_free",
+            "ep_batch_apportion",
             "ep_decode_status", "ep_status_string")
 
 LUT_BYTES = 131104  # EP_LUT_BYTES: a prepared decode table
@@ -412,6 +415,32 @@ def decode_tensor_prepared(db: DeviceBlob, lut, out_dtype: int = BF16, out=None,
     if rc:
         raise EntroPackError(rc, "ep_decode_tensor_prepared")
     return out
+
+
+GEMV_TOKENS = (1, 2, 4, 8)
+
+
+def decode_gemv(db: DeviceBlob, x, lut=None, y=None, stream=None):
+    """ep_decode_gemv: y = x W^T with W the tensor's decoded float32 weight, computed inside the
+    decode (x: float32 CUDA tensor [ntok, cols], ntok in GEMV_TOKENS; lut: a prepare_lut table or
+    None).  Returns y, float32 [ntok, rows]."""
+    import torch
+
+    if not (isinstance(x, torch.Tensor) and x.is_cuda and x.dtype == torch.float32 and x.dim() == 2
+            and x.shape[1] == db.cols):
+        raise ValueError("x must be a float32 CUDA tensor [tokens, cols]")
+    x = x.contiguous()
+    if y is None:
+        y = torch.empty((x.shape[0], db.rows), dtype=torch.float32, device=x.device)
+    st = stream if stream is not None else torch.cuda.current_stream(db.payload.device)
+    rc = lib().ep_decode_gemv(C.c_void_p(st.cuda_stream), db.payload.data_ptr(), db.tile_index.data_ptr(),
+                              db.freq_tables.data_ptr(), db.row_scales.data_ptr(),
+                              lut.data_ptr() if lut is not None else None,
+                              lut.numel() * lut.element_size() if lut is not None else 0, db.rows, db.cols,
+                              x.data_ptr(), int(x.shape[0]), y.data_ptr())
+    if rc:
+        raise EntroPackError(rc, "ep_decode_gemv")
+    return y
 
 
 def batch_apportion(ntiles, tile_vectors, prob_bits, num_ctas: int):

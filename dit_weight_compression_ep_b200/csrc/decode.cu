@@ -1,9 +1,10 @@
 // decode.cu -- fused EntroPack weight reconstruction for B200 (sm_100a).
 //
-// EntroPack paper, Fig. 2b: symbol decoding, lattice reconstruction, row
-// rescaling and dtype conversion fused on the GPU; §3.6 "one tile to a GPU warp
-// and one state to each lane"; App. C.3 tile layout, state normalisation and the
-// decoder lookup tables ("in shared memory or packed global memory").
+// EntroPack paper, Fig. 2b: the GPU decode runs the rANS symbol decode, the
+// lattice point, the per-row scale and the output conversion in one pass; §3.6:
+// a warp per tile, a lane per interleaved state; App. C.3 tile layout, state
+// normalisation and the decoder's lookup tables (shared memory, or a packed
+// global form when they do not fit).
 //
 // One call = one cooperative launch of decode_kernel on the caller's stream:
 // one persistent CTA of 24 warps per SM (all co-resident).  Its prologue parses
@@ -107,6 +108,12 @@ constexpr unsigned kStTimeout = 8u;      // a bulk copy did not complete in time
 
 constexpr unsigned kFull = 0xFFFFFFFFu;
 constexpr uint32_t kWaitSpins = 1u << 20;  // bound on mbarrier polls
+
+// Output modes of ep_decode_gemv (not ep_dtype values): the decoded FP32 weights multiplied
+// by NT rows of activations inside the decode, NT = mode - kGemv.
+constexpr int kGemv = 100;
+template <int DT>
+__host__ __device__ constexpr int gemv_tokens() { return DT > kGemv ? DT - kGemv : 0; }
 
 // PACKED modes: b (entries hold f - 1) or 16 + b (entries hold f; one add fewer
 // per symbol, needs one more bit); COARSE otherwise.
@@ -687,6 +694,36 @@ struct TileCtx {
     uint32_t two, four, k64, mneg, df, nf0;
     int64_t cols;  // (a width that is not a multiple of 8 pads each row to whole vectors)
     uint32_t cta, G;  // this CTA's rank among the G CTAs that share the tensor: its tiles are cta + i G
+    const float* gx;  // ep_decode_gemv: activations [tokens, cols]
+    float* gy;        // ep_decode_gemv: the product [tokens, rows]
+    uint32_t rows;
+};
+
+// ep_decode_gemv: a lane's partial dot products for the row its vectors are in; they go to the
+// product by atomic adds when the lane's vectors move to the next row and at the tile's end.
+template <int NT>
+struct GemvAcc {
+    float a[NT];
+    uint32_t row;  // 0xFFFFFFFF: nothing accumulated
+    __device__ __forceinline__ void init() {
+        row = 0xFFFFFFFFu;
+#pragma unroll
+        for (int t = 0; t < NT; ++t) a[t] = 0.0f;
+    }
+    __device__ __forceinline__ void flush(const TileCtx& tc) {
+        if (row != 0xFFFFFFFFu) {
+#pragma unroll
+            for (int t = 0; t < NT; ++t) atomicAdd(tc.gy + (size_t)t * tc.rows + row, a[t]);
+        }
+        row = 0xFFFFFFFFu;
+#pragma unroll
+        for (int t = 0; t < NT; ++t) a[t] = 0.0f;
+    }
+};
+template <>
+struct GemvAcc<0> {
+    __device__ __forceinline__ void init() {}
+    __device__ __forceinline__ void flush(const TileCtx&) {}
 };
 
 // One tile's bookkeeping: record, staging state and every lane's row.
@@ -785,7 +822,8 @@ __device__ __forceinline__ void renorm(uint32_t& x, uint32_t xn, bool act, uint3
 template <int DT, bool RAGGED, typename Lut, bool FULL>
 __device__ __forceinline__ void decode_round(void* out, const float sigma, const Lut& lut, const TileCtx& tc,
                                              Tile& tl, uint32_t& pb, uint32_t r, uint32_t lt, int lane,
-                                             bool& corrupt) {
+                                             bool& corrupt, GemvAcc<gemv_tokens<DT>()>& acc, uint32_t row_now,
+                                             uint32_t q_now) {
     const uint32_t u = (r << 5) + lane;
     const bool act = FULL || u < tl.vt;
     const int64_t g = tl.v0 + u;
@@ -875,6 +913,30 @@ __device__ __forceinline__ void decode_round(void* out, const float sigma, const
                 for (int k = 0; k < 8; ++k)
                     if (k < n) put_elem<DT>(out, e0 + k, wf[k]);
             }
+        } else if constexpr (gemv_tokens<DT>() > 0) {
+            // the vector's eight FP32 weights times the tokens' eight activations of its columns
+            constexpr int NT = gemv_tokens<DT>();
+            wf[7] = sigma * (__uint_as_float(yb[7]) - 6291456.0f);
+            if (row_now != acc.row) {
+                acc.flush(tc);
+                acc.row = row_now;
+            }
+            const float4* xp = reinterpret_cast<const float4*>(tc.gx + 8 * (size_t)q_now);
+            const size_t xs4 = (size_t)tc.cols / 4;
+#pragma unroll
+            for (int t = 0; t < NT; ++t) {
+                const float4 a = __ldg(xp + t * xs4), b = __ldg(xp + t * xs4 + 1);
+                float d = acc.a[t];
+                d = fmaf(wf[0], a.x, d);
+                d = fmaf(wf[1], a.y, d);
+                d = fmaf(wf[2], a.z, d);
+                d = fmaf(wf[3], a.w, d);
+                d = fmaf(wf[4], b.x, d);
+                d = fmaf(wf[5], b.y, d);
+                d = fmaf(wf[6], b.z, d);
+                acc.a[t] = fmaf(wf[7], b.w, d);
+            }
+            (void)out;
         } else if constexpr (DT == EP_LATTICE_I32) {
             int4* o = reinterpret_cast<int4*>(out) + 2 * g;
             o[0] = make_int4((int)(yb[0] - kLat), (int)(yb[1] - kLat), (int)(yb[2] - kLat), (int)(yb[3] - kLat));
@@ -896,6 +958,8 @@ __device__ void decode_tiles(const uint16_t* tiles, const uint32_t* tix, const f
     const uint32_t G = tc.G;
     bool corrupt = false;
     bool have = tl.t != 0xFFFFFFFFu;
+    GemvAcc<gemv_tokens<DT>()> acc;
+    acc.init();
 
     for (uint32_t i = first_i; have;) {
         if (!tl.ok) {
@@ -928,6 +992,7 @@ __device__ void decode_tiles(const uint16_t* tiles, const uint32_t* tix, const f
                 uint32_t pb = rg.ring_s + 2u * ((tl.org + cur) & (kRingWords - 1));
                 const uint32_t p_start = pb;
                 const float sigma = sig_next;
+                const uint32_t row_now = tl.rowl, q_now = tl.ql;  // this round's row and column block
                 // advance every lane's row by 32 vectors and prefetch the next round's scale
                 tl.ql += 32;
                 if (tc.nq >= 32) {
@@ -941,13 +1006,15 @@ __device__ void decode_tiles(const uint16_t* tiles, const uint32_t* tix, const f
                     }
                 }
                 if (FULL) sig_next = ((r + 1) << 5) + lane < tl.vt ? __ldg(scales + tl.rowl) : 1.0f;
-                decode_round<DT, RAGGED, Lut, FULL>(out, sigma, lut, tc, tl, pb, r, lt, lane, corrupt);
+                decode_round<DT, RAGGED, Lut, FULL>(out, sigma, lut, tc, tl, pb, r, lt, lane, corrupt, acc,
+                                                    row_now, q_now);
                 cur += (pb - p_start) >> 1;
             };
             for (uint32_t r = 0; r + 1 < tl.rounds; ++r) round(std::true_type{}, r);
             round(std::false_type{}, tl.rounds - 1);
             // tile end: every lane back at 2^15 and the cursor on the next offset
             if (!__all_sync(kFull, tl.x == kStateLow) || cur != tl.off1 - tl.base) corrupt = true;
+            acc.flush(tc);
         }
         // drain this tile's copies before the ring is reused
         while (rg.waited < rg.seq && !rg.timed_out) ring_wait_one(rg);
@@ -978,6 +1045,8 @@ struct Params {
     int64_t rows, cols;
     uint32_t one;       // 1, set by the host (see TileCtx)
     uint32_t prepared;  // ws holds a table ep_decode_prepare wrote: no build, no grid barrier
+    const float* gx;    // ep_decode_gemv: activations [tokens, cols]; the product [tokens, rows]
+    float* gy;
 };
 
 // The decode loop for the stream's LUT format.  Rows padded to whole vectors (a width
@@ -1105,6 +1174,9 @@ __device__ __forceinline__ void decode_body(const Params& p, const uint32_t cta,
     tc.T = g.T;
     tc.nq = (uint32_t)((p.cols + 7) / 8);
     tc.cols = p.cols;
+    tc.gx = p.gx;
+    tc.gy = p.gy;
+    tc.rows = (uint32_t)p.rows;
     tc.b = g.b;
     tc.two = p.one << 1;
     tc.four = p.one << 2;
@@ -1308,6 +1380,7 @@ struct DevState {
     int num_sms = 0;
     bool attr_done[8] = {};
     bool prep_attr_done = false;
+    bool gemv_attr_done = false;
     uint8_t* ws = nullptr;         // the LUT workspace of this device
     cudaEvent_t ws_free = nullptr;  // recorded after every decode that used it
 };
@@ -1364,6 +1437,13 @@ cudaError_t dev_setup(int dev, int dt, DevState*& ds, bool need_ws = true) {
     return cudaSuccess;
 }
 
+// ep_decode_gemv's kernels (widths that are a multiple of 8 only)
+template <int NT>
+cudaError_t set_gemv_attr() {
+    return cudaFuncSetAttribute(decode_kernel<kGemv + NT, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                kSmemBytes);
+}
+
 template <int DT>
 cudaError_t launch_decode(const Params& prm, cudaStream_t st, int num_sms) {
     cudaLaunchConfig_t cfg = {};
@@ -1386,6 +1466,37 @@ cudaError_t launch_decode(const Params& prm, cudaStream_t st, int num_sms) {
     cfg.numAttrs = 1;
     return (prm.cols & 7) ? cudaLaunchKernelEx(&cfg, decode_kernel<DT, true>, prm)
                           : cudaLaunchKernelEx(&cfg, decode_kernel<DT, false>, prm);
+}
+
+// ep_decode_gemv: NT tokens; cooperative with the grid-built table, or an ordinary launch with
+// programmatic dependent launch when a prepared table is given (as launch_decode)
+template <int NT>
+cudaError_t launch_gemv_nt(const Params& prm, cudaStream_t st, int num_sms) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)num_sms);
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = kSmemBytes;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    if (prm.prepared) {
+        attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[0].val.programmaticStreamSerializationAllowed = 1;
+    } else {
+        attr[0].id = cudaLaunchAttributeCooperative;
+        attr[0].val.cooperative = 1;
+    }
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, decode_kernel<kGemv + NT, false>, prm);
+}
+
+cudaError_t launch_gemv(int ntok, const Params& prm, cudaStream_t st, int num_sms) {
+    switch (ntok) {
+        case 1: return launch_gemv_nt<1>(prm, st, num_sms);
+        case 2: return launch_gemv_nt<2>(prm, st, num_sms);
+        case 4: return launch_gemv_nt<4>(prm, st, num_sms);
+        default: return launch_gemv_nt<8>(prm, st, num_sms);
+    }
 }
 
 cudaError_t launch_any(ep_dtype dt, const Params& prm, cudaStream_t st, int num_sms) {
@@ -1444,6 +1555,21 @@ double batch_time(int64_t T, int64_t V, int b, int64_t c) {
 
 bool misaligned(const void* q, uintptr_t a) { return (reinterpret_cast<uintptr_t>(q) & (a - 1)) != 0; }
 
+// A launch that builds the table in the device's workspace: it waits (on the GPU) for the
+// previous such launch, whatever stream that ran on (not applied while the stream is being
+// captured), and marks the workspace busy until it ends.
+template <typename Launch>
+ep_status workspace_launch(DevState* ds, cudaStream_t st, Launch launch) {
+    std::lock_guard<std::mutex> lk(g_mu);
+    cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
+    cudaError_t e = cudaStreamIsCapturing(st, &cap);
+    const bool capturing = e == cudaSuccess && cap != cudaStreamCaptureStatusNone;
+    if (e == cudaSuccess && !capturing) e = cudaStreamWaitEvent(st, ds->ws_free, 0);
+    if (e == cudaSuccess) e = launch(st);
+    if (e == cudaSuccess && !capturing) e = cudaEventRecord(ds->ws_free, st);
+    return e == cudaSuccess ? EP_OK : EP_ECUDA;
+}
+
 // the host checks every decode entry point shares
 ep_status check_decode_args(const uint16_t* tiles, const uint32_t* tile_index, const uint8_t* freq_tables,
                             const float* row_scales, int64_t rows, int64_t cols, ep_dtype out_dtype, void* out) {
@@ -1474,20 +1600,9 @@ ep_status ep_decode_tensor(void* stream, const uint16_t* tiles, const uint32_t* 
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return EP_ECUDA;
     DevState* ds = nullptr;
     if (dev_setup(dev, (int)out_dtype, ds) != cudaSuccess) return EP_ECUDA;
-    cudaStream_t st = static_cast<cudaStream_t>(stream);
-    // decodes on the device share its workspace: a decode waits (on the GPU)
-    // for the previous one, whatever stream that ran on
-    std::lock_guard<std::mutex> lk(g_mu);
-    cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
-    cudaError_t e = cudaStreamIsCapturing(st, &cap);
-    const bool capturing = e == cudaSuccess && cap != cudaStreamCaptureStatusNone;
-    if (e == cudaSuccess && !capturing) e = cudaStreamWaitEvent(st, ds->ws_free, 0);
-    if (e == cudaSuccess) {
-        const Params prm{tiles, tile_index, freq_tables, row_scales, out, ds->ws, rows, cols, 1u, 0u};
-        e = launch_any(out_dtype, prm, st, ds->num_sms);
-    }
-    if (e == cudaSuccess && !capturing) e = cudaEventRecord(ds->ws_free, st);
-    return e == cudaSuccess ? EP_OK : EP_ECUDA;
+    const Params prm{tiles, tile_index, freq_tables, row_scales, out, ds->ws, rows, cols, 1u, 0u};
+    return workspace_launch(ds, static_cast<cudaStream_t>(stream),
+                            [&](cudaStream_t st) { return launch_any(out_dtype, prm, st, ds->num_sms); });
 }
 
 ep_status ep_decode_prepare(void* stream, const uint8_t* freq_tables, int64_t rows, int64_t cols, void* lut,
@@ -1535,6 +1650,41 @@ ep_status ep_decode_tensor_prepared(void* stream, const uint16_t* tiles, const u
                      const_cast<uint8_t*>(static_cast<const uint8_t*>(lut)), rows, cols, 1u, 1u};
     return launch_any(out_dtype, prm, static_cast<cudaStream_t>(stream), ds->num_sms) == cudaSuccess ? EP_OK
                                                                                                      : EP_ECUDA;
+}
+
+ep_status ep_decode_gemv(void* stream, const uint16_t* tiles, const uint32_t* tile_index, const uint8_t* freq_tables,
+                         const float* row_scales, const void* lut, size_t lut_bytes, int64_t rows, int64_t cols,
+                         const float* x, int ntok, float* y) {
+    using namespace ep;
+    const ep_status as = check_decode_args(tiles, tile_index, freq_tables, row_scales, rows, cols, EP_FP32, y);
+    if (as != EP_OK) return as;
+    if (!x || misaligned(x, 16)) return EP_EINVAL;
+    if (ntok != 1 && ntok != 2 && ntok != 4 && ntok != 8) return EP_EUNSUPPORTED;
+    if (cols & 7) return EP_EUNSUPPORTED;
+    if (lut && (lut_bytes < (size_t)EP_LUT_BYTES || misaligned(lut, 16))) return EP_EINVAL;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return EP_ECUDA;
+    DevState* ds = nullptr;
+    if (dev_setup(dev, EP_FP32, ds) != cudaSuccess) return EP_ECUDA;
+    {
+        std::lock_guard<std::mutex> lk(g_mu);
+        if (!ds->gemv_attr_done) {
+            if (set_gemv_attr<1>() != cudaSuccess || set_gemv_attr<2>() != cudaSuccess ||
+                set_gemv_attr<4>() != cudaSuccess || set_gemv_attr<8>() != cudaSuccess)
+                return EP_ECUDA;
+            ds->gemv_attr_done = true;
+        }
+    }
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    // the product accumulates by atomic adds: it starts at zero
+    if (cudaMemsetAsync(y, 0, (size_t)ntok * (size_t)rows * sizeof(float), st) != cudaSuccess) return EP_ECUDA;
+    if (lut) {
+        const Params prm{tiles, tile_index, freq_tables, row_scales, y,
+                         const_cast<uint8_t*>(static_cast<const uint8_t*>(lut)), rows, cols, 1u, 1u, x, y};
+        return launch_gemv(ntok, prm, st, ds->num_sms) == cudaSuccess ? EP_OK : EP_ECUDA;
+    }
+    const Params prm{tiles, tile_index, freq_tables, row_scales, y, ds->ws, rows, cols, 1u, 0u, x, y};
+    return workspace_launch(ds, st, [&](cudaStream_t s2) { return launch_gemv(ntok, prm, s2, ds->num_sms); });
 }
 
 ep_status ep_batch_apportion(int n, const int64_t* ntiles, const int64_t* tile_vectors, const int* prob_bits,

@@ -8,8 +8,8 @@
  * This library offers:
  *   ep_encode_tensor  -- the CPU packer (§3.1 pipeline, §3.4 scale search,
  *                        §3.5 refit, §3.6 tiles; App. C.1, C.3), threaded;
- *   ep_decode_tensor  -- the fused GPU reconstruction (Fig. 2b; §3.6 "one tile
- *                        to a GPU warp and one state to each lane"; App. C.3),
+ *   ep_decode_tensor  -- the fused GPU reconstruction (Fig. 2b; §3.6: a warp
+ *                        per tile, a lane per interleaved state; App. C.3),
  *                        stream-ordered, one kernel launch per call.
  *
  * Stored representation (all little-endian; the packer writes it, the decoder
@@ -297,6 +297,31 @@ ep_status ep_decode_tensor_prepared(void* stream, const uint16_t* tiles, const u
                                     const uint8_t* freq_tables, const float* row_scales, const void* lut,
                                     size_t lut_bytes, int64_t rows, int64_t cols, ep_dtype out_dtype,
                                     void* out);
+
+/*
+ * ep_decode_gemv -- a linear layer on a few tokens with the weight decoded inside the product
+ * (the on-demand reconstruction of paper §4.3 and Fig. 5, for the decode-bound case of
+ * small token counts, e.g. the pages' 8-token draft-verify decode): y = x W^T, where
+ * W [rows, cols] is the tensor's decoded FP32 weight (sigma_r * y_rc, the values
+ * ep_decode_tensor writes for EP_FP32).  Every lane multiplies the eight weights it has
+ * just reconstructed by the tokens' eight activations of those columns and accumulates per
+ * row; the weight is never written to memory.
+ *   tiles .. cols   as ep_decode_tensor (cols must be a multiple of 8: else EP_EUNSUPPORTED).
+ *   lut, lut_bytes  a table ep_decode_prepare built for this tensor (then the call uses no
+ *                   workspace and launches as ep_decode_tensor_prepared), or NULL (the table
+ *                   is built per call in the workspace, as ep_decode_tensor).
+ *   x               device, float32 [ntok, cols] row-major, 16-byte aligned; read only.
+ *   ntok            1, 2, 4 or 8 (else EP_EUNSUPPORTED).
+ *   y               device, float32 [ntok, rows] row-major, 16-byte aligned; overwritten: the
+ *                   call zeroes it on the stream, then adds the partial sums of each row by
+ *                   atomic adds, so the order of the float32 additions is unspecified (the
+ *                   result lies within the float32 dot-product bound of the exact product).
+ * Asynchronous on `stream`; argument errors as ep_decode_tensor; stream errors raise the
+ * status word that ep_decode_status reads.
+ */
+ep_status ep_decode_gemv(void* stream, const uint16_t* tiles, const uint32_t* tile_index, const uint8_t* freq_tables,
+                         const float* row_scales, const void* lut, size_t lut_bytes, int64_t rows, int64_t cols,
+                         const float* x, int ntok, float* y);
 
 /*
  * Batched decode: several tensors in one launch.  A layer-by-layer decode leaves

@@ -588,8 +588,8 @@ static void write_tables(epo_blob* bl, const table_t* tabs) {
 
 /*
  * Entropy-code given fields (rows x ceil(cols/8) vectors, 9 fields each) with given
- * row scales: tables from the full-tensor counts (§3.6 "We recount the final
- * full-tensor fields"), tiles of V vectors, interleaved rANS per tile.
+ * row scales: tables from the counts over the whole tensor's final fields
+ * (§3.6), tiles of V vectors, interleaved rANS per tile.
  * Returns 0, or a negative code when an alphabet exceeds 2^b.
  */
 static int code_fields(epo_blob* bl, int pooled) {
@@ -669,10 +669,10 @@ float epo_refit_row(const float* w, const double* y, int64_t cols) {
 }
 
 /*
- * A10 Per-row rate-distortion refinement ([paper] §3.5 "RDO compares several
- * quantization resolutions per row and allocates them under a common storage
- * budget"; App. C.2; Figs. 3-4).  Off unless asked for ([paper] §4.1: "RDO is
- * disabled except in its dedicated ablations").
+ * A10 Per-row rate-distortion refinement ([paper] §3.5: each row picks one of
+ * several quantisation steps, all rows sharing one storage budget; App. C.2;
+ * Figs. 3-4).  Off unless asked for ([paper] §4.1 runs it in its own ablations
+ * only).
  *
  * Candidate ratios (§3.5): K ratios in [0.70, 1.45], starting from 1; each
  * further ratio bisects, in log scale, the widest interval between neighbouring
@@ -1046,8 +1046,8 @@ int8_t epo_f32_to_int8(float x) {
 }
 
 /* UINT8 container with its offset ([paper] App. B, Table 6: integer inputs are
- * scaled per tensor before casting, "with an offset for unsigned values"; the
- * errors are taken "with the UINT8 offset removed").  Reading: the codec codes
+ * scaled per tensor before the cast, the unsigned container carrying an offset,
+ * which the error figures subtract again).  Reading: the codec codes
  * the container's codes minus 128, and the decoder adds the 128 back: the
  * nearest integer (ties to even), clamped to [-128, 127], plus 128. */
 uint8_t epo_f32_to_uint8(float x) {

@@ -186,8 +186,8 @@ def _rel_l2(ob, W):
 
 
 def test_rdo_candidate_ratios_are_nested_log_bisections():
-    # §3.5: ratios in [0.70, 1.45], starting from 1, each bisecting the widest remaining interval
-    # in log scale (the two halves of [1, 1.45] tie; the lower one goes first)
+    # §3.5: ratios in [0.70, 1.45], the first 1, each next one the log-scale midpoint of the
+    # largest gap left (the two halves of [1, 1.45] tie; the lower one goes first)
     want = [1.0, 1.45 ** 0.5, 0.70 ** 0.5, 1.45 ** 0.25, 1.45 ** 0.75]
     np.testing.assert_allclose(oracle.rdo_ratios(5), want, rtol=1e-15)
     r20 = oracle.rdo_ratios(20)

@@ -24,7 +24,7 @@ def test_table5_tile_metadata_closed_form():
         assert oracle.tile_vectors(int(S)) == V
         assert -(-nvec // int(V)) == T
         assert oracle.tile_metadata_bytes(int(T)) == meta
-        # App. C.1: b starts at 11 for targets up to 7 bpp and at 12 above
+        # App. C.1: the starting b is 11 at or below 7 bpp, else 12
         assert (11 if tgt <= 7 else 12) == b
 
 
