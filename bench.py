@@ -1063,12 +1063,11 @@ def run_gemv(args):
     stream_bytes = blob.stored_device_bytes()
     out = []
     for ntok in ep.GEMV_TOKENS:
-        x = torch.randn(ntok, cols, device=dev) * 0.5
-        xb = x.to(torch.bfloat16)
+        xb = (torch.randn(ntok, cols, device=dev) * 0.5).to(torch.bfloat16)
         y = torch.empty(ntok, rows, device=dev)
         t_res = tmin(lambda: torch.matmul(xb, Wb.t()))
-        t_fused = tmin(lambda: ep.decode_gemv(db, x, lut=lut, y=y))
-        t_fused_call = tmin(lambda: ep.decode_gemv(db, x, y=y))
+        t_fused = tmin(lambda: ep.decode_gemv(db, xb, lut=lut, y=y))
+        t_fused_call = tmin(lambda: ep.decode_gemv(db, xb, y=y))
         t_dec = tmin(lambda: ep.decode_tensor_prepared(db, lut, ep.BF16, out=Wd))
         t_both = tmin(lambda: torch.matmul(xb, ep.decode_tensor_prepared(db, lut, ep.BF16, out=Wd).t()))
         if ep.decode_status() != 0:
@@ -1076,7 +1075,7 @@ def run_gemv(args):
         r = {"tokens": ntok, "gemv_resident_bf16_us": round(t_res, 2), "fused_prepared_us": round(t_fused, 2),
              "fused_per_call_us": round(t_fused_call, 2), "decode_prepared_us": round(t_dec, 2),
              "decode_then_gemm_us": round(t_both, 2), "fused_vs_decode_then_gemm": round(t_both / t_fused, 3),
-             "fused_hbm_gbs": round((stream_bytes + x.nbytes + y.nbytes) / (t_fused * 1e-6) / 1e9, 1)}
+             "fused_hbm_gbs": round((stream_bytes + xb.nbytes + y.nbytes) / (t_fused * 1e-6) / 1e9, 1)}
         out.append(r)
         print(json.dumps(r), flush=True)
     print("\n| tokens | GEMV, BF16 weight resident (µs) | fused decode-GEMV, prepared (µs) | fused, per call (µs) | "

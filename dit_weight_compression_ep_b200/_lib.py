@@ -422,13 +422,13 @@ GEMV_TOKENS = (1, 2, 4, 8)
 
 def decode_gemv(db: DeviceBlob, x, lut=None, y=None, stream=None):
     """ep_decode_gemv: y = x W^T with W the tensor's decoded float32 weight, computed inside the
-    decode (x: float32 CUDA tensor [ntok, cols], ntok in GEMV_TOKENS; lut: a prepare_lut table or
+    decode (x: bfloat16 CUDA tensor [ntok, cols], ntok in GEMV_TOKENS; lut: a prepare_lut table or
     None).  Returns y, float32 [ntok, rows]."""
     import torch
 
-    if not (isinstance(x, torch.Tensor) and x.is_cuda and x.dtype == torch.float32 and x.dim() == 2
+    if not (isinstance(x, torch.Tensor) and x.is_cuda and x.dtype == torch.bfloat16 and x.dim() == 2
             and x.shape[1] == db.cols):
-        raise ValueError("x must be a float32 CUDA tensor [tokens, cols]")
+        raise ValueError("x must be a bfloat16 CUDA tensor [tokens, cols]")
     x = x.contiguous()
     if y is None:
         y = torch.empty((x.shape[0], db.rows), dtype=torch.float32, device=x.device)

@@ -694,17 +694,51 @@ struct TileCtx {
     uint32_t two, four, k64, mneg, df, nf0;
     int64_t cols;  // (a width that is not a multiple of 8 pads each row to whole vectors)
     uint32_t cta, G;  // this CTA's rank among the G CTAs that share the tensor: its tiles are cta + i G
-    const float* gx;  // ep_decode_gemv: activations [tokens, cols]
-    float* gy;        // ep_decode_gemv: the product [tokens, rows]
+    const uint16_t* gx;  // ep_decode_gemv: BF16 activations [tokens, cols]
+    float* gy;           // ep_decode_gemv: the product [tokens, rows]
     uint32_t rows;
 };
 
 // ep_decode_gemv: a lane's partial dot products for the row its vectors are in; they go to the
 // product by atomic adds when the lane's vectors move to the next row and at the tile's end.
+// The eight BF16 activations of a vector's columns (one 16-byte load a token) come in a round
+// ahead for up to 4 tokens, so that their latency hides behind the round's nine symbol steps;
+// for 8 tokens they are loaded where they are used (held a round ahead, they would not fit in
+// the registers).
 template <int NT>
 struct GemvAcc {
+    static constexpr bool kAhead = NT <= 4;
     float a[NT];
+    uint4 xv[kAhead ? NT : 1];
     uint32_t row;  // 0xFFFFFFFF: nothing accumulated
+    __device__ __forceinline__ static uint4 xload(const TileCtx& tc, uint32_t q, int t) {
+        return __ldg(reinterpret_cast<const uint4*>(tc.gx + (size_t)t * (size_t)tc.cols) + q);
+    }
+    // the activations of column block q (the lane's vector in the next round)
+    __device__ __forceinline__ void ahead(const TileCtx& tc, uint32_t q) {
+        if constexpr (kAhead) {
+#pragma unroll
+            for (int t = 0; t < NT; ++t) xv[t] = xload(tc, q, t);
+        }
+    }
+    // a[t] += <w, x_t> over the vector's eight columns (block q); BF16 widens to FP32 exactly
+    __device__ __forceinline__ void madd(const TileCtx& tc, uint32_t q, const float* w) {
+#pragma unroll
+        for (int t = 0; t < NT; ++t) {
+            uint4 p;
+            if constexpr (kAhead) p = xv[t];
+            else p = xload(tc, q, t);
+            float d = a[t];
+            d = fmaf(w[0], __uint_as_float(p.x << 16), d);
+            d = fmaf(w[1], __uint_as_float(p.x & 0xFFFF0000u), d);
+            d = fmaf(w[2], __uint_as_float(p.y << 16), d);
+            d = fmaf(w[3], __uint_as_float(p.y & 0xFFFF0000u), d);
+            d = fmaf(w[4], __uint_as_float(p.z << 16), d);
+            d = fmaf(w[5], __uint_as_float(p.z & 0xFFFF0000u), d);
+            d = fmaf(w[6], __uint_as_float(p.w << 16), d);
+            a[t] = fmaf(w[7], __uint_as_float(p.w & 0xFFFF0000u), d);
+        }
+    }
     __device__ __forceinline__ void init() {
         row = 0xFFFFFFFFu;
 #pragma unroll
@@ -722,6 +756,7 @@ struct GemvAcc {
 };
 template <>
 struct GemvAcc<0> {
+    __device__ __forceinline__ void ahead(const TileCtx&, uint32_t) {}
     __device__ __forceinline__ void init() {}
     __device__ __forceinline__ void flush(const TileCtx&) {}
 };
@@ -915,27 +950,12 @@ __device__ __forceinline__ void decode_round(void* out, const float sigma, const
             }
         } else if constexpr (gemv_tokens<DT>() > 0) {
             // the vector's eight FP32 weights times the tokens' eight activations of its columns
-            constexpr int NT = gemv_tokens<DT>();
             wf[7] = sigma * (__uint_as_float(yb[7]) - 6291456.0f);
             if (row_now != acc.row) {
                 acc.flush(tc);
                 acc.row = row_now;
             }
-            const float4* xp = reinterpret_cast<const float4*>(tc.gx + 8 * (size_t)q_now);
-            const size_t xs4 = (size_t)tc.cols / 4;
-#pragma unroll
-            for (int t = 0; t < NT; ++t) {
-                const float4 a = __ldg(xp + t * xs4), b = __ldg(xp + t * xs4 + 1);
-                float d = acc.a[t];
-                d = fmaf(wf[0], a.x, d);
-                d = fmaf(wf[1], a.y, d);
-                d = fmaf(wf[2], a.z, d);
-                d = fmaf(wf[3], a.w, d);
-                d = fmaf(wf[4], b.x, d);
-                d = fmaf(wf[5], b.y, d);
-                d = fmaf(wf[6], b.z, d);
-                acc.a[t] = fmaf(wf[7], b.w, d);
-            }
+            acc.madd(tc, q_now, wf);
             (void)out;
         } else if constexpr (DT == EP_LATTICE_I32) {
             int4* o = reinterpret_cast<int4*>(out) + 2 * g;
@@ -972,6 +992,7 @@ __device__ void decode_tiles(const uint16_t* tiles, const uint32_t* tix, const f
             uint32_t thr = 0;
             // every lane's row for round 0, its row scale, and the row of round 1
             float sig_next = tl.vt > (uint32_t)lane ? __ldg(scales + tl.rowl) : 1.0f;
+            acc.ahead(tc, tl.ql);
             auto round = [&](auto full, uint32_t r) {
                 constexpr bool FULL = decltype(full)::value;
                 if (cur >= thr) {
@@ -1008,6 +1029,7 @@ __device__ void decode_tiles(const uint16_t* tiles, const uint32_t* tix, const f
                 if (FULL) sig_next = ((r + 1) << 5) + lane < tl.vt ? __ldg(scales + tl.rowl) : 1.0f;
                 decode_round<DT, RAGGED, Lut, FULL>(out, sigma, lut, tc, tl, pb, r, lt, lane, corrupt, acc,
                                                     row_now, q_now);
+                if (FULL) acc.ahead(tc, tl.ql);  // the next round's activations
                 cur += (pb - p_start) >> 1;
             };
             for (uint32_t r = 0; r + 1 < tl.rounds; ++r) round(std::true_type{}, r);
@@ -1045,7 +1067,7 @@ struct Params {
     int64_t rows, cols;
     uint32_t one;       // 1, set by the host (see TileCtx)
     uint32_t prepared;  // ws holds a table ep_decode_prepare wrote: no build, no grid barrier
-    const float* gx;    // ep_decode_gemv: activations [tokens, cols]; the product [tokens, rows]
+    const uint16_t* gx;  // ep_decode_gemv: BF16 activations [tokens, cols]; the product [tokens, rows]
     float* gy;
 };
 
@@ -1654,7 +1676,7 @@ ep_status ep_decode_tensor_prepared(void* stream, const uint16_t* tiles, const u
 
 ep_status ep_decode_gemv(void* stream, const uint16_t* tiles, const uint32_t* tile_index, const uint8_t* freq_tables,
                          const float* row_scales, const void* lut, size_t lut_bytes, int64_t rows, int64_t cols,
-                         const float* x, int ntok, float* y) {
+                         const void* x, int ntok, float* y) {
     using namespace ep;
     const ep_status as = check_decode_args(tiles, tile_index, freq_tables, row_scales, rows, cols, EP_FP32, y);
     if (as != EP_OK) return as;
@@ -1680,10 +1702,12 @@ ep_status ep_decode_gemv(void* stream, const uint16_t* tiles, const uint32_t* ti
     if (cudaMemsetAsync(y, 0, (size_t)ntok * (size_t)rows * sizeof(float), st) != cudaSuccess) return EP_ECUDA;
     if (lut) {
         const Params prm{tiles, tile_index, freq_tables, row_scales, y,
-                         const_cast<uint8_t*>(static_cast<const uint8_t*>(lut)), rows, cols, 1u, 1u, x, y};
+                         const_cast<uint8_t*>(static_cast<const uint8_t*>(lut)), rows, cols, 1u, 1u,
+                         static_cast<const uint16_t*>(x), y};
         return launch_gemv(ntok, prm, st, ds->num_sms) == cudaSuccess ? EP_OK : EP_ECUDA;
     }
-    const Params prm{tiles, tile_index, freq_tables, row_scales, y, ds->ws, rows, cols, 1u, 0u, x, y};
+    const Params prm{tiles, tile_index, freq_tables, row_scales, y, ds->ws, rows, cols, 1u, 0u,
+                     static_cast<const uint16_t*>(x), y};
     return workspace_launch(ds, st, [&](cudaStream_t s2) { return launch_gemv(ntok, prm, s2, ds->num_sms); });
 }
 

@@ -301,16 +301,16 @@ ep_status ep_decode_tensor_prepared(void* stream, const uint16_t* tiles, const u
 /*
  * ep_decode_gemv -- a linear layer on a few tokens with the weight decoded inside the product
  * (the on-demand reconstruction of paper §4.3 and Fig. 5, for the decode-bound case of
- * small token counts, e.g. the pages' 8-token draft-verify decode): y = x W^T, where
- * W [rows, cols] is the tensor's decoded FP32 weight (sigma_r * y_rc, the values
- * ep_decode_tensor writes for EP_FP32).  Every lane multiplies the eight weights it has
- * just reconstructed by the tokens' eight activations of those columns and accumulates per
- * row; the weight is never written to memory.
+ * small token counts): y = x W^T, where W [rows, cols] is the tensor's decoded FP32 weight
+ * (sigma_r * y_rc, the values ep_decode_tensor writes for EP_FP32) and x holds BF16
+ * activations, widened exactly to FP32.  Every lane multiplies the eight weights it has just
+ * reconstructed by the tokens' eight activations of those columns with FP32 multiply-adds
+ * and accumulates per row; the weight is never written to memory.
  *   tiles .. cols   as ep_decode_tensor (cols must be a multiple of 8: else EP_EUNSUPPORTED).
  *   lut, lut_bytes  a table ep_decode_prepare built for this tensor (then the call uses no
  *                   workspace and launches as ep_decode_tensor_prepared), or NULL (the table
  *                   is built per call in the workspace, as ep_decode_tensor).
- *   x               device, float32 [ntok, cols] row-major, 16-byte aligned; read only.
+ *   x               device, BF16 bits [ntok, cols] row-major, 16-byte aligned; read only.
  *   ntok            1, 2, 4 or 8 (else EP_EUNSUPPORTED).
  *   y               device, float32 [ntok, rows] row-major, 16-byte aligned; overwritten: the
  *                   call zeroes it on the stream, then adds the partial sums of each row by
@@ -321,7 +321,7 @@ ep_status ep_decode_tensor_prepared(void* stream, const uint16_t* tiles, const u
  */
 ep_status ep_decode_gemv(void* stream, const uint16_t* tiles, const uint32_t* tile_index, const uint8_t* freq_tables,
                          const float* row_scales, const void* lut, size_t lut_bytes, int64_t rows, int64_t cols,
-                         const float* x, int ntok, float* y);
+                         const void* x, int ntok, float* y);
 
 /*
  * Batched decode: several tensors in one launch.  A layer-by-layer decode leaves

@@ -2,9 +2,9 @@
 (EntroPack paper §4.3 and Fig. 5: the weight is reconstructed on demand for the matmul).
 
 The reference is the oracle's float64 product of its own float32 decode of the weight
-(`oracle.linear`), and the tolerance is the oracle's float32-accumulation bound
-(`oracle.linear_tolerance`, gamma_K sum|x w|: any order of float32 additions, the atomic adds
-included) with no output rounding beyond float32.  Cases: every token count (1, 2, 4, 8), the
+(`oracle.linear`) with the BF16 activations widened exactly, and the tolerance is the oracle's
+float32-accumulation bound (`oracle.linear_tolerance`, gamma_K sum|x w|: any order of float32
+additions, the atomic adds included) with no output rounding beyond float32.  Cases: every token count (1, 2, 4, 8), the
 packed (b = 11), two-level (b = 12) and bucketed (b = 13) tables, widths whose rows do not end
 on a round of 32 vectors, per-call and prepared tables, several tiles per row and several rows
 per tile, and the 3840x10240 headline on sampled rows.
@@ -35,12 +35,12 @@ def _x(ntok, cols, seed):
     import torch
 
     g = torch.Generator(device="cpu").manual_seed(seed)
-    return (torch.randn(ntok, cols, generator=g) * 0.5).cuda()
+    return (torch.randn(ntok, cols, generator=g) * 0.5).to(torch.bfloat16).cuda()
 
 
 def _check(blob, x, y, rows_sel=None):
     """y against the oracle's product on the whole matrix, or on the rows rows_sel."""
-    xs = x.cpu().numpy().astype(np.float64)
+    xs = x.cpu().float().numpy().astype(np.float64)  # BF16 widens to float64 exactly
     got = y.cpu().numpy().astype(np.float64)
     if rows_sel is None:
         W = oracle_decode(blob, ep.FP32).reshape(blob.rows, blob.cols).astype(np.float64)
@@ -108,6 +108,27 @@ def test_refusals_on_the_host():
         ep.decode_gemv(db, _x(3, blob.cols, 1))  # 3 tokens
     odd = ep.encode_tensor(np.ones((8, 12), np.float32) * 0.01, 4.0)
     with pytest.raises(ep.EntroPackError):
-        ep.decode_gemv(ep.DeviceBlob(odd), torch.zeros((1, 12), device="cuda"))  # width not a multiple of 8
+        ep.decode_gemv(ep.DeviceBlob(odd), torch.zeros((1, 12), dtype=torch.bfloat16, device="cuda"))  # width % 8
     with pytest.raises(ValueError):
-        ep.decode_gemv(db, torch.zeros((1, blob.cols), dtype=torch.bfloat16, device="cuda"))
+        ep.decode_gemv(db, torch.zeros((1, blob.cols), dtype=torch.float32, device="cuda"))
+
+
+def test_compressed_linear_matvec_with_bias():
+    import torch
+
+    blob = ep.encode_tensor(synth.generate(synth.small_fp32()), 4.0)
+    db = ep.DeviceBlob(blob)
+    bias = torch.linspace(-1, 1, blob.rows, device="cuda")
+    lin = ep.CompressedLinear(db, "bf16", bias=bias)
+    x = _x(2, blob.cols, 11)
+    y = lin.matvec(x)
+    assert ep.decode_status() == 0
+    W = oracle_decode(blob, ep.FP32).reshape(blob.rows, blob.cols).astype(np.float64)
+    xs = x.cpu().float().numpy().astype(np.float64)
+    b = bias.cpu().numpy().astype(np.float64)
+    want = oracle.linear(W, xs) + b
+    # the product's bound, plus one float32 rounding of the bias add
+    tol = oracle.linear_tolerance(W, xs, 0.0) + np.abs(want) * 2.0 ** -23
+    assert np.all(np.abs(y.cpu().numpy().astype(np.float64) - want) <= tol)
+    with pytest.raises(ValueError):
+        lin.matvec(_x(3, blob.cols, 1))
