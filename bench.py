@@ -4,6 +4,7 @@
     python bench.py --sweep      (every workload, one GPU: a table, not the bench line)
     python bench.py --linear     (decode-then-GEMM against a resident weight, one GPU)
     python bench.py --gemv       (the fused decode-GEMV on 1 to 8 tokens, one GPU)
+    python bench.py --split      (the decode on part of the GPU beside the GEMM, one GPU)
 
 One step = one ep_decode_tensor call: the whole hot path (tile setup, table
 staging, payload staging, rANS decode, lattice reconstruction, row rescale,
@@ -1086,6 +1087,97 @@ def run_gemv(args):
               f"{r['decode_prepared_us']} | {r['decode_then_gemm_us']} | {r['fused_vs_decode_then_gemm']} |")
 
 
+def run_split(args):
+    """The decode on part of the GPU beside the GEMM: 16 consecutive 3840x10240 layers at 4 bpp,
+    the next layer's weight decoded on s SMs (a one-tensor batch from ep_batch_create_on) on a
+    second stream while the current layer's bf16 GEMM runs on the main stream, two output buffers.
+    Against decode then GEMM on one stream, for 256, 1,024 and 4,096 tokens.  Each figure is the
+    minimum of 5 passes over the 16 layers, each pass after a 256 MiB L2 flush, in µs per layer."""
+    import torch
+
+    import dit_weight_compression_ep_b200 as ep
+    from dit_weight_compression_ep_b200 import build, synth
+
+    build.build()
+    dev = torch.device("cuda")
+    st = torch.cuda.current_stream()
+    s_dec = torch.cuda.Stream()
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    nl = 16
+
+    def per_layer(fn, reps=5):
+        fn()
+        torch.cuda.synchronize()
+        ts = []
+        for _ in range(reps):
+            flush.zero_()
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record()
+            fn()
+            b.record()
+            torch.cuda.synchronize()
+            ts.append(a.elapsed_time(b))
+        return round(min(ts) * 1e3 / nl, 1)
+
+    W = synth.generate(synth.headline())
+    rows, cols = W.shape
+    db = ep.DeviceBlob(ep.encode_tensor(W, TARGET))
+    lut = ep.prepare_lut(db)
+    bufs = [torch.empty(rows, cols, dtype=torch.bfloat16, device=dev) for _ in range(2)]
+    nsm = torch.cuda.get_device_properties(dev).multi_processor_count
+    splits = [s for s in (32, 64, 100, nsm) if s <= nsm]
+    out = []
+    for tokens in (256, 1024, 4096):
+        X = torch.randn(tokens, cols, dtype=torch.bfloat16, device=dev)
+
+        def seq():
+            for i in range(nl):
+                ep.decode_tensor_prepared(db, lut, ep.BF16, out=bufs[i % 2], stream=st)
+                torch.matmul(X, bufs[i % 2].t())
+
+        def gemm():
+            for i in range(nl):
+                torch.matmul(X, bufs[i % 2].t())
+
+        r = {"tokens": tokens, "decode_then_gemm_us": per_layer(seq), "gemm_us": per_layer(gemm)}
+        for s in splits:
+            bs = [ep.DecodeBatch([(db, lut, bufs[k])], ep.BF16, num_ctas=s) for k in range(2)]
+
+            def dec():
+                for i in range(nl):
+                    bs[i % 2].run(stream=st)
+
+            def pipe():
+                ev_dec = [torch.cuda.Event() for _ in range(nl)]
+                ev_mm = [torch.cuda.Event() for _ in range(nl)]
+                s_dec.wait_stream(st)
+                for i in range(nl + 1):
+                    if i < nl:
+                        if i >= 2:
+                            s_dec.wait_event(ev_mm[i - 2])  # the GEMM that last read this buffer
+                        bs[i % 2].run(stream=s_dec)
+                        ev_dec[i].record(s_dec)
+                    j = i - 1
+                    if j >= 0:
+                        st.wait_event(ev_dec[j])
+                        torch.matmul(X, bufs[j % 2].t())
+                        ev_mm[j].record(st)
+                st.wait_stream(s_dec)
+
+            r[f"decode_on_{s}_us"] = per_layer(dec)
+            r[f"pipelined_{s}_us"] = per_layer(pipe)
+        if ep.decode_status() != 0:
+            raise RuntimeError("decode reported a corrupt stream")
+        out.append(r)
+        print(json.dumps(r), flush=True)
+    head = " | ".join([f"decode on {s}" for s in splits] + [f"pipelined, s = {s}" for s in splits])
+    print(f"\n| tokens | decode then GEMM, one stream | GEMM alone | {head} |")
+    print("|---" * (3 + 2 * len(splits)) + "|")
+    for r in out:
+        cells = [r[f"decode_on_{s}_us"] for s in splits] + [r[f"pipelined_{s}_us"] for s in splits]
+        print(f"| {r['tokens']} | {r['decode_then_gemm_us']} | {r['gemm_us']} | " + " | ".join(map(str, cells)) + " |")
+
+
 PROBE_CHAINS = [
     ("imad", "mad.lo.u32 (state update, addresses)"),
     ("lds32+imad", "32-bit shared load (lookup-table entry) + its address multiply-add"),
@@ -1184,6 +1276,7 @@ def main():
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--sweep", action="store_true", help="every workload's decode throughput (one GPU)")
     ap.add_argument("--linear", action="store_true", help="decode-then-GEMM against a resident weight (one GPU)")
+    ap.add_argument("--split", action="store_true", help="the decode on part of the GPU beside the GEMM (one GPU)")
     ap.add_argument("--gemv", action="store_true", help="the fused decode-GEMV on 1 to 8 tokens (one GPU)")
     ap.add_argument("--dit", action="store_true", help="the whole DiT stack: per layer, prepared, block batches")
     ap.add_argument("--encode", action="store_true", help="conversion speed: CPU packer and GPU encoder")
@@ -1196,7 +1289,7 @@ def main():
         ap.error("--warmup must be at least 3")
     if args.gpus < 1:
         ap.error("--gpus must be at least 1")
-    one_gpu_mode = args.sweep or args.linear or args.gemv or args.dit or args.encode or args.latency or args.chain
+    one_gpu_mode = args.sweep or args.linear or args.split or args.gemv or args.dit or args.encode or args.latency or args.chain
     if args.gpus > 1 and "WORLD_SIZE" not in os.environ and not one_gpu_mode:
         # no launcher: start the N ranks here (one process per GPU) and pass on their status
         sys.exit(relaunch(args.gpus, os.path.abspath(__file__), sys.argv[1:]).returncode)
@@ -1211,6 +1304,9 @@ def main():
         return
     if args.linear:
         run_linear(args)
+        return
+    if args.split:
+        run_split(args)
         return
     if args.gemv:
         run_gemv(args)

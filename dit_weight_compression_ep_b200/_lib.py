@@ -141,6 +141,8 @@ def lib() -> C.CDLL:
         L.ep_decode_gemv.restype = C.c_int
         L.ep_batch_create.argtypes = [C.POINTER(_BatchItem), C.c_int, C.c_int, C.POINTER(C.c_void_p)]
         L.ep_batch_create.restype = C.c_int
+        L.ep_batch_create_on.argtypes = [C.POINTER(_BatchItem), C.c_int, C.c_int, C.c_int, C.POINTER(C.c_void_p)]
+        L.ep_batch_create_on.restype = C.c_int
         L.ep_decode_batch.argtypes = [P, P]
         L.ep_decode_batch.restype = C.c_int
         L.ep_batch_free.argtypes = [P]
@@ -158,9 +160,8 @@ def lib() -> C.CDLL:
 
 EXPORTED = ("ep_encode_tensor", "ep_encode_tensor_gpu", "ep_encode_tensor_gpu_device", "ep_free_device_blob",
             "ep_free_blob", "ep_decode_tensor", "ep_decode_tensor_noalloc", "ep_decode_prepare",
-            "ep_decode_tensor_prepared", "ep_decode_gemv", "ep_batch_create", "ep_decode_batch", "ep_batch_free",
-            "ep_batch_apportion",
-            "ep_decode_status", "ep_status_string")
+            "ep_decode_tensor_prepared", "ep_decode_gemv", "ep_batch_create", "ep_batch_create_on",
+            "ep_decode_batch", "ep_batch_free", "ep_batch_apportion", "ep_decode_status", "ep_status_string")
 
 LUT_BYTES = 131104  # EP_LUT_BYTES: a prepared decode table
 
@@ -458,9 +459,10 @@ class DecodeBatch:
     """ep_batch_create / ep_decode_batch: decode several tensors in one launch.
 
     items: (DeviceBlob, prepared table, output tensor or None) triples; the outputs are allocated
-    here when None.  The blobs, tables and outputs are kept alive with the handle."""
+    here when None.  The blobs, tables and outputs are kept alive with the handle.  num_ctas:
+    the SMs the launch uses (ep_batch_create_on), None for all of them."""
 
-    def __init__(self, items, out_dtype: int = BF16):
+    def __init__(self, items, out_dtype: int = BF16, num_ctas=None):
         import torch
 
         self.out_dtype = out_dtype
@@ -474,7 +476,10 @@ class DecodeBatch:
                                 db.row_scales.data_ptr(), lut.data_ptr(), db.rows, db.cols, db.ntiles, db.V, db.b,
                                 out.data_ptr())
         h = C.c_void_p()
-        rc = lib().ep_batch_create(arr, len(items), int(out_dtype), C.byref(h))
+        if num_ctas is None:
+            rc = lib().ep_batch_create(arr, len(items), int(out_dtype), C.byref(h))
+        else:
+            rc = lib().ep_batch_create_on(arr, len(items), int(out_dtype), int(num_ctas), C.byref(h))
         if rc:
             raise EntroPackError(rc, "ep_batch_create")
         self._h = h

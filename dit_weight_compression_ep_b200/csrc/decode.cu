@@ -1750,8 +1750,13 @@ struct ep_batch {
 extern "C" {
 
 ep_status ep_batch_create(const ep_batch_item* items, int n_items, ep_dtype out_dtype, ep_batch** out) {
+    return ep_batch_create_on(items, n_items, out_dtype, 0, out);
+}
+
+ep_status ep_batch_create_on(const ep_batch_item* items, int n_items, ep_dtype out_dtype, int num_ctas,
+                             ep_batch** out) {
     using namespace ep;
-    if (!items || !out || n_items <= 0) return EP_EINVAL;
+    if (!items || !out || n_items <= 0 || num_ctas < 0) return EP_EINVAL;
     *out = nullptr;
     if ((int)out_dtype < EP_BF16 || (int)out_dtype > EP_UINT8) return EP_EUNSUPPORTED;
     bool ragged = false;
@@ -1767,7 +1772,9 @@ ep_status ep_batch_create(const ep_batch_item* items, int n_items, ep_dtype out_
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return EP_ECUDA;
     DevState* ds = nullptr;
     if (dev_setup(dev, (int)out_dtype, ds, false) != cudaSuccess) return EP_ECUDA;
-    if (n_items > ds->num_sms) return EP_EINVAL;  // at most one tensor per SM
+    const int nctas = num_ctas == 0 ? ds->num_sms : num_ctas;
+    if (nctas > ds->num_sms) return EP_EINVAL;  // at most one CTA per SM
+    if (n_items > nctas) return EP_EINVAL;      // at most one tensor per SM
     std::vector<int64_t> T(n_items), V(n_items);
     std::vector<int> b(n_items), counts(n_items);
     for (int k = 0; k < n_items; ++k) {
@@ -1775,9 +1782,9 @@ ep_status ep_batch_create(const ep_batch_item* items, int n_items, ep_dtype out_
         V[k] = items[k].tile_vectors;
         b[k] = items[k].prob_bits;
     }
-    if (ep_batch_apportion(n_items, T.data(), V.data(), b.data(), ds->num_sms, counts.data()) != EP_OK)
+    if (ep_batch_apportion(n_items, T.data(), V.data(), b.data(), nctas, counts.data()) != EP_OK)
         return EP_EINVAL;
-    std::vector<BatchCta> plan((size_t)ds->num_sms);
+    std::vector<BatchCta> plan((size_t)nctas);
     size_t c = 0;
     for (int k = 0; k < n_items; ++k) {
         const ep_batch_item& it = items[k];
@@ -1786,7 +1793,7 @@ ep_status ep_batch_create(const ep_batch_item* items, int n_items, ep_dtype out_
         for (int r = 0; r < counts[k]; ++r, ++c) plan[c] = BatchCta{prm, (uint32_t)r, (uint32_t)counts[k]};
     }
     for (; c < plan.size(); ++c) plan[c] = BatchCta{};  // count 0: no work
-    ep_batch* h = new (std::nothrow) ep_batch{dev, ds->num_sms, out_dtype, ragged, nullptr};
+    ep_batch* h = new (std::nothrow) ep_batch{dev, nctas, out_dtype, ragged, nullptr};
     if (!h) return EP_ENOMEM;
     void* d = nullptr;
     if (cudaMalloc(&d, plan.size() * sizeof(BatchCta)) != cudaSuccess) {

@@ -370,6 +370,18 @@ typedef struct ep_batch ep_batch;
 ep_status ep_batch_create(const ep_batch_item* items, int n_items, ep_dtype out_dtype, ep_batch** out);
 
 /*
+ * ep_batch_create_on -- ep_batch_create on num_ctas SMs instead of all of them
+ * (num_ctas = 0: all; else n_items <= num_ctas <= the SM count, else
+ * EP_EINVAL).  The launch has num_ctas CTAs, so the other SMs stay free for
+ * kernels on other streams.  Each warp decodes one tile at a time as one
+ * sequential chain, so a tensor whose tiles outnumber its CTAs' warps (24 per
+ * CTA) takes more than one chain's time.  Same ownership and errors as
+ * ep_batch_create.
+ */
+ep_status ep_batch_create_on(const ep_batch_item* items, int n_items, ep_dtype out_dtype, int num_ctas,
+                             ep_batch** out);
+
+/*
  * ep_decode_batch -- one launch on `stream` (an ordinary launch, one CTA per
  * SM, with programmatic dependent launch as ep_decode_tensor_prepared's) that
  * decodes every tensor of the batch into its `out`.  Outputs, status

@@ -142,3 +142,43 @@ def test_one_tensor_per_sm_and_the_limit():
         assert_parity(to_raw(o), oracle_decode(blob, ep.BF16), ep.BF16, f"item {k}")
     with pytest.raises(ep.EntroPackError):
         ep.DecodeBatch(items + items[:1], ep.BF16)
+
+
+@pytest.mark.parametrize("num_ctas", [7, 8, 23, 100])
+def test_batch_on_part_of_the_gpu(num_ctas):
+    """ep_batch_create_on: the mixed batch on a few SMs (several tiles per warp, several tensors
+    sharing few CTAs) decodes exactly as on all of them."""
+    blobs = _mixed_blobs()
+    dbs = [ep.DeviceBlob(b) for b in blobs]
+    outs = ep.DecodeBatch([(db, ep.prepare_lut(db), None) for db in dbs], ep.BF16, num_ctas=num_ctas).run()
+    assert ep.decode_status() == 0
+    for k, (blob, o) in enumerate(zip(blobs, outs)):
+        assert_parity(to_raw(o), oracle_decode(blob, ep.BF16), ep.BF16, f"item {k} on {num_ctas} CTAs")
+
+
+def test_headline_on_one_sm_sampled_tiles():
+    """The 2,701-tile headline tensor on a single CTA: every warp walks about 113 tiles."""
+    blob = ep.encode_tensor(synth.generate(synth.headline()), 4.0)
+    db = ep.DeviceBlob(blob)
+    (o,) = ep.DecodeBatch([(db, ep.prepare_lut(db), None)], ep.BF16, num_ctas=1).run()
+    assert ep.decode_status() == 0
+    got = to_raw(o).reshape(-1)
+    per = 8 * blob.V
+    rng = np.random.default_rng(5)
+    for t in sorted(set([0, 1, 24, blob.ntiles - 1] + list(rng.choice(blob.ntiles, 6, replace=False)))):
+        lo, hi = t * per, min((t + 1) * per, blob.rows * blob.cols)
+        assert_parity(got[lo:hi], oracle_decode(blob, ep.BF16, t, t + 1), ep.BF16, f"tile {t}")
+
+
+def test_batch_cta_count_refusals():
+    import torch
+
+    nsm = torch.cuda.get_device_properties(0).multi_processor_count
+    blobs = _mixed_blobs()
+    dbs = [ep.DeviceBlob(b) for b in blobs]
+    items = [(db, ep.prepare_lut(db), None) for db in dbs]
+    for bad in (nsm + 1, len(items) - 1, -1):
+        with pytest.raises(ep.EntroPackError):
+            ep.DecodeBatch(items, ep.BF16, num_ctas=bad)
+    ep.DecodeBatch(items, ep.BF16, num_ctas=len(items)).run()  # one CTA per tensor is allowed
+    assert ep.decode_status() == 0
