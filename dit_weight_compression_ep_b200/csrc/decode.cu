@@ -699,8 +699,9 @@ struct TileCtx {
     uint32_t rows;
 };
 
-// ep_decode_gemv: a lane's partial dot products for the row its vectors are in; they go to the
-// product by atomic adds when the lane's vectors move to the next row and at the tile's end.
+// ep_decode_gemv: a lane's partial dot products for the row its vectors are in.  They go to the
+// product when the lane's vectors move on to the next row, and at the tile's end: the lanes that
+// leave the same row sum theirs across the warp first, so one atomic add a token carries them.
 // The eight BF16 activations of a vector's columns (one 16-byte load a token) come in a round
 // ahead for up to 4 tokens, so that their latency hides behind the round's nine symbol steps;
 // for 8 tokens they are loaded where they are used (held a round ahead, they would not fit in
@@ -739,26 +740,53 @@ struct GemvAcc {
             a[t] = fmaf(w[7], __uint_as_float(p.w & 0xFFFF0000u), d);
         }
     }
+    // the lane's vector of this round is in row r (act: the lane has a vector this round)
+    __device__ __forceinline__ void enter(const TileCtx& tc, uint32_t r, bool act) {
+        warp_flush(tc, act && row != r && row != 0xFFFFFFFFu);
+        if (act) row = r;
+    }
     __device__ __forceinline__ void init() {
         row = 0xFFFFFFFFu;
 #pragma unroll
         for (int t = 0; t < NT; ++t) a[t] = 0.0f;
     }
-    __device__ __forceinline__ void flush(const TileCtx& tc) {
-        if (row != 0xFFFFFFFFu) {
+    // every lane of the warp calls this; the lanes with `need` add their sums to y and reset them.
+    // Lanes that flush the same row add their sums by a butterfly first (one atomic add a token);
+    // after two such rows the rest add one by one.
+    __device__ __forceinline__ void warp_flush(const TileCtx& tc, bool need) {
+        uint32_t bal = __ballot_sync(0xFFFFFFFFu, need);
+        for (int pass = 0; pass < 2 && bal; ++pass) {
+            const int lead = __ffs(bal) - 1;
+            const uint32_t row0 = __shfl_sync(0xFFFFFFFFu, row, lead);
+            const bool grp = need && row == row0;
 #pragma unroll
-            for (int t = 0; t < NT; ++t) atomicAdd(tc.gy + (size_t)t * tc.rows + row, a[t]);
+            for (int t = 0; t < NT; ++t) {
+                float v = grp ? a[t] : 0.0f;
+#pragma unroll
+                for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xFFFFFFFFu, v, o);
+                if ((int)(threadIdx.x & 31) == lead) atomicAdd(tc.gy + (size_t)t * tc.rows + row0, v);
+                if (grp) a[t] = 0.0f;
+            }
+            if (grp) need = false;
+            bal &= ~__ballot_sync(0xFFFFFFFFu, grp);
         }
-        row = 0xFFFFFFFFu;
+        if (need) {
 #pragma unroll
-        for (int t = 0; t < NT; ++t) a[t] = 0.0f;
+            for (int t = 0; t < NT; ++t) {
+                atomicAdd(tc.gy + (size_t)t * tc.rows + row, a[t]);
+                a[t] = 0.0f;
+            }
+        }
     }
+    __device__ __forceinline__ bool pending() const { return row != 0xFFFFFFFFu; }
 };
 template <>
 struct GemvAcc<0> {
+    __device__ __forceinline__ void enter(const TileCtx&, uint32_t, bool) {}
+    __device__ __forceinline__ void warp_flush(const TileCtx&, bool) {}
     __device__ __forceinline__ void ahead(const TileCtx&, uint32_t) {}
     __device__ __forceinline__ void init() {}
-    __device__ __forceinline__ void flush(const TileCtx&) {}
+    __device__ __forceinline__ bool pending() const { return false; }
 };
 
 // One tile's bookkeeping: record, staging state and every lane's row.
@@ -857,8 +885,7 @@ __device__ __forceinline__ void renorm(uint32_t& x, uint32_t xn, bool act, uint3
 template <int DT, bool RAGGED, typename Lut, bool FULL>
 __device__ __forceinline__ void decode_round(void* out, const float sigma, const Lut& lut, const TileCtx& tc,
                                              Tile& tl, uint32_t& pb, uint32_t r, uint32_t lt, int lane,
-                                             bool& corrupt, GemvAcc<gemv_tokens<DT>()>& acc, uint32_t row_now,
-                                             uint32_t q_now) {
+                                             bool& corrupt, GemvAcc<gemv_tokens<DT>()>& acc, uint32_t q_now) {
     const uint32_t u = (r << 5) + lane;
     const bool act = FULL || u < tl.vt;
     const int64_t g = tl.v0 + u;
@@ -951,10 +978,6 @@ __device__ __forceinline__ void decode_round(void* out, const float sigma, const
         } else if constexpr (gemv_tokens<DT>() > 0) {
             // the vector's eight FP32 weights times the tokens' eight activations of its columns
             wf[7] = sigma * (__uint_as_float(yb[7]) - 6291456.0f);
-            if (row_now != acc.row) {
-                acc.flush(tc);
-                acc.row = row_now;
-            }
             acc.madd(tc, q_now, wf);
             (void)out;
         } else if constexpr (DT == EP_LATTICE_I32) {
@@ -970,6 +993,7 @@ __device__ __forceinline__ void decode_round(void* out, const float sigma, const
 }
 
 // Decode the tiles of this warp; the first one was begun in the prologue.
+
 template <int DT, bool RAGGED, typename Lut>
 __device__ void decode_tiles(const uint16_t* tiles, const uint32_t* tix, const float* scales, void* out,
                              const Lut& lut, const TileCtx& tc, Ring& rg, Tile& tl, uint32_t first_i) {
@@ -1014,6 +1038,7 @@ __device__ void decode_tiles(const uint16_t* tiles, const uint32_t* tix, const f
                 const uint32_t p_start = pb;
                 const float sigma = sig_next;
                 const uint32_t row_now = tl.rowl, q_now = tl.ql;  // this round's row and column block
+                acc.enter(tc, row_now, FULL || (r << 5) + (uint32_t)lane < tl.vt);
                 // advance every lane's row by 32 vectors and prefetch the next round's scale
                 tl.ql += 32;
                 if (tc.nq >= 32) {
@@ -1027,8 +1052,7 @@ __device__ void decode_tiles(const uint16_t* tiles, const uint32_t* tix, const f
                     }
                 }
                 if (FULL) sig_next = ((r + 1) << 5) + lane < tl.vt ? __ldg(scales + tl.rowl) : 1.0f;
-                decode_round<DT, RAGGED, Lut, FULL>(out, sigma, lut, tc, tl, pb, r, lt, lane, corrupt, acc,
-                                                    row_now, q_now);
+                decode_round<DT, RAGGED, Lut, FULL>(out, sigma, lut, tc, tl, pb, r, lt, lane, corrupt, acc, q_now);
                 if (FULL) acc.ahead(tc, tl.ql);  // the next round's activations
                 cur += (pb - p_start) >> 1;
             };
@@ -1036,7 +1060,8 @@ __device__ void decode_tiles(const uint16_t* tiles, const uint32_t* tix, const f
             round(std::false_type{}, tl.rounds - 1);
             // tile end: every lane back at 2^15 and the cursor on the next offset
             if (!__all_sync(kFull, tl.x == kStateLow) || cur != tl.off1 - tl.base) corrupt = true;
-            acc.flush(tc);
+            acc.warp_flush(tc, acc.pending());
+            acc.init();
         }
         // drain this tile's copies before the ring is reused
         while (rg.waited < rg.seq && !rg.timed_out) ring_wait_one(rg);
