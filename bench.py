@@ -513,10 +513,22 @@ def cpu_baseline(blob, seconds: float = 10.0):
         if time.time() - t0 >= seconds:
             break
     dt = time.time() - t0
+    # the same decoder on one thread, over a quarter of the time budget
+    w1, p1 = 0, 0
+    t1 = time.time()
+    while True:
+        w1 += _oracle_threads(blob, ranges[:1], 1, oracle.BF16)
+        p1 += 1
+        if time.time() - t1 >= seconds / 4:
+            break
+    dt1 = time.time() - t1
     return {"value": round(weights / dt / 1e9, 5), "unit": UNIT, "cores": cores, "kind": "oracle",
             "sample": f"{passes} pass(es) over tiles 0..{ranges[min(2 * cores, len(ranges)) - 1][1]} of the "
                       f"{blob.ntiles}-tile stream ({weights / passes / 1e6:.1f} M weights per pass), "
-                      f"{cores} threads, {dt:.1f} s"}
+                      f"{cores} threads, {dt:.1f} s",
+            "single_thread": {"value": round(w1 / dt1 / 1e9, 5), "unit": UNIT,
+                              "sample": f"{p1} pass(es) over tiles {ranges[0][0]}..{ranges[0][1]}, one thread, "
+                                        f"{dt1:.1f} s"}}
 
 
 def run_reference(args, world: int = 1):
