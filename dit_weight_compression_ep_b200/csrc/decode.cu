@@ -1144,6 +1144,14 @@ __device__ __forceinline__ void run_decode(const Params& p, const Geo& g, uint32
 
 // The decode of one tensor by G CTAs, this one of rank cta (the tensor's tiles cta + i G).
 // BATCH: a batch launch, always with a prepared table.
+// This CTA's share of zeroing n floats (y 16-byte aligned): 16-byte stores, then the tail
+__device__ __forceinline__ void zero_share(float* y, size_t n, uint32_t cta, uint32_t G) {
+    const size_t n4 = n >> 2, step = (size_t)G * kThreads;
+    for (size_t i = (size_t)cta * kThreads + threadIdx.x; i < n4; i += step)
+        reinterpret_cast<float4*>(y)[i] = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+    if (cta == 0 && threadIdx.x < (n & 3u)) y[(n4 << 2) + threadIdx.x] = 0.0f;
+}
+
 template <int DT, bool RAGGED, bool BATCH>
 __device__ __forceinline__ void decode_body(const Params& p, const uint32_t cta, const uint32_t G) {
     extern __shared__ __align__(1024) uint8_t smem[];
@@ -1152,6 +1160,12 @@ __device__ __forceinline__ void decode_body(const Params& p, const uint32_t cta,
     uint32_t* s_A = reinterpret_cast<uint32_t*>(smem + kOffDesc + 128);
     uint32_t* s_off = reinterpret_cast<uint32_t*>(smem + kOffDesc + 256);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    // ep_decode_gemv with the per-call table: the product starts at zero, and the grid barrier
+    // of the table build orders these stores before every CTA's first atomic add (stores issued
+    // here, before the prologue's values fill the registers)
+    if constexpr (gemv_tokens<DT>() > 0) {
+        if (!p.prepared) zero_share(p.gy, (size_t)gemv_tokens<DT>() * (size_t)p.rows, cta, G);
+    }
 
     // ---- prologue: header, descriptors, barriers, the first chunks of every warp's first tile
     Geo g;
@@ -1723,9 +1737,10 @@ ep_status ep_decode_gemv(void* stream, const uint16_t* tiles, const uint32_t* ti
         }
     }
     cudaStream_t st = static_cast<cudaStream_t>(stream);
-    // the product accumulates by atomic adds: it starts at zero
-    if (cudaMemsetAsync(y, 0, (size_t)ntok * (size_t)rows * sizeof(float), st) != cudaSuccess) return EP_ECUDA;
     if (lut) {
+        // the product accumulates by atomic adds: it starts at zero (with the per-call table the
+        // kernel zeroes it before its grid barrier)
+        if (cudaMemsetAsync(y, 0, (size_t)ntok * (size_t)rows * sizeof(float), st) != cudaSuccess) return EP_ECUDA;
         const Params prm{tiles, tile_index, freq_tables, row_scales, y,
                          const_cast<uint8_t*>(static_cast<const uint8_t*>(lut)), rows, cols, 1u, 1u,
                          static_cast<const uint16_t*>(x), y};

@@ -312,10 +312,12 @@ ep_status ep_decode_tensor_prepared(void* stream, const uint16_t* tiles, const u
  *                   is built per call in the workspace, as ep_decode_tensor).
  *   x               device, BF16 bits [ntok, cols] row-major, 16-byte aligned; read only.
  *   ntok            1, 2, 4 or 8 (else EP_EUNSUPPORTED).
- *   y               device, float32 [ntok, rows] row-major, 16-byte aligned; overwritten: the
- *                   call zeroes it on the stream, then adds the partial sums of each row by
- *                   atomic adds, so the order of the float32 additions is unspecified (the
- *                   result lies within the float32 dot-product bound of the exact product).
+ *   y               device, float32 [ntok, rows] row-major, 16-byte aligned; overwritten: it
+ *                   is zeroed first (with a prepared table by a memset on the stream, else by
+ *                   the kernel before its grid barrier), then the partial sums of each row are
+ *                   added by atomic adds, so the order of the float32 additions is unspecified
+ *                   (the result lies within the float32 dot-product bound of the exact
+ *                   product).  After a stream error its contents are unspecified.
  * Asynchronous on `stream`; argument errors as ep_decode_tensor; stream errors raise the
  * status word that ep_decode_status reads.
  */
