@@ -492,12 +492,17 @@ struct Out<EP_FP8_E4M3> {
         reinterpret_cast<uint2*>(out)[g] = v;
     }
 };
+// INT8 / UINT8: the clamped value plus 1.5 * 2^23 (+ 128 for UINT8) lands in [2^23, 2^24), where
+// the float spacing is 1, so the addition rounds to the nearest integer, ties to even, and the
+// low byte of the sum's bits is the integer's byte.  This keeps the conversion on the FMA pipe.
+__device__ __forceinline__ int round_to_byte(float v, float magic) { return __float_as_int(v + magic); }
+
 template <>
 struct Out<EP_INT8> {
     __device__ static void store(void* out, int64_t g, const float w[8]) {
         int q[8];
 #pragma unroll
-        for (int i = 0; i < 8; ++i) q[i] = __float2int_rn(fminf(fmaxf(w[i], -127.0f), 127.0f));
+        for (int i = 0; i < 8; ++i) q[i] = round_to_byte(fminf(fmaxf(w[i], -127.0f), 127.0f), 12582912.0f);
         uint2 v;
         v.x = __byte_perm(__byte_perm(q[0], q[1], 0x0040), __byte_perm(q[2], q[3], 0x0040), 0x5410);
         v.y = __byte_perm(__byte_perm(q[4], q[5], 0x0040), __byte_perm(q[6], q[7], 0x0040), 0x5410);
@@ -509,7 +514,7 @@ struct Out<EP_UINT8> {
     __device__ static void store(void* out, int64_t g, const float w[8]) {
         int q[8];
 #pragma unroll
-        for (int i = 0; i < 8; ++i) q[i] = __float2int_rn(fminf(fmaxf(w[i], -128.0f), 127.0f)) + 128;
+        for (int i = 0; i < 8; ++i) q[i] = round_to_byte(fminf(fmaxf(w[i], -128.0f), 127.0f), 12583040.0f);
         uint2 v;
         v.x = __byte_perm(__byte_perm(q[0], q[1], 0x0040), __byte_perm(q[2], q[3], 0x0040), 0x5410);
         v.y = __byte_perm(__byte_perm(q[4], q[5], 0x0040), __byte_perm(q[6], q[7], 0x0040), 0x5410);
