@@ -356,12 +356,30 @@ def _torch_dtype(dt: int):
             FP32: torch.float32, LATTICE_I32: torch.int32, UINT8: torch.uint8}[dt]
 
 
+def _output(db: DeviceBlob, out_dtype: int, out, shape=None):
+    """`out`, or a new tensor, for a decode of db into out_dtype; a given buffer must be a
+    contiguous CUDA tensor of the output dtype on db's device, large enough for the result (the
+    C ABI takes a bare pointer and cannot check its extent)."""
+    import torch
+
+    shape = shape or (db.rows, db.cols)
+    tdt = _torch_dtype(out_dtype) if isinstance(out_dtype, int) else out_dtype
+    if out is None:
+        return torch.empty(shape, dtype=tdt, device=db.payload.device)
+    n = 1
+    for d in shape:
+        n *= int(d)
+    if not (isinstance(out, torch.Tensor) and out.is_cuda and out.dtype == tdt and out.is_contiguous()
+            and out.device == db.payload.device and out.numel() >= n):
+        raise ValueError(f"out must be a contiguous {tdt} CUDA tensor on {db.payload.device} with at least {n} elements")
+    return out
+
+
 def decode_tensor(db: DeviceBlob, out_dtype: int = BF16, out=None, stream=None):
     """Launch ep_decode_tensor on `stream` (default: torch's current stream); returns `out`."""
     import torch
 
-    if out is None:
-        out = torch.empty((db.rows, db.cols), dtype=_torch_dtype(out_dtype), device=db.payload.device)
+    out = _output(db, out_dtype, out)
     st = stream if stream is not None else torch.cuda.current_stream(db.payload.device)
     rc = lib().ep_decode_tensor(C.c_void_p(st.cuda_stream), db.payload.data_ptr(), db.tile_index.data_ptr(),
                                 db.freq_tables.data_ptr(), db.row_scales.data_ptr(), db.rows, db.cols,
@@ -376,8 +394,7 @@ def decode_tensor_noalloc(db: DeviceBlob, out_dtype: int = BF16, out=None, strea
     (no device allocation by the library); calls that overlap on the GPU must be ordered by the caller."""
     import torch
 
-    if out is None:
-        out = torch.empty((db.rows, db.cols), dtype=_torch_dtype(out_dtype), device=db.payload.device)
+    out = _output(db, out_dtype, out)
     st = stream if stream is not None else torch.cuda.current_stream(db.payload.device)
     rc = lib().ep_decode_tensor_noalloc(C.c_void_p(st.cuda_stream), db.payload.data_ptr(), db.tile_index.data_ptr(),
                                         db.freq_tables.data_ptr(), db.row_scales.data_ptr(), db.rows, db.cols,
@@ -387,6 +404,14 @@ def decode_tensor_noalloc(db: DeviceBlob, out_dtype: int = BF16, out=None, strea
     return out
 
 
+def _check_lut(db: DeviceBlob, lut):
+    """A prepared-table buffer: a contiguous CUDA tensor on db's device (its size the C ABI checks)."""
+    import torch
+
+    if not (isinstance(lut, torch.Tensor) and lut.is_cuda and lut.is_contiguous() and lut.device == db.payload.device):
+        raise ValueError(f"the table buffer must be a contiguous CUDA tensor on {db.payload.device}")
+
+
 def prepare_lut(db: DeviceBlob, lut=None, stream=None):
     """ep_decode_prepare: build the tensor's decode lookup table once into a LUT_BYTES uint8
     device buffer (allocated here when `lut` is None); returns the buffer."""
@@ -394,6 +419,7 @@ def prepare_lut(db: DeviceBlob, lut=None, stream=None):
 
     if lut is None:
         lut = torch.empty(LUT_BYTES, dtype=torch.uint8, device=db.payload.device)
+    _check_lut(db, lut)
     st = stream if stream is not None else torch.cuda.current_stream(db.payload.device)
     rc = lib().ep_decode_prepare(C.c_void_p(st.cuda_stream), db.freq_tables.data_ptr(), db.rows, db.cols,
                                  lut.data_ptr(), lut.numel() * lut.element_size())
@@ -406,8 +432,8 @@ def decode_tensor_prepared(db: DeviceBlob, lut, out_dtype: int = BF16, out=None,
     """ep_decode_tensor_prepared: the decode with a table prepare_lut built from this tensor."""
     import torch
 
-    if out is None:
-        out = torch.empty((db.rows, db.cols), dtype=_torch_dtype(out_dtype), device=db.payload.device)
+    _check_lut(db, lut)
+    out = _output(db, out_dtype, out)
     st = stream if stream is not None else torch.cuda.current_stream(db.payload.device)
     rc = lib().ep_decode_tensor_prepared(C.c_void_p(st.cuda_stream), db.payload.data_ptr(),
                                          db.tile_index.data_ptr(), db.freq_tables.data_ptr(),
@@ -428,11 +454,12 @@ def decode_gemv(db: DeviceBlob, x, lut=None, y=None, stream=None):
     import torch
 
     if not (isinstance(x, torch.Tensor) and x.is_cuda and x.dtype == torch.bfloat16 and x.dim() == 2
-            and x.shape[1] == db.cols):
-        raise ValueError("x must be a bfloat16 CUDA tensor [tokens, cols]")
+            and x.shape[1] == db.cols and x.device == db.payload.device):
+        raise ValueError("x must be a bfloat16 CUDA tensor [tokens, cols] on the blob's device")
     x = x.contiguous()
-    if y is None:
-        y = torch.empty((x.shape[0], db.rows), dtype=torch.float32, device=x.device)
+    if lut is not None:
+        _check_lut(db, lut)
+    y = _output(db, torch.float32, y, (x.shape[0], db.rows))
     st = stream if stream is not None else torch.cuda.current_stream(db.payload.device)
     rc = lib().ep_decode_gemv(C.c_void_p(st.cuda_stream), db.payload.data_ptr(), db.tile_index.data_ptr(),
                               db.freq_tables.data_ptr(), db.row_scales.data_ptr(),
@@ -469,8 +496,8 @@ class DecodeBatch:
         self.items = []
         arr = (_BatchItem * len(items))()
         for k, (db, lut, out) in enumerate(items):
-            if out is None:
-                out = torch.empty((db.rows, db.cols), dtype=_torch_dtype(out_dtype), device=db.payload.device)
+            _check_lut(db, lut)
+            out = _output(db, out_dtype, out)
             self.items.append((db, lut, out))
             arr[k] = _BatchItem(db.payload.data_ptr(), db.tile_index.data_ptr(), db.freq_tables.data_ptr(),
                                 db.row_scales.data_ptr(), lut.data_ptr(), db.rows, db.cols, db.ntiles, db.V, db.b,

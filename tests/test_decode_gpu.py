@@ -383,3 +383,35 @@ def test_dit_stack_layers_sampled():
         W = synth.generate(synth.dit_stack_layer(blk, kind))
         blob = ep.encode_tensor(W, alloc[(blk, kind)])
         _full_check(blob, [ep.BF16], f"dit {kind}", sample_tiles=16)
+
+
+def test_binding_refuses_outputs_it_cannot_fill():
+    """The C ABI takes bare output pointers; the binding checks a given buffer's device, dtype,
+    layout and extent before passing it on (no launch happens on a refusal)."""
+    import torch
+
+    blob = ep.encode_tensor(synth.generate(synth.small_fp32(seed=3)), 4.0)
+    db = ep.DeviceBlob(blob)
+    lut = ep.prepare_lut(db)
+    small = torch.empty((blob.rows, blob.cols - 8), dtype=torch.bfloat16, device="cuda")
+    host = torch.empty((blob.rows, blob.cols), dtype=torch.bfloat16)
+    wrong = torch.empty((blob.rows, blob.cols), dtype=torch.float16, device="cuda")
+    strided = torch.empty((blob.cols, blob.rows), dtype=torch.bfloat16, device="cuda").t()
+    for out in (small, host, wrong, strided):
+        with pytest.raises(ValueError):
+            ep.decode_tensor(db, ep.BF16, out=out)
+        with pytest.raises(ValueError):
+            ep.decode_tensor_prepared(db, lut, ep.BF16, out=out)
+        with pytest.raises(ValueError):
+            ep.decode_tensor_noalloc(db, ep.BF16, out=out)
+    with pytest.raises(ValueError):
+        ep.decode_tensor_prepared(db, lut.cpu(), ep.BF16)
+    x = torch.zeros((2, blob.cols), dtype=torch.bfloat16, device="cuda")
+    with pytest.raises(ValueError):
+        ep.decode_gemv(db, x, y=torch.empty((1, blob.rows), device="cuda"))
+    assert ep.decode_status() == 0
+    # a larger contiguous buffer of the right dtype is accepted (the result fills its head)
+    big = torch.empty((blob.rows + 3, blob.cols), dtype=torch.bfloat16, device="cuda")
+    ep.decode_tensor(db, ep.BF16, out=big)
+    assert ep.decode_status() == 0
+    assert np.array_equal(to_raw(big).reshape(-1)[: blob.rows * blob.cols], oracle_decode(blob, ep.BF16))
