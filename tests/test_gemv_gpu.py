@@ -132,3 +132,22 @@ def test_compressed_linear_matvec_with_bias():
     assert np.all(np.abs(y.cpu().numpy().astype(np.float64) - want) <= tol)
     with pytest.raises(ValueError):
         lin.matvec(_x(3, blob.cols, 1))
+
+
+@pytest.mark.parametrize("seed", range(6))
+def test_random_shapes_rates_and_token_counts(seed):
+    """Seeded random widths (multiples of 8), heights, rates, tile sizes and token counts, per-call
+    and prepared tables, against the oracle's product."""
+    rng = np.random.default_rng(900 + seed)
+    rows, cols = int(rng.integers(1, 400)), 8 * int(rng.integers(1, 300))
+    bpp = float(rng.choice([2.3, 3.0, 4.0, 5.0, 6.0, 8.0]))
+    V = int(rng.choice([32, 33, 100, 455, 910]))
+    W = (rng.standard_t(6, (rows, cols)) * 0.02 * np.exp(rng.normal(0, 0.3, (rows, 1)))).astype(np.float32)
+    blob = ep.encode_tensor(W, bpp, tile_vectors=V)
+    db = ep.DeviceBlob(blob)
+    ntok = int(rng.choice(ep.GEMV_TOKENS))
+    x = _x(ntok, cols, 1000 + seed)
+    lut = ep.prepare_lut(db) if seed % 2 else None
+    y = ep.decode_gemv(db, x, lut=lut)
+    assert ep.decode_status() == 0
+    _check(blob, x, y)
