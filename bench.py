@@ -5,6 +5,7 @@
     python bench.py --linear     (decode-then-GEMM against a resident weight, one GPU)
     python bench.py --gemv       (the fused decode-GEMV on 1 to 8 tokens, one GPU)
     python bench.py --split      (the decode on part of the GPU beside the GEMM, one GPU)
+    python bench.py --knee       (cycles per step against tiles per warp scheduler, one GPU)
 
 One step = one ep_decode_tensor call: the whole hot path (tile setup, table
 staging, payload staging, rANS decode, lattice reconstruction, row rescale,
@@ -1253,6 +1254,63 @@ def run_chain(args):
                       "headline_eager_us": round(head, 2)}), flush=True)
 
 
+def run_knee(args):
+    """Cycles per symbol step against the number of tiles each warp scheduler holds: for k = 1 ..
+    6 (24 warps a CTA: 6 per sub-partition), tensors of exactly 4 k tiles per SM (k warps on each
+    of its four sub-partitions, one tile each) at three tile sizes; the slope of time over steps per tile is the time per step with k
+    chains interleaved on a sub-partition.  Against k x (warp instructions per step), it shows
+    where the decode turns from chain-bound to issue-bound.  Eager launches, 4 rotating outputs,
+    the SM clock taken as 1,965 MHz (the bench line records the clock it saw).  Prints JSON lines
+    and a markdown table."""
+    import numpy as np
+    import torch
+
+    import dit_weight_compression_ep_b200 as ep
+    from dit_weight_compression_ep_b200 import build
+
+    build.build()
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    rng = np.random.default_rng(0)
+
+    def timed(db, outs, n=20):
+        for i in range(4):
+            ep.decode_tensor_prepared(db, lut, ep.BF16, out=outs[i % len(outs)])
+        torch.cuda.synchronize()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        for i in range(n):
+            ep.decode_tensor_prepared(db, lut, ep.BF16, out=outs[i % len(outs)])
+        b.record()
+        torch.cuda.synchronize()
+        return a.elapsed_time(b) / n * 1e3
+
+    rows_out = []
+    for k in (1, 2, 3, 4, 5, 6):
+        pts = []
+        for V in (640, 1280, 2560):
+            tiles = 4 * k * sms
+            W = (rng.standard_t(6, (tiles * V // 128, 1024)) * 0.02).astype(np.float32)
+            blob = ep.encode_tensor(W, TARGET, tile_vectors=V, prob_bits=11)
+            assert blob.ntiles == tiles
+            db = ep.DeviceBlob(blob)
+            lut = ep.prepare_lut(db)
+            outs = [torch.empty((blob.rows, blob.cols), dtype=torch.bfloat16, device="cuda") for _ in range(4)]
+            pts.append((9 * ((V + 31) // 32), timed(db, outs)))
+        A = np.array([[1.0, st] for st, _ in pts])
+        (fixed, per), *_ = np.linalg.lstsq(A, np.array([u for _, u in pts]), rcond=None)
+        r = {"tiles_per_sub_partition": k, "cycles_per_step": round(float(per) * 1965, 1),
+             "fixed_us": round(float(fixed), 2), "points_steps_us": [(st, round(u, 2)) for st, u in pts]}
+        rows_out.append(r)
+        print(json.dumps(r), flush=True)
+        if ep.decode_status() != 0:
+            raise RuntimeError("decode reported a corrupt stream")
+    print("\n| tiles per sub-partition | cycles per symbol step | cycles per step per tile | fixed cost (µs) |")
+    print("|---|---|---|---|")
+    for r in rows_out:
+        print(f"| {r['tiles_per_sub_partition']} | {r['cycles_per_step']} | "
+              f"{r['cycles_per_step'] / r['tiles_per_sub_partition']:.1f} | {r['fixed_us']} |")
+
+
 def run_latency(args):
     """Latencies of the operations on the decode step's dependent chain on this GPU: one warp,
     dependent chains timed with clock64 (csrc/latency_probe.cu).  Prints a table and one JSON
@@ -1293,6 +1351,7 @@ def main():
     ap.add_argument("--dit", action="store_true", help="the whole DiT stack: per layer, prepared, block batches")
     ap.add_argument("--encode", action="store_true", help="conversion speed: CPU packer and GPU encoder")
     ap.add_argument("--latency", action="store_true", help="latencies of the decode step's operations (one GPU)")
+    ap.add_argument("--knee", action="store_true", help="cycles per step against tiles per sub-partition (one GPU)")
     ap.add_argument("--chain", action="store_true", help="decode chain latency and fixed cost per call (one GPU)")
     ap.add_argument("--workload", choices=["headline", *OTHER_WORKLOADS], default="headline",
                     help="time another workload with the default protocol (a measurement, not the benchmark)")
@@ -1301,7 +1360,8 @@ def main():
         ap.error("--warmup must be at least 3")
     if args.gpus < 1:
         ap.error("--gpus must be at least 1")
-    one_gpu_mode = args.sweep or args.linear or args.split or args.gemv or args.dit or args.encode or args.latency or args.chain
+    one_gpu_mode = (args.sweep or args.linear or args.split or args.gemv or args.dit or args.encode or args.latency
+                    or args.chain or args.knee)
     if args.gpus > 1 and "WORLD_SIZE" not in os.environ and not one_gpu_mode:
         # no launcher: start the N ranks here (one process per GPU) and pass on their status
         sys.exit(relaunch(args.gpus, os.path.abspath(__file__), sys.argv[1:]).returncode)
@@ -1334,6 +1394,9 @@ def main():
         return
     if args.chain:
         run_chain(args)
+        return
+    if args.knee:
+        run_knee(args)
         return
     if args.impl == "reference":
         if args.workload != "headline":
