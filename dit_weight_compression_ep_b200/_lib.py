@@ -448,7 +448,7 @@ GEMV_TOKENS = (1, 2, 4, 8)
 
 
 def decode_gemv(db: DeviceBlob, x, lut=None, y=None, stream=None):
-    """ep_decode_gemv: y = x W^T with W the tensor's decoded float32 weight, computed inside the
+    """ep_decode_gemv: y = x W^T with W the tensor's decoded weight in BF16, computed inside the
     decode (x: bfloat16 CUDA tensor [ntok, cols], ntok in GEMV_TOKENS; lut: a prepare_lut table or
     None).  Returns y, float32 [ntok, rows]."""
     import torch

@@ -727,22 +727,37 @@ struct GemvAcc {
             for (int t = 0; t < NT; ++t) xv[t] = xload(tc, q, t);
         }
     }
-    // a[t] += <w, x_t> over the vector's eight columns (block q); BF16 widens to FP32 exactly
+    // d + x0 w0 + x1 w1 for a pair of BF16 activations and a pair of BF16 weights (low halves
+    // first): FP32 multiply-adds of BF16 operands, whose products are exact in FP32
+    __device__ __forceinline__ static float fma_pair(uint32_t xp, uint32_t wp, float d) {
+        asm("{\n\t.reg .b16 x0, x1, w0, w1;\n\t"
+            "mov.b32 {x0, x1}, %1;\n\t"
+            "mov.b32 {w0, w1}, %2;\n\t"
+            "fma.rn.f32.bf16 %0, x0, w0, %0;\n\t"
+            "fma.rn.f32.bf16 %0, x1, w1, %0;\n\t}"
+            : "+f"(d)
+            : "r"(xp), "r"(wp));
+        return d;
+    }
+    // a[t] += <w, x_t> over the vector's eight columns (block q), w the weights rounded to BF16
+    // (the values the BF16 output holds); the activations stay packed
     __device__ __forceinline__ void madd(const TileCtx& tc, uint32_t q, const float* w) {
+        uint32_t wb[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const __nv_bfloat162 h = __floats2bfloat162_rn(w[2 * i], w[2 * i + 1]);
+            wb[i] = *reinterpret_cast<const uint32_t*>(&h);
+        }
 #pragma unroll
         for (int t = 0; t < NT; ++t) {
             uint4 p;
             if constexpr (kAhead) p = xv[t];
             else p = xload(tc, q, t);
             float d = a[t];
-            d = fmaf(w[0], __uint_as_float(p.x << 16), d);
-            d = fmaf(w[1], __uint_as_float(p.x & 0xFFFF0000u), d);
-            d = fmaf(w[2], __uint_as_float(p.y << 16), d);
-            d = fmaf(w[3], __uint_as_float(p.y & 0xFFFF0000u), d);
-            d = fmaf(w[4], __uint_as_float(p.z << 16), d);
-            d = fmaf(w[5], __uint_as_float(p.z & 0xFFFF0000u), d);
-            d = fmaf(w[6], __uint_as_float(p.w << 16), d);
-            a[t] = fmaf(w[7], __uint_as_float(p.w & 0xFFFF0000u), d);
+            d = fma_pair(p.x, wb[0], d);
+            d = fma_pair(p.y, wb[1], d);
+            d = fma_pair(p.z, wb[2], d);
+            a[t] = fma_pair(p.w, wb[3], d);
         }
     }
     // the lane's vector of this round is in row r (act: the lane has a vector this round)
@@ -981,7 +996,7 @@ __device__ __forceinline__ void decode_round(void* out, const float sigma, const
                     if (k < n) put_elem<DT>(out, e0 + k, wf[k]);
             }
         } else if constexpr (gemv_tokens<DT>() > 0) {
-            // the vector's eight FP32 weights times the tokens' eight activations of its columns
+            // the vector's eight weights times the tokens' eight activations of its columns
             wf[7] = sigma * (__uint_as_float(yb[7]) - 6291456.0f);
             acc.madd(tc, q_now, wf);
             (void)out;

@@ -12,9 +12,10 @@ prepared once, when the layer is built) and multiplies with the library GEMM thr
 
 Layers that run one after another can share one scratch buffer (pass the same tensor).
 
-For a few tokens, `matvec` multiplies inside the decode instead (ep_decode_gemv): the FP32
-weights go straight into FP32 multiply-adds with the BF16 activations and are never written;
-on B200 that is the faster route up to 2 tokens and even at 4."""
+For a few tokens, `matvec` multiplies inside the decode instead (ep_decode_gemv): the weights,
+rounded to BF16 as the bf16 route's are, go straight into float32 multiply-adds with the BF16
+activations and are never written; on B200 that is the faster route up to 2 tokens and even
+at 4."""
 from __future__ import annotations
 
 from ._lib import (BF16, FP8_E4M3, GEMV_TOKENS, INT8, DecodeBatch, DeviceBlob, _torch_dtype, decode_gemv,
@@ -76,8 +77,9 @@ class CompressedLinear:
 
     def matvec(self, x, out=None):
         """y = x W^T (+ bias) with the product taken inside the decode (ep_decode_gemv): x bf16
-        [tokens, in_features] with tokens in GEMV_TOKENS, W the decoded FP32 weight (whatever the
-        route), FP32 accumulation.  Returns float32 [tokens, out_features] (into `out` if given)."""
+        [tokens, in_features] with tokens in GEMV_TOKENS, W the decoded weight in BF16 (whatever
+        the route), float32 accumulation.  Returns float32 [tokens, out_features] (into `out` if
+        given)."""
         if x.dim() != 2 or x.shape[0] not in GEMV_TOKENS:
             raise ValueError(f"matvec takes {GEMV_TOKENS} tokens")
         y = decode_gemv(self.weight, x, lut=self.lut, y=out)

@@ -301,11 +301,12 @@ ep_status ep_decode_tensor_prepared(void* stream, const uint16_t* tiles, const u
 /*
  * ep_decode_gemv -- a linear layer on a few tokens with the weight decoded inside the product
  * (the on-demand reconstruction of paper §4.3 and Fig. 5, for the decode-bound case of
- * small token counts): y = x W^T, where W [rows, cols] is the tensor's decoded FP32 weight
- * (sigma_r * y_rc, the values ep_decode_tensor writes for EP_FP32) and x holds BF16
- * activations, widened exactly to FP32.  Every lane multiplies the eight weights it has just
- * reconstructed by the tokens' eight activations of those columns with FP32 multiply-adds
- * and accumulates per row; the weight is never written to memory.
+ * small token counts): y = x W^T, where W [rows, cols] is the tensor's decoded weight in
+ * BF16 (the values ep_decode_tensor writes for EP_BF16) and x holds BF16 activations: the
+ * numerics of a BF16 GEMM (exact products, float32 accumulation).  Every lane rounds the
+ * eight weights it has just reconstructed to BF16 and multiplies them by the tokens' eight
+ * activations of those columns with float32 multiply-adds, accumulating per row; the weight
+ * is never written to memory.
  *   tiles .. cols   as ep_decode_tensor (cols must be a multiple of 8: else EP_EUNSUPPORTED).
  *   lut, lut_bytes  a table ep_decode_prepare built for this tensor (then the call uses no
  *                   workspace and launches as ep_decode_tensor_prepared), or NULL (the table

@@ -1,7 +1,7 @@
 """ep_decode_gemv: a linear layer on a few tokens whose weight is decoded inside the product
 (EntroPack paper §4.3 and Fig. 5: the weight is reconstructed on demand for the matmul).
 
-The reference is the oracle's float64 product of its own float32 decode of the weight
+The reference is the oracle's float64 product of its own BF16 decode of the weight
 (`oracle.linear`) with the BF16 activations widened exactly, and the tolerance is the oracle's
 float32-accumulation bound (`oracle.linear_tolerance`, gamma_K sum|x w|: any order of float32
 additions, the atomic adds included) with no output rounding beyond float32.  Cases: every token count (1, 2, 4, 8), the
@@ -38,12 +38,18 @@ def _x(ntok, cols, seed):
     return (torch.randn(ntok, cols, generator=g) * 0.5).to(torch.bfloat16).cuda()
 
 
+def _bf16_weights(blob, t0=0, t1=None):
+    """The oracle's BF16 decode (written from the format definition), widened to float64."""
+    bits = np.asarray(oracle_decode(blob, ep.BF16, t0, t1), np.uint16).astype(np.uint32) << 16
+    return bits.view(np.float32).astype(np.float64)
+
+
 def _check(blob, x, y, rows_sel=None):
     """y against the oracle's product on the whole matrix, or on the rows rows_sel."""
     xs = x.cpu().float().numpy().astype(np.float64)  # BF16 widens to float64 exactly
     got = y.cpu().numpy().astype(np.float64)
     if rows_sel is None:
-        W = oracle_decode(blob, ep.FP32).reshape(blob.rows, blob.cols).astype(np.float64)
+        W = _bf16_weights(blob).reshape(blob.rows, blob.cols)
         want, tol = oracle.linear(W, xs), oracle.linear_tolerance(W, xs, 0.0)
         bad = np.abs(got - want) > tol
         assert not bad.any(), f"{bad.sum()} of {bad.size} outside the bound; worst {np.abs(got - want)[bad].max()}"
@@ -52,8 +58,8 @@ def _check(blob, x, y, rows_sel=None):
     for r in rows_sel:
         e0, e1 = r * blob.cols, (r + 1) * blob.cols
         t0, t1 = e0 // per, (e1 - 1) // per + 1
-        flat = oracle_decode(blob, ep.FP32, t0, t1)
-        w = flat[e0 - t0 * per:e1 - t0 * per].astype(np.float64)[None, :]
+        flat = _bf16_weights(blob, t0, t1)
+        w = flat[e0 - t0 * per:e1 - t0 * per][None, :]
         want, tol = oracle.linear(w, xs), oracle.linear_tolerance(w, xs, 0.0)
         assert np.all(np.abs(got[:, [r]] - want) <= tol), f"row {r}"
 
@@ -123,7 +129,7 @@ def test_compressed_linear_matvec_with_bias():
     x = _x(2, blob.cols, 11)
     y = lin.matvec(x)
     assert ep.decode_status() == 0
-    W = oracle_decode(blob, ep.FP32).reshape(blob.rows, blob.cols).astype(np.float64)
+    W = _bf16_weights(blob).reshape(blob.rows, blob.cols)
     xs = x.cpu().float().numpy().astype(np.float64)
     b = bias.cpu().numpy().astype(np.float64)
     want = oracle.linear(W, xs) + b
