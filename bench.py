@@ -835,8 +835,23 @@ def run_dit(args):
     if ep.decode_status(st) != 0 or not all(torch.equal(ref[k].view(torch.int16), outs[k].view(torch.int16))
                                             for k in kinds):
         raise RuntimeError("batched and prepared decodes differ")
+    # several blocks' weights in one launch (each block into its own output set): more tiles per
+    # launch, so the sub-partitions' loads even out
+    multi = {}
+    for n in (2, 3, 6):
+        sets = [outs] + [{k: torch.empty_like(o) for k, o in outs.items()} for _ in range(n - 1)]
+        groups = [blocks[i:i + n] for i in range(0, len(blocks), n)]
+        multi[n] = [ep.DecodeBatch([(streams[kb][1], streams[kb][2], sets[j][kb[0]])
+                                    for j, blk in enumerate(g) for kb in blk], ep.BF16) for g in groups]
     res = {"case": f"DiT linear stack, {nblocks} blocks x {len(kinds)} layers, per-layer rates {synth.DIT_BPP_CHOICES}",
            "weights": numel, "algorithmic_bytes": nbytes, "hbm_peak_gbs": peak, "peak_kind": peak_kind}
+    for n, gb in multi.items():
+        tmin, tmed = timed(lambda gb=gb: [b.run(stream=st) for b in gb])
+        res[f"batches_of_{n}_blocks_ms"] = [tmin, tmed]
+        res[f"batches_of_{n}_blocks_gweights_s"] = round(numel / (tmin * 1e-3) / 1e9, 1)
+        res[f"batches_of_{n}_blocks_hbm_frac"] = round(nbytes / (tmin * 1e-3) / 1e9 / peak, 4)
+        print(json.dumps({f"batches_of_{n}_blocks": [tmin, tmed]}), flush=True)
+    del multi
     for name, fn in (("per_layer_decode", per_call), ("per_layer_prepared", prepared), ("block_batches", batched),
                      ("matmuls_only_4096", matmuls_only), ("step_block_batches_then_matmuls", step_batched),
                      ("step_block_batches_pipelined", step_pipelined),
