@@ -1272,7 +1272,8 @@ def run_chain(args):
 def run_knee(args):
     """Cycles per symbol step against the number of tiles each warp scheduler holds: for k = 1 ..
     6 (24 warps a CTA: 6 per sub-partition), tensors of exactly 4 k tiles per SM (k warps on each
-    of its four sub-partitions, one tile each) at three tile sizes; the slope of time over steps per tile is the time per step with k
+    of its four sub-partitions, one tile each) at three tile sizes, with the packed b = 11 table
+    and (k = 1, 3, 6) the two-level b = 12 one; the slope of time over steps per tile is the time per step with k
     chains interleaved on a sub-partition.  Against k x (warp instructions per step), it shows
     where the decode turns from chain-bound to issue-bound.  Eager launches, 4 rotating outputs,
     the SM clock taken as 1,965 MHz (the bench line records the clock it saw).  Prints JSON lines
@@ -1300,29 +1301,29 @@ def run_knee(args):
         return a.elapsed_time(b) / n * 1e3
 
     rows_out = []
-    for k in (1, 2, 3, 4, 5, 6):
+    for b, k in [(11, k) for k in (1, 2, 3, 4, 5, 6)] + [(12, k) for k in (1, 3, 6)]:
         pts = []
         for V in (640, 1280, 2560):
             tiles = 4 * k * sms
             W = (rng.standard_t(6, (tiles * V // 128, 1024)) * 0.02).astype(np.float32)
-            blob = ep.encode_tensor(W, TARGET, tile_vectors=V, prob_bits=11)
-            assert blob.ntiles == tiles
+            blob = ep.encode_tensor(W, TARGET, tile_vectors=V, prob_bits=b)
+            assert blob.ntiles == tiles and blob.b == b
             db = ep.DeviceBlob(blob)
             lut = ep.prepare_lut(db)
             outs = [torch.empty((blob.rows, blob.cols), dtype=torch.bfloat16, device="cuda") for _ in range(4)]
             pts.append((9 * ((V + 31) // 32), timed(db, outs)))
         A = np.array([[1.0, st] for st, _ in pts])
         (fixed, per), *_ = np.linalg.lstsq(A, np.array([u for _, u in pts]), rcond=None)
-        r = {"tiles_per_sub_partition": k, "cycles_per_step": round(float(per) * 1965, 1),
+        r = {"b": b, "tiles_per_sub_partition": k, "cycles_per_step": round(float(per) * 1965, 1),
              "fixed_us": round(float(fixed), 2), "points_steps_us": [(st, round(u, 2)) for st, u in pts]}
         rows_out.append(r)
         print(json.dumps(r), flush=True)
         if ep.decode_status() != 0:
             raise RuntimeError("decode reported a corrupt stream")
-    print("\n| tiles per sub-partition | cycles per symbol step | cycles per step per tile | fixed cost (µs) |")
-    print("|---|---|---|---|")
+    print("\n| b | tiles per sub-partition | cycles per symbol step | cycles per step per tile | fixed cost (µs) |")
+    print("|---|---|---|---|---|")
     for r in rows_out:
-        print(f"| {r['tiles_per_sub_partition']} | {r['cycles_per_step']} | "
+        print(f"| {r['b']} | {r['tiles_per_sub_partition']} | {r['cycles_per_step']} | "
               f"{r['cycles_per_step'] / r['tiles_per_sub_partition']:.1f} | {r['fixed_us']} |")
 
 
