@@ -1657,9 +1657,11 @@ ep_status check_decode_args(const uint16_t* tiles, const uint32_t* tile_index, c
     if (!tiles || !tile_index || !freq_tables || !row_scales || !out) return EP_EINVAL;
     if (rows <= 0 || cols <= 0) return EP_EINVAL;
     if ((int)out_dtype < EP_BF16 || (int)out_dtype > EP_UINT8) return EP_EUNSUPPORTED;
-    // the largest tensor: fewer than 2^31 vectors of eight
+    // the largest tensor: fewer than 2^31 vectors of eight (each factor bounded first, so that
+    // the product cannot overflow)
+    if (rows >= (1ll << 31) || cols >= (1ll << 34)) return EP_EINVAL;
     const int64_t nvec = rows * ((cols + 7) / 8);
-    if (nvec >= (1ll << 31) || rows >= (1ll << 31)) return EP_EINVAL;
+    if (nvec >= (1ll << 31)) return EP_EINVAL;
     if (misaligned(tiles, 16) || misaligned(freq_tables, 16) || misaligned(tile_index, 4) ||
         misaligned(row_scales, 4) || misaligned(out, 16))
         return EP_EINVAL;

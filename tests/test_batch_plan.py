@@ -70,7 +70,10 @@ def _item(**kw):
 
 @pytest.mark.parametrize("bad", [dict(tiles=None), dict(lut=None), dict(out=None), dict(lut=0x10008),
                                  dict(tiles=0x10008), dict(out=0x10004), dict(rows=0), dict(cols=-8),
-                                 dict(ntiles=0), dict(tile_vectors=0)])
+                                 dict(ntiles=0), dict(tile_vectors=0),
+                                 dict(rows=1 << 31), dict(rows=1, cols=1 << 34),
+                                 dict(rows=1 << 20, cols=1 << 20),   # 2^37 vectors
+                                 dict(rows=1 << 40, cols=1 << 40)])  # a product that would overflow
 def test_batch_create_refuses_bad_items_on_host(bad):
     lib = ep.lib()
     arr = (ep._lib._BatchItem * 2)(_item(), _item(**bad))
