@@ -415,3 +415,22 @@ def test_binding_refuses_outputs_it_cannot_fill():
     ep.decode_tensor(db, ep.BF16, out=big)
     assert ep.decode_status() == 0
     assert np.array_equal(to_raw(big).reshape(-1)[: blob.rows * blob.cols], oracle_decode(blob, ep.BF16))
+
+
+@pytest.mark.parametrize("zero_first_column,bpp", [(False, 4.0), (False, 6.6), (True, 6.6), (True, 4.0)])
+@pytest.mark.parametrize("dt", [ep.BF16, ep.LATTICE_I32])
+def test_packed_table_field_widths(zero_first_column, bpp, dt):
+    """Both packed-entry layouts at b = 11: f in b + 1 bits (coordinate alphabets within +-256, at
+    4 bpp) and f - 1 in b bits (wider alphabets, at 6.6 bpp), each with and without a
+    single-symbol coordinate table (every vector's first coordinate zero, so coset 0's z1 table
+    holds only 0, f = 2^b).  Bit-exact against the oracle."""
+    rng = np.random.default_rng(41)
+    W = (rng.standard_t(6, (256, 1024)) * 0.02).astype(np.float32)
+    if zero_first_column:
+        W[:, ::8] = 0.0
+    blob = ep.encode_tensor(W, bpp)
+    assert blob.b == 11
+    db = ep.DeviceBlob(blob)
+    for got in (ep.decode_tensor(db, dt), ep.decode_tensor_prepared(db, ep.prepare_lut(db), dt)):
+        assert ep.decode_status() == 0
+        assert_parity(to_raw(got), oracle_decode(blob, dt), dt, f"bpp {bpp}, zeroed column {zero_first_column}")
