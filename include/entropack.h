@@ -10,7 +10,11 @@
  *                        §3.5 refit, §3.6 tiles; App. C.1, C.3), threaded;
  *   ep_decode_tensor  -- the fused GPU reconstruction (Fig. 2b; §3.6: a warp
  *                        per tile, a lane per interleaved state; App. C.3),
- *                        stream-ordered, one kernel launch per call.
+ *                        stream-ordered, one kernel launch per call;
+ * and, declared below with their own notes: the GPU encoder, the same decode
+ * without a library allocation, prepared tables, batches of tensors (on all SMs
+ * or a given number), and the product with 1 to 8 tokens taken inside the
+ * decode (ep_decode_gemv).
  *
  * Stored representation (all little-endian; the packer writes it, the decoder
  * reads it):
